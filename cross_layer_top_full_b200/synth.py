@@ -1,0 +1,218 @@
+"""Seeded synthetic inputs for the IndexCache hot path.
+
+This module only draws random numbers and stores them in the layouts the
+library reads; it holds none of the method's arithmetic, so both the CUDA
+path and the CPU oracle may use it.  Everything is drawn with
+``torch.Generator`` on the requested device from a seed derived from
+(workload seed, layer, tensor name); CPU and CUDA generators give different
+streams, so a test always moves the very tensors the GPU read to the host.
+
+Workloads (shapes and distributions; the pages give none of them, see the
+reading notes in each entry):
+
+* ``prefill_512_fp32``     1 sequence, L=512, FSSS, indexer H_I=4, d_I=32,
+  k=64; attention 8 heads sharing one K/V head, d_qk=d_v=64; float32.
+* ``prefill_8k_bf16``      1 sequence, L=8192, FSSS, H_I=64, d_I=128, k=2048;
+  MQA with 128 heads over one latent KV row of width 576 (V = its first 512
+  columns); bf16 activations.
+* ``decode_b32_t32k_bf16`` 32 sequences x 32768 cached keys, one new query
+  each, pattern FSSSFSSS; caches N(0,1)/sqrt(d) with 16 heavy-hitter
+  positions per sequence scaled x4.
+* ``chunked_prefill_64k_bf16`` 1 sequence, L=65536 in 4096-row chunks,
+  12 layers FSSFSSSSFSSS; k_I^(l) = base + 0.3 * noise^(l).
+* ``decode_b8_t200k_fp8``  8 sequences x 200000 keys, (FSSS)x12; indexer
+  operands as E4M3 codes with one float32 scale per token (absmax/448).
+"""
+from __future__ import annotations
+
+import dataclasses
+import hashlib
+import math
+from typing import Dict, Optional
+
+import torch
+
+__all__ = ["Workload", "WORKLOADS", "layer_inputs", "heavy_hitters", "fp8_per_token"]
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    L: int                  # query rows per sequence in one pass (prefill) / 1 (decode)
+    T: int                  # keys per sequence
+    q_start: int
+    H_I: int
+    d_I: int
+    k: int
+    Hq: int
+    d_qk: int
+    d_v: int
+    idx_dtype: str          # 'f32' | 'bf16' | 'e4m3'
+    attn_dtype: str         # 'f32' | 'bf16'
+    latent: bool            # K and V share one row of width d_qk (V = first d_v cols)
+    pattern: str
+    seed: int
+    w_std: float
+    qI_std: float
+    kI_std: float
+    q_std: float
+    kv_std: float
+    heavy: int = 0          # planted high-norm positions per sequence
+    heavy_gain: float = 1.0
+    chunk: int = 0          # chunked prefill: query rows per chunk (0 = one pass)
+    kI_noise: float = 0.0   # chunked prefill: per-layer key noise relative to base
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d_qk)
+
+    @property
+    def n_layers(self) -> int:
+        return len(self.pattern)
+
+    @property
+    def kv_width(self) -> int:
+        return self.d_qk
+
+
+WORKLOADS: Dict[str, Workload] = {
+    "prefill_512_fp32": Workload(
+        "prefill_512_fp32", B=1, L=512, T=512, q_start=0, H_I=4, d_I=32, k=64,
+        Hq=8, d_qk=64, d_v=64, idx_dtype="f32", attn_dtype="f32", latent=False,
+        pattern="FSSS", seed=0, w_std=1 / math.sqrt(4), qI_std=1 / math.sqrt(32),
+        kI_std=1 / math.sqrt(32), q_std=1.0, kv_std=1.0),
+    "prefill_8k_bf16": Workload(
+        "prefill_8k_bf16", B=1, L=8192, T=8192, q_start=0, H_I=64, d_I=128, k=2048,
+        Hq=128, d_qk=576, d_v=512, idx_dtype="bf16", attn_dtype="bf16", latent=True,
+        pattern="FSSS", seed=1, w_std=1 / 8, qI_std=1 / math.sqrt(128),
+        kI_std=1 / math.sqrt(128), q_std=1.0, kv_std=1.0),
+    # decode q / q_I / w follow the prefill workload (only the caches are
+    # specified for decode); KV and K_I caches are N(0,1)/sqrt(d).
+    "decode_b32_t32k_bf16": Workload(
+        "decode_b32_t32k_bf16", B=32, L=1, T=32768, q_start=32767, H_I=64, d_I=128, k=2048,
+        Hq=128, d_qk=576, d_v=512, idx_dtype="bf16", attn_dtype="bf16", latent=True,
+        pattern="FSSSFSSS", seed=2, w_std=1 / 8, qI_std=1 / math.sqrt(128),
+        kI_std=1 / math.sqrt(128), q_std=1.0, kv_std=1 / math.sqrt(576), heavy=16,
+        heavy_gain=4.0),
+    "chunked_prefill_64k_bf16": Workload(
+        "chunked_prefill_64k_bf16", B=1, L=65536, T=65536, q_start=0, H_I=64, d_I=128,
+        k=2048, Hq=128, d_qk=576, d_v=512, idx_dtype="bf16", attn_dtype="bf16",
+        latent=True, pattern="FSSFSSSSFSSS", seed=3, w_std=1 / 8,
+        qI_std=1 / math.sqrt(128), kI_std=1 / math.sqrt(128), q_std=1.0, kv_std=1.0,
+        chunk=4096, kI_noise=0.3),
+    "decode_b8_t200k_fp8": Workload(
+        "decode_b8_t200k_fp8", B=8, L=1, T=200000, q_start=199999, H_I=64, d_I=128, k=2048,
+        Hq=128, d_qk=576, d_v=512, idx_dtype="e4m3", attn_dtype="bf16", latent=True,
+        pattern="FSSS" * 12, seed=4, w_std=1 / 8, qI_std=1 / math.sqrt(128),
+        kI_std=1 / math.sqrt(128), q_std=1.0, kv_std=1 / math.sqrt(576), heavy=16,
+        heavy_gain=4.0),
+}
+
+
+def _gen(device, *key) -> torch.Generator:
+    h = hashlib.sha256(repr(key).encode()).digest()
+    g = torch.Generator(device=device)
+    g.manual_seed(int.from_bytes(h[:8], "little") & ((1 << 63) - 1))
+    return g
+
+
+def _randn(shape, std, device, *key, dtype=torch.float32) -> torch.Tensor:
+    x = torch.randn(shape, generator=_gen(device, *key), device=device, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(dtype)
+
+
+def _store_dtype(name: str) -> torch.dtype:
+    return {"f32": torch.float32, "bf16": torch.bfloat16}[name]
+
+
+def heavy_hitters(wl: Workload, device) -> Optional[torch.Tensor]:
+    """[B, heavy] int64 positions per sequence, uniform without replacement;
+    the same positions in every layer (they are properties of the sequence)."""
+    if wl.heavy == 0:
+        return None
+    rows = []
+    for b in range(wl.B):
+        g = _gen("cpu", wl.seed, "heavy", b)
+        rows.append(torch.randperm(wl.T, generator=g)[: wl.heavy])
+    return torch.stack(rows).to(device)
+
+
+def fp8_per_token(x: torch.Tensor, token_dims: int):
+    """Store ``x`` as E4M3 codes with one float32 scale per token.
+
+    The first ``token_dims`` axes index tokens; all remaining axes are that
+    token's values.  scale = absmax/448 (1 where the token is all zero);
+    codes = float8_e4m3fn(x / scale) by torch's round-to-nearest-even cast,
+    after clamping to the finite range.  Returns (uint8 codes, float32 scale).
+    """
+    flat = x.reshape(*x.shape[:token_dims], -1)
+    amax = flat.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax)).to(torch.float32)
+    y = (flat / scale.unsqueeze(-1)).clamp_(-448.0, 448.0)
+    codes = y.to(torch.float8_e4m3fn).view(torch.uint8).reshape(x.shape)
+    return codes.contiguous(), scale.contiguous()
+
+
+def _plant(x: torch.Tensor, hh: Optional[torch.Tensor], gain: float) -> torch.Tensor:
+    if hh is None:
+        return x
+    for b in range(x.shape[0]):
+        x[b, hh[b]] *= gain
+    return x
+
+
+def layer_inputs(wl: Workload, layer: int, device="cpu", *, indexer: bool = True,
+                 attention: bool = True, chunk: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """Inputs of one layer.
+
+    Keys: 'q_I' [B,L,H_I,d_I], 'w' [B,L,H_I] f32, 'k_I' [B,T,d_I]
+    (+ 'q_scale' [B,L], 'k_scale' [B,T] for e4m3), 'q' [B,L,Hq,d_qk], and
+    either 'kv' [B,T,d_qk] (latent) or 'k' [B,T,d_qk], 'v' [B,T,d_v].
+    For a chunked workload, ``chunk`` selects the query rows
+    [chunk*wl.chunk, (chunk+1)*wl.chunk) of 'q', 'q_I' and 'w'; keys cover the
+    full sequence (a call uses the causal prefix).
+    """
+    out: Dict[str, torch.Tensor] = {}
+    B, L, T = wl.B, wl.L, wl.T
+    hh = heavy_hitters(wl, device)
+    if wl.chunk:
+        c = 0 if chunk is None else chunk
+        qrows = wl.chunk
+    else:
+        c, qrows = 0, L
+    if indexer:
+        if wl.kI_noise:
+            # base shared by all layers + per-layer noise at kI_noise x base's std
+            base = _randn((B, T, wl.d_I), wl.kI_std, device, wl.seed, "kI_base")
+            noise = _randn((B, T, wl.d_I), wl.kI_std * wl.kI_noise, device, wl.seed, "kI_noise", layer)
+            kI = base + noise
+            # queries of the indexer are shared by all layers of this workload
+            qkey, wkey = ("qI_shared", c), ("w_shared", c)
+        else:
+            kI = _randn((B, T, wl.d_I), wl.kI_std, device, wl.seed, "kI", layer)
+            qkey, wkey = ("qI", layer, c), ("w", layer, c)
+        kI = _plant(kI, hh, wl.heavy_gain)
+        qI = _randn((B, qrows, wl.H_I, wl.d_I), wl.qI_std, device, wl.seed, *qkey)
+        out["w"] = _randn((B, qrows, wl.H_I), wl.w_std, device, wl.seed, *wkey)
+        if wl.idx_dtype == "e4m3":
+            out["q_I"], out["q_scale"] = fp8_per_token(qI, 2)
+            out["k_I"], out["k_scale"] = fp8_per_token(kI, 2)
+        else:
+            dt = _store_dtype(wl.idx_dtype)
+            out["q_I"] = qI.to(dt).contiguous()
+            out["k_I"] = kI.to(dt).contiguous()
+        del qI, kI
+    if attention:
+        adt = _store_dtype(wl.attn_dtype)
+        out["q"] = _randn((B, qrows, wl.Hq, wl.d_qk), wl.q_std, device, wl.seed, "q", layer, c,
+                          dtype=adt)
+        if wl.latent:
+            kv = _randn((B, T, wl.d_qk), wl.kv_std, device, wl.seed, "kv", layer)
+            out["kv"] = _plant(kv, hh, wl.heavy_gain).to(adt).contiguous()
+        else:
+            out["k"] = _randn((B, T, wl.d_qk), wl.kv_std, device, wl.seed, "k", layer, dtype=adt)
+            out["v"] = _randn((B, T, wl.d_v), wl.kv_std, device, wl.seed, "v", layer, dtype=adt)
+    return out

@@ -1,0 +1,236 @@
+/*
+ * indexcache.h -- C ABI of the IndexCache hot path on NVIDIA B200 (sm_100a).
+ *
+ * IndexCache ("IndexCache: Accelerating Sparse Attention via Cross-Layer
+ * Index Reuse", summarised on gist.science) splits a stack of DeepSeek
+ * sparse-attention (DSA) layers into F and S layers by a binary pattern:
+ *   - an F ("Full") layer runs its lightning indexer over every causal key of
+ *     every query, keeps the top-k key positions per query and stores them in
+ *     a temporary index cache;
+ *   - an S ("Shared") layer has no indexer and reuses the cached indices of
+ *     the nearest preceding F layer;
+ *   - every layer runs sparse attention over its query's selected keys only.
+ * (es page, section 2 "Arquitectura del Método"; pt page, section 2
+ * "Arquitetura"; de page, section 2 "Methodik: IndexCache".)
+ *
+ * Conventions shared by every call:
+ *   - All array arguments are DEVICE pointers unless stated otherwise.  The
+ *     caller owns every buffer; the library never allocates device memory and
+ *     keeps no per-call state on the device.
+ *   - Arrays are dense, row-major, with the layouts stated per argument.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronise, except ic_read_status.
+ *   - Argument errors are returned before anything is launched.  A failed
+ *     launch returns IC_ERR_CUDA.  Errors the kernels detect themselves (an
+ *     index outside its row's causal range, a wait that ran out of time) are
+ *     recorded as bits of a status word at the start of the workspace and
+ *     read back with ic_read_status.  No kernel traps or asserts.
+ *   - Workspace: every call takes `ws`/`ws_bytes`.  The first
+ *     IC_STATUS_BYTES bytes hold the status word; zero them once with
+ *     ic_workspace_init.  `ws` must be 256-byte aligned.  The size a call
+ *     needs is given by its *_workspace_size function.
+ *   - Causality: query row i of sequence b sits at absolute position
+ *     t = q_start + i and its candidate keys are s = 0..t (its own key
+ *     included).  A decode step is Lq = 1, q_start = T - 1.
+ */
+#ifndef INDEXCACHE_H
+#define INDEXCACHE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define IC_STATUS_BYTES 256
+
+typedef enum {
+    IC_OK = 0,
+    IC_ERR_INVALID_ARG = -1,  /* null pointer, bad size, stride or alignment        */
+    IC_ERR_PATTERN = -2,      /* pattern not of 'F'/'S', wrong length, or starts 'S' */
+    IC_ERR_UNSUPPORTED = -3,  /* dtype / shape combination not implemented          */
+    IC_ERR_WORKSPACE = -4,    /* ws too small or misaligned                         */
+    IC_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed                */
+    IC_ERR_INDEX_RANGE = -6,  /* (device) an index was outside [0, t]; row skipped   */
+    IC_ERR_TIMEOUT = -7       /* (device) a pipeline wait ran out of time            */
+} ic_status;
+
+typedef enum {
+    IC_F32 = 0,       /* IEEE float32                                   */
+    IC_BF16 = 1,      /* bfloat16                                       */
+    IC_FP8_E4M3 = 2   /* OCP E4M3 "FN" byte codes with per-token scale  */
+} ic_dtype;
+
+/* Rows of a call: B sequences, Lq query rows each starting at absolute
+ * position q_start, T keys per sequence.  Requires q_start + Lq <= T. */
+typedef struct {
+    int B;
+    int Lq;
+    int q_start;
+    int T;
+} ic_rows;
+
+/* ------------------------------------------------------------------------ */
+/* Status and workspace                                                      */
+/* ------------------------------------------------------------------------ */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* ic_status_string(ic_status st);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int ic_version(void);
+
+/* Zero the status word at the start of `ws` (asynchronous memset on stream).
+ * ws_bytes must be >= IC_STATUS_BYTES. */
+ic_status ic_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read the status word of `ws` into *device_status
+ * (host pointer; bit 0 = index out of range, bit 1 = wait timeout) and clear
+ * it.  Returns IC_OK when no bit was set, else the error of the lowest bit. */
+ic_status ic_read_status(void* ws, void* stream, int32_t* device_status);
+
+/* Number of kernels this library has launched in this process, by kind:
+ * 0 = all, 1 = indexer, 2 = top-k, 3 = attention, 4 = split-k combine.
+ * A host-side diagnostic counter (thread-safe). */
+uint64_t ic_kernel_launches(int kind);
+
+/* ------------------------------------------------------------------------ */
+/* a1  Lightning indexer scores (F layers)                                   */
+/* ------------------------------------------------------------------------ */
+/*
+ * The indexer scores every preceding token of each query so the top-k most
+ * relevant can be kept; it is O(L^2) per layer (es page, section 1
+ * "El Problema"; pt page, section 1 "O Gargalo do Indexador").  The score
+ * form is not printed on the pages; this library computes
+ *     scores[b,i,s] = sum_h w[b,i,h] * max(0, q_I[b,i,h,:] . k_I[b,s,:])
+ * for s <= t = q_start + i.  Entries s > t of a row are NOT written.
+ *
+ *   q_idx   [B, Lq, H_I, d_I] of dt   (IC_F32, IC_BF16 or IC_FP8_E4M3 codes)
+ *   q_scale [B, Lq] float32, one non-negative scale per query token
+ *           (IC_FP8_E4M3 only; NULL otherwise): q value = e4m3(code)*scale
+ *   w       [B, Lq, H_I] float32 head weights
+ *   k_idx   [B, T, d_I] of dt
+ *   k_scale [B, T] float32 (IC_FP8_E4M3 only; NULL otherwise)
+ *   scores  [B, Lq, ld_scores] float32; ld_scores >= T, ld_scores % 4 == 0
+ * Accumulation is float32.  With FP8 operands the scales are applied after
+ * the head-sum (exact for non-negative scales, ReLU being positively
+ * homogeneous).  Supported: H_I in [1,128]; d_I in [1,256].  The tensor-core
+ * path is used for IC_BF16 / IC_FP8_E4M3 with d_I == 128 and H_I in
+ * {16,32,64,128}; other shapes and IC_F32 use a CUDA-core path.
+ */
+size_t ic_indexer_workspace_size(ic_rows r, int H_I, int d_I, ic_dtype dt);
+ic_status ic_indexer_scores(const void* q_idx, const float* q_scale, const float* w,
+                            const void* k_idx, const float* k_scale, ic_dtype dt,
+                            ic_rows r, int H_I, int d_I,
+                            float* scores, int64_t ld_scores,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* a2  Top-k selection (F layers)                                            */
+/* ------------------------------------------------------------------------ */
+/*
+ * DSA keeps the k most relevant keys of each query (es page, section 1).
+ * Row t keeps the min(k, t+1) candidates s <= t with the largest score,
+ * ordered by (score descending, position ascending): equal scores go to the
+ * smaller position, -0.0 counts as +0.0.  The kept positions are written in
+ * ASCENDING order, followed by -1 up to k entries.
+ *
+ *   scores [B, Lq, ld_scores] float32 (only s <= t of each row is read;
+ *          ld_scores >= T, ld_scores % 4 == 0); must not hold NaN
+ *   idx    [B, Lq, k] int32 (output)
+ *   k      in [1, 16384]
+ */
+size_t ic_topk_workspace_size(ic_rows r, int k);
+ic_status ic_topk(const float* scores, int64_t ld_scores, ic_rows r, int k, int32_t* idx,
+                  void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* a4/a5  Sparse multi-query attention (every layer)                         */
+/* ------------------------------------------------------------------------ */
+/*
+ * Core attention restricted to the selected keys, O(Lk) (es page,
+ * section 1; de page, section 1).  For row (b,i), head h and the entries j
+ * of idx[b,i,:] that are >= 0:
+ *     p_j = softmax_j(scale * q[b,i,h,0:d_qk] . K[b,j,0:d_qk])
+ *     out[b,i,h,0:d_v] = sum_j p_j * V[b,j,0:d_v]
+ * All Hq heads share the same key/value rows (multi-query attention).
+ *
+ *   q    [B, Lq, Hq, d_qk] of dt (IC_F32 or IC_BF16)
+ *   kmat key row (b,s) starts at kmat + (b*T + s) * k_row_stride elements
+ *   vmat value row (b,s) starts at vmat + (b*T + s) * v_row_stride elements
+ *        (a latent KV cache passes the same pointer twice: K = the whole
+ *        576-wide row, V = its first 512 columns)
+ *   idx  [B, Lq, k] int32: positions in [0, t] or -1 (skipped).  The valid
+ *        entries must form a prefix of the row when the tensor-core path is
+ *        used (ic_topk's output always does).  An entry outside [0, t] is
+ *        never dereferenced: the row is computed without it and the status
+ *        bit IC_ERR_INDEX_RANGE is set.
+ *   out  [B, Lq, Hq, d_v] of dt.  A row with no valid index gets zeros.
+ * Supported: Hq in [1,128], d_qk, d_v in [1,576].  The tensor-core path is
+ * used for IC_BF16 with Hq == 128, d_qk == 576, d_v == 512 and kmat == vmat
+ * (the latent MQA layout); other shapes use a CUDA-core path.  Rows with few
+ * query rows per call (decode) are split over the k keys and merged by a
+ * log-sum-exp combine (a5), which needs workspace.
+ */
+size_t ic_sparse_attn_workspace_size(ic_rows r, int k, int Hq, int d_qk, int d_v, ic_dtype dt);
+ic_status ic_sparse_attn(const void* q, const void* kmat, int64_t k_row_stride,
+                         const void* vmat, int64_t v_row_stride, const int32_t* idx, int k,
+                         ic_dtype dt, ic_rows r, int Hq, int d_qk, int d_v, float scale,
+                         void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* a3  The layer stack with the F/S branch                                   */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    ic_rows rows;
+    int H_I, d_I;          /* indexer heads and width                          */
+    ic_dtype idx_dtype;    /* dtype of q_idx / k_idx                           */
+    int k;                 /* top-k                                            */
+    int Hq, d_qk, d_v;     /* attention heads and widths                       */
+    ic_dtype attn_dtype;   /* dtype of q, kmat, vmat, out                      */
+    int64_t k_row_stride;  /* elements between consecutive key rows           */
+    int64_t v_row_stride;  /* elements between consecutive value rows         */
+    float scale;           /* softmax scale                                    */
+} ic_stack_shape;
+
+/* Per-layer device buffers, same layouts as the single calls above.  The
+ * indexer fields (q_idx, q_scale, w, k_idx, k_scale) are ignored, and may be
+ * NULL, on S layers. */
+typedef struct {
+    const void* q_idx;
+    const float* q_scale;
+    const float* w;
+    const void* k_idx;
+    const float* k_scale;
+    const void* q;
+    const void* kmat;
+    const void* vmat;
+    void* out;
+} ic_layer_io;
+
+/*
+ * Run n_layers layers in order.  pattern is a NUL-terminated string of
+ * exactly n_layers characters 'F' or 'S' whose first character is 'F'
+ * (an S layer inherits from the nearest PRECEDING F layer, so a leading S
+ * has nothing to inherit); anything else returns IC_ERR_PATTERN.
+ *   F layer: indexer -> scores (workspace) -> top-k -> idx_buf
+ *   S layer: idx_buf is used unchanged (no copy, no indexer launch)
+ *   every layer: sparse attention over idx_buf -> layers[l].out
+ * idx_buf [B, Lq, k] int32 is the single index cache.  idx_out is either
+ * NULL or a HOST array of n_layers device pointers, each NULL or an
+ * [B, Lq, k] int32 buffer that receives a copy of the indices layer l used
+ * (for checking; costs one device copy per non-NULL entry).
+ * ws_bytes >= ic_workspace_size(shape).
+ */
+size_t ic_workspace_size(const ic_stack_shape* shape);
+ic_status ic_layer_stack_forward(const char* pattern, int n_layers, const ic_layer_io* layers,
+                                 const ic_stack_shape* shape, int32_t* idx_buf,
+                                 int32_t* const* idx_out, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INDEXCACHE_H */
