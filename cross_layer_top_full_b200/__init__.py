@@ -1,0 +1,236 @@
+"""IndexCache on B200: Python binding of the C-ABI library ``libindexcache.so``.
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels.  PyTorch supplies device memory and streams.  If the library is
+missing this package raises on first use; there is no CPU fallback.
+
+Entry points mirror ``include/indexcache.h``:
+``indexer_scores``, ``topk``, ``sparse_attn``, ``layer_stack_forward``,
+their ``*_workspace_size`` queries, ``workspace_init``, ``read_status``,
+``kernel_launches`` and ``status_string``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional, Sequence
+
+__all__ = [
+    "IcError", "lib", "library_path", "Rows", "StackShape", "LayerIO",
+    "F32", "BF16", "FP8_E4M3", "STATUS_BYTES",
+    "status_string", "version", "kernel_launches", "workspace_init", "read_status",
+    "indexer_workspace_size", "indexer_scores", "topk_workspace_size", "topk",
+    "sparse_attn_workspace_size", "sparse_attn", "workspace_size", "layer_stack_forward",
+]
+
+F32, BF16, FP8_E4M3 = 0, 1, 2
+STATUS_BYTES = 256
+_STATUS = {0: "IC_OK", -1: "IC_ERR_INVALID_ARG", -2: "IC_ERR_PATTERN", -3: "IC_ERR_UNSUPPORTED",
+           -4: "IC_ERR_WORKSPACE", -5: "IC_ERR_CUDA", -6: "IC_ERR_INDEX_RANGE",
+           -7: "IC_ERR_TIMEOUT"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def library_path() -> str:
+    return os.environ.get("INDEXCACHE_LIB", os.path.join(_HERE, "libindexcache.so"))
+
+
+class IcError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__("%s failed: %s (%d)" % (where, _STATUS.get(code, "?"), code))
+
+
+class Rows(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Lq", ctypes.c_int), ("q_start", ctypes.c_int),
+                ("T", ctypes.c_int)]
+
+
+class StackShape(ctypes.Structure):
+    _fields_ = [("rows", Rows), ("H_I", ctypes.c_int), ("d_I", ctypes.c_int),
+                ("idx_dtype", ctypes.c_int), ("k", ctypes.c_int), ("Hq", ctypes.c_int),
+                ("d_qk", ctypes.c_int), ("d_v", ctypes.c_int), ("attn_dtype", ctypes.c_int),
+                ("k_row_stride", ctypes.c_int64), ("v_row_stride", ctypes.c_int64),
+                ("scale", ctypes.c_float)]
+
+
+class LayerIO(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("q_idx", "q_scale", "w", "k_idx", "k_scale", "q", "kmat", "vmat", "out")]
+
+
+_P = ctypes.c_void_p
+_SIG = {
+    "ic_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "ic_version": (ctypes.c_int, []),
+    "ic_kernel_launches": (ctypes.c_uint64, [ctypes.c_int]),
+    "ic_workspace_init": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
+    "ic_read_status": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
+    "ic_indexer_workspace_size": (ctypes.c_size_t, [Rows, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "ic_indexer_scores": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, Rows, ctypes.c_int,
+                                         ctypes.c_int, _P, ctypes.c_int64, _P, ctypes.c_size_t, _P]),
+    "ic_topk_workspace_size": (ctypes.c_size_t, [Rows, ctypes.c_int]),
+    "ic_topk": (ctypes.c_int, [_P, ctypes.c_int64, Rows, ctypes.c_int, _P, _P, ctypes.c_size_t, _P]),
+    "ic_sparse_attn_workspace_size": (ctypes.c_size_t, [Rows, ctypes.c_int, ctypes.c_int,
+                                                        ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "ic_sparse_attn": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P, ctypes.c_int64, _P, ctypes.c_int,
+                                      ctypes.c_int, Rows, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+    "ic_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(StackShape)]),
+    "ic_layer_stack_forward": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_int,
+                                              ctypes.POINTER(LayerIO), ctypes.POINTER(StackShape),
+                                              _P, ctypes.POINTER(_P), _P, ctypes.c_size_t, _P]),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (loaded on first use; raises if it is missing)."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise ImportError("libindexcache.so not built at %s: run "
+                              "`python -m cross_layer_top_full_b200.build`" % path)
+        handle = ctypes.CDLL(path)
+        for name, (res, args) in _SIG.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+# --------------------------------------------------------------------------- helpers
+def _ptr(x) -> Optional[int]:
+    """Device/host address of a tensor, or an int address, or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        if torch.cuda.is_available():
+            return torch.cuda.current_stream().cuda_stream
+        return None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _nbytes(x) -> int:
+    return x.numel() * x.element_size()
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise IcError(code, where)
+
+
+def _rows(rows) -> Rows:
+    if isinstance(rows, Rows):
+        return rows
+    B, Lq, q_start, T = rows
+    return Rows(int(B), int(Lq), int(q_start), int(T))
+
+
+def _dtype_of(t) -> int:
+    import torch
+    return {torch.float32: F32, torch.bfloat16: BF16, torch.uint8: FP8_E4M3,
+            torch.float8_e4m3fn: FP8_E4M3}[t.dtype]
+
+
+# --------------------------------------------------------------------------- API
+def status_string(code: int) -> str:
+    return lib().ic_status_string(code).decode()
+
+
+def version() -> int:
+    return lib().ic_version()
+
+
+def kernel_launches(kind: int = 0) -> int:
+    return int(lib().ic_kernel_launches(kind))
+
+
+def workspace_init(ws, stream=None) -> None:
+    _check(lib().ic_workspace_init(_ptr(ws), _nbytes(ws), _stream(stream)), "ic_workspace_init")
+
+
+def read_status(ws, stream=None) -> int:
+    """Raw device status bits (0 = clean); clears them."""
+    v = ctypes.c_int32(0)
+    code = lib().ic_read_status(_ptr(ws), _stream(stream), ctypes.byref(v))
+    if code not in (0, -6, -7):
+        raise IcError(code, "ic_read_status")
+    return int(v.value)
+
+
+def indexer_workspace_size(rows, H_I: int, d_I: int, dtype: int) -> int:
+    return int(lib().ic_indexer_workspace_size(_rows(rows), H_I, d_I, dtype))
+
+
+def indexer_scores(q_idx, w, k_idx, rows, scores, ws, *, q_scale=None, k_scale=None,
+                   dtype: Optional[int] = None, ld_scores: Optional[int] = None,
+                   stream=None) -> None:
+    """scores[b,i,s] = sum_h w * ReLU(q_idx[b,i,h] . k_idx[b,s]) for s <= q_start+i."""
+    r = _rows(rows)
+    dt = _dtype_of(q_idx) if dtype is None else dtype
+    H_I, d_I = q_idx.shape[-2], q_idx.shape[-1]
+    ld = scores.shape[-1] if ld_scores is None else ld_scores
+    _check(lib().ic_indexer_scores(_ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(k_idx), _ptr(k_scale),
+                                   dt, r, H_I, d_I, _ptr(scores), ld, _ptr(ws), _nbytes(ws),
+                                   _stream(stream)), "ic_indexer_scores")
+
+
+def topk_workspace_size(rows, k: int) -> int:
+    return int(lib().ic_topk_workspace_size(_rows(rows), k))
+
+
+def topk(scores, rows, k: int, idx, ws, *, ld_scores: Optional[int] = None, stream=None) -> None:
+    ld = scores.shape[-1] if ld_scores is None else ld_scores
+    _check(lib().ic_topk(_ptr(scores), ld, _rows(rows), k, _ptr(idx), _ptr(ws), _nbytes(ws),
+                         _stream(stream)), "ic_topk")
+
+
+def sparse_attn_workspace_size(rows, k: int, Hq: int, d_qk: int, d_v: int, dtype: int) -> int:
+    return int(lib().ic_sparse_attn_workspace_size(_rows(rows), k, Hq, d_qk, d_v, dtype))
+
+
+def sparse_attn(q, kmat, k_row_stride: int, vmat, v_row_stride: int, idx, rows, d_v: int,
+                scale: float, out, ws, *, dtype: Optional[int] = None, stream=None) -> None:
+    """Sparse MQA attention of q [B,Lq,Hq,d_qk] over the keys listed in idx."""
+    dt = _dtype_of(q) if dtype is None else dtype
+    Hq, d_qk = q.shape[-2], q.shape[-1]
+    k = idx.shape[-1]
+    _check(lib().ic_sparse_attn(_ptr(q), _ptr(kmat), k_row_stride, _ptr(vmat), v_row_stride,
+                                _ptr(idx), k, dt, _rows(rows), Hq, d_qk, d_v, float(scale),
+                                _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "ic_sparse_attn")
+
+
+def workspace_size(shape: StackShape) -> int:
+    return int(lib().ic_workspace_size(ctypes.byref(shape)))
+
+
+def layer_stack_forward(pattern: str, layers: Sequence[Dict], shape: StackShape, idx_buf, ws, *,
+                        idx_out: Optional[List] = None, stream=None) -> None:
+    """Run the F/S layer stack.  Each layer dict may hold q_idx, q_scale, w,
+    k_idx, k_scale (F layers), q, kmat, vmat, out (tensors or int addresses)."""
+    n = len(layers)
+    arr = (LayerIO * max(1, n))()
+    for l, L in enumerate(layers):
+        for name, _ in LayerIO._fields_:
+            setattr(arr[l], name, _ptr(L.get(name)))
+    outs = None
+    if idx_out is not None:
+        outs = (_P * max(1, n))(*[_ptr(x) for x in idx_out])
+    _check(lib().ic_layer_stack_forward(pattern.encode(), n, arr, ctypes.byref(shape),
+                                        _ptr(idx_buf), outs, _ptr(ws), _nbytes(ws),
+                                        _stream(stream)), "ic_layer_stack_forward")

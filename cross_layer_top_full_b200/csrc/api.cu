@@ -1,0 +1,259 @@
+// api.cu -- the C ABI of the IndexCache library (see include/indexcache.h).
+//
+// Argument validation, workspace layout, dispatch between the tensor-core and
+// CUDA-core kernels, and the layer stack with IndexCache's F/S branch:
+// F layers run indexer -> top-k into the single index cache, S layers reuse
+// the cache unchanged, every layer runs sparse attention (IndexCache summary,
+// es page, section 2 "Arquitectura del Método"; it page, section 2
+// "Architettura e Funzionamento").
+#include <atomic>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace ic {
+
+static std::atomic<uint64_t> g_launches[5];
+
+void count_launch(int kind) {
+    g_launches[IC_LK_ALL].fetch_add(1, std::memory_order_relaxed);
+    if (kind > 0 && kind < 5) g_launches[kind].fetch_add(1, std::memory_order_relaxed);
+}
+
+ic_status last_launch_status() {
+    return cudaGetLastError() == cudaSuccess ? IC_OK : IC_ERR_CUDA;
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool rows_ok(const ic_rows& r) {
+    if (r.B < 0 || r.Lq < 0 || r.q_start < 0 || r.T < 0) return false;
+    return (int64_t)r.q_start + r.Lq <= r.T;
+}
+bool rows_empty(const ic_rows& r) { return r.B == 0 || r.Lq == 0; }
+
+bool ws_ok(const void* ws, size_t bytes, size_t need) {
+    return ws != nullptr && bytes >= need && ((uintptr_t)ws % kAlign) == 0;
+}
+
+uint32_t* status_of(void* ws) { return static_cast<uint32_t*>(ws); }
+char* scratch_of(void* ws) { return static_cast<char*>(ws) + IC_STATUS_BYTES; }
+
+size_t scores_bytes(const ic_rows& r) {
+    const int64_t ld = ((int64_t)r.T + 3) / 4 * 4;
+    return (size_t)r.B * r.Lq * ld * sizeof(float);
+}
+
+bool attn_args_ok(ic_dtype dt, int Hq, int d_qk, int d_v, int k) {
+    return (dt == IC_F32 || dt == IC_BF16) && Hq >= 1 && Hq <= 128 && d_qk >= 1 && d_qk <= 576 &&
+           d_v >= 1 && d_v <= 576 && k >= 1 && k <= 16384;
+}
+
+bool indexer_args_ok(ic_dtype dt, int H_I, int d_I) {
+    return (dt == IC_F32 || dt == IC_BF16 || dt == IC_FP8_E4M3) && H_I >= 1 && H_I <= 128 &&
+           d_I >= 1 && d_I <= 256;
+}
+
+size_t attn_scratch(const ic_rows& r, int k, int Hq, int d_qk, int d_v, ic_dtype dt) {
+    // the tensor-core path may be taken when the shapes match; size for it
+    if (dt == IC_BF16 && Hq == 128 && d_qk == 576 && d_v == 512) return attn_tc_scratch_bytes(r, k);
+    return 0;
+}
+
+ic_status run_indexer(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
+                      const float* k_scale, ic_dtype dt, ic_rows r, int H_I, int d_I,
+                      float* scores, int64_t ld, uint32_t* status, cudaStream_t s) {
+    if (indexer_tc_supported(dt, H_I, d_I))
+        return launch_indexer_tc(q_idx, q_scale, w, k_idx, k_scale, dt, r, H_I, d_I, scores, ld,
+                                 status, s);
+    return launch_indexer_simt(q_idx, q_scale, w, k_idx, k_scale, dt, r, H_I, d_I, scores, ld, s);
+}
+
+ic_status run_attn(const void* q, const void* kmat, int64_t ks, const void* vmat, int64_t vs,
+                   const int32_t* idx, int k, ic_dtype dt, ic_rows r, int Hq, int d_qk, int d_v,
+                   float scale, void* out, uint32_t* status, void* scratch, size_t scratch_bytes,
+                   cudaStream_t s) {
+    if (attn_tc_supported(kmat, vmat, ks, vs, dt, Hq, d_qk, d_v) &&
+        scratch_bytes >= attn_tc_scratch_bytes(r, k))
+        return launch_attn_tc(q, kmat, ks, idx, k, r, scale, out, status, scratch, scratch_bytes, s);
+    return launch_attn_simt(q, kmat, ks, vmat, vs, idx, k, dt, r, Hq, d_qk, d_v, scale, out,
+                            status, s);
+}
+
+}  // namespace
+}  // namespace ic
+
+using namespace ic;
+
+extern "C" {
+
+const char* ic_status_string(ic_status st) {
+    switch (st) {
+        case IC_OK: return "IC_OK";
+        case IC_ERR_INVALID_ARG: return "IC_ERR_INVALID_ARG";
+        case IC_ERR_PATTERN: return "IC_ERR_PATTERN";
+        case IC_ERR_UNSUPPORTED: return "IC_ERR_UNSUPPORTED";
+        case IC_ERR_WORKSPACE: return "IC_ERR_WORKSPACE";
+        case IC_ERR_CUDA: return "IC_ERR_CUDA";
+        case IC_ERR_INDEX_RANGE: return "IC_ERR_INDEX_RANGE";
+        case IC_ERR_TIMEOUT: return "IC_ERR_TIMEOUT";
+    }
+    return "IC_ERR_UNKNOWN";
+}
+
+int ic_version(void) { return 10000; }
+
+uint64_t ic_kernel_launches(int kind) {
+    if (kind < 0 || kind > 4) return 0;
+    return g_launches[kind].load(std::memory_order_relaxed);
+}
+
+ic_status ic_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    if (!ws_ok(ws, ws_bytes, IC_STATUS_BYTES)) return IC_ERR_WORKSPACE;
+    if (cudaMemsetAsync(ws, 0, IC_STATUS_BYTES, (cudaStream_t)stream) != cudaSuccess)
+        return IC_ERR_CUDA;
+    return IC_OK;
+}
+
+ic_status ic_read_status(void* ws, void* stream, int32_t* device_status) {
+    if (ws == nullptr || device_status == nullptr) return IC_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return IC_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return IC_ERR_CUDA;
+    if (v != 0) {
+        if (cudaMemsetAsync(ws, 0, sizeof(v), s) != cudaSuccess) return IC_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return IC_ERR_CUDA;
+    }
+    *device_status = (int32_t)v;
+    if (v & IC_DEV_INDEX_RANGE) return IC_ERR_INDEX_RANGE;
+    if (v & IC_DEV_TIMEOUT) return IC_ERR_TIMEOUT;
+    return IC_OK;
+}
+
+size_t ic_indexer_workspace_size(ic_rows r, int H_I, int d_I, ic_dtype dt) {
+    (void)r; (void)H_I; (void)d_I; (void)dt;
+    return IC_STATUS_BYTES;
+}
+
+ic_status ic_indexer_scores(const void* q_idx, const float* q_scale, const float* w,
+                            const void* k_idx, const float* k_scale, ic_dtype dt, ic_rows r,
+                            int H_I, int d_I, float* scores, int64_t ld_scores, void* ws,
+                            size_t ws_bytes, void* stream) {
+    if (!rows_ok(r) || !indexer_args_ok(dt, H_I, d_I)) return IC_ERR_INVALID_ARG;
+    if (ld_scores < r.T || ld_scores % 4 != 0) return IC_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, ic_indexer_workspace_size(r, H_I, d_I, dt))) return IC_ERR_WORKSPACE;
+    if (rows_empty(r)) return IC_OK;
+    if (!q_idx || !w || !k_idx || !scores) return IC_ERR_INVALID_ARG;
+    if (dt == IC_FP8_E4M3 && (!q_scale || !k_scale)) return IC_ERR_INVALID_ARG;
+    if (dt != IC_FP8_E4M3 && (q_scale || k_scale)) return IC_ERR_INVALID_ARG;
+    return run_indexer(q_idx, q_scale, w, k_idx, k_scale, dt, r, H_I, d_I, scores, ld_scores,
+                       status_of(ws), (cudaStream_t)stream);
+}
+
+size_t ic_topk_workspace_size(ic_rows r, int k) {
+    (void)r; (void)k;
+    return IC_STATUS_BYTES;
+}
+
+ic_status ic_topk(const float* scores, int64_t ld_scores, ic_rows r, int k, int32_t* idx,
+                  void* ws, size_t ws_bytes, void* stream) {
+    if (!rows_ok(r) || k < 1 || k > 16384) return IC_ERR_INVALID_ARG;
+    if (ld_scores < r.T || ld_scores % 4 != 0) return IC_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, ic_topk_workspace_size(r, k))) return IC_ERR_WORKSPACE;
+    if (rows_empty(r)) return IC_OK;
+    if (!scores || !idx) return IC_ERR_INVALID_ARG;
+    return launch_topk(scores, ld_scores, r, k, idx, (cudaStream_t)stream);
+}
+
+size_t ic_sparse_attn_workspace_size(ic_rows r, int k, int Hq, int d_qk, int d_v, ic_dtype dt) {
+    return IC_STATUS_BYTES + align_up(attn_scratch(r, k, Hq, d_qk, d_v, dt));
+}
+
+ic_status ic_sparse_attn(const void* q, const void* kmat, int64_t k_row_stride, const void* vmat,
+                         int64_t v_row_stride, const int32_t* idx, int k, ic_dtype dt, ic_rows r,
+                         int Hq, int d_qk, int d_v, float scale, void* out, void* ws,
+                         size_t ws_bytes, void* stream) {
+    if (!rows_ok(r) || !attn_args_ok(dt, Hq, d_qk, d_v, k)) return IC_ERR_INVALID_ARG;
+    if (k_row_stride < d_qk || v_row_stride < d_v) return IC_ERR_INVALID_ARG;
+    const size_t need = ic_sparse_attn_workspace_size(r, k, Hq, d_qk, d_v, dt);
+    if (!ws_ok(ws, ws_bytes, need)) return IC_ERR_WORKSPACE;
+    if (rows_empty(r)) return IC_OK;
+    if (!q || !kmat || !vmat || !idx || !out) return IC_ERR_INVALID_ARG;
+    return run_attn(q, kmat, k_row_stride, vmat, v_row_stride, idx, k, dt, r, Hq, d_qk, d_v, scale,
+                    out, status_of(ws), scratch_of(ws), ws_bytes - IC_STATUS_BYTES,
+                    (cudaStream_t)stream);
+}
+
+size_t ic_workspace_size(const ic_stack_shape* sh) {
+    if (sh == nullptr) return 0;
+    const ic_rows& r = sh->rows;
+    return IC_STATUS_BYTES + align_up(scores_bytes(r)) +
+           align_up(attn_scratch(r, sh->k, sh->Hq, sh->d_qk, sh->d_v, sh->attn_dtype));
+}
+
+ic_status ic_layer_stack_forward(const char* pattern, int n_layers, const ic_layer_io* layers,
+                                 const ic_stack_shape* sh, int32_t* idx_buf,
+                                 int32_t* const* idx_out, void* ws, size_t ws_bytes,
+                                 void* stream) {
+    if (pattern == nullptr || n_layers < 0) return IC_ERR_PATTERN;
+    if (strlen(pattern) != (size_t)n_layers) return IC_ERR_PATTERN;
+    for (int l = 0; l < n_layers; ++l)
+        if (pattern[l] != 'F' && pattern[l] != 'S') return IC_ERR_PATTERN;
+    if (n_layers > 0 && pattern[0] != 'F') return IC_ERR_PATTERN;
+    if (sh == nullptr || (n_layers > 0 && layers == nullptr)) return IC_ERR_INVALID_ARG;
+    const ic_rows r = sh->rows;
+    if (!rows_ok(r) || !indexer_args_ok(sh->idx_dtype, sh->H_I, sh->d_I) ||
+        !attn_args_ok(sh->attn_dtype, sh->Hq, sh->d_qk, sh->d_v, sh->k))
+        return IC_ERR_INVALID_ARG;
+    if (sh->k_row_stride < sh->d_qk || sh->v_row_stride < sh->d_v) return IC_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, ic_workspace_size(sh))) return IC_ERR_WORKSPACE;
+    if (rows_empty(r) || n_layers == 0) return IC_OK;
+    if (idx_buf == nullptr) return IC_ERR_INVALID_ARG;
+    // validate every layer's pointers before launching anything
+    for (int l = 0; l < n_layers; ++l) {
+        const ic_layer_io& L = layers[l];
+        if (!L.q || !L.kmat || !L.vmat || !L.out) return IC_ERR_INVALID_ARG;
+        if (pattern[l] == 'F') {
+            if (!L.q_idx || !L.w || !L.k_idx) return IC_ERR_INVALID_ARG;
+            const bool fp8 = sh->idx_dtype == IC_FP8_E4M3;
+            if (fp8 != (L.q_scale != nullptr) || fp8 != (L.k_scale != nullptr))
+                return IC_ERR_INVALID_ARG;
+        }
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t* status = status_of(ws);
+    float* scores = reinterpret_cast<float*>(scratch_of(ws));
+    const int64_t ld = ((int64_t)r.T + 3) / 4 * 4;
+    char* attn_ws = scratch_of(ws) + align_up(scores_bytes(r));
+    const size_t attn_ws_bytes = ws_bytes - IC_STATUS_BYTES - align_up(scores_bytes(r));
+    const size_t idx_bytes = (size_t)r.B * r.Lq * sh->k * sizeof(int32_t);
+
+    for (int l = 0; l < n_layers; ++l) {
+        const ic_layer_io& L = layers[l];
+        if (pattern[l] == 'F') {  // the one conditional branch of IndexCache
+            ic_status st = run_indexer(L.q_idx, L.q_scale, L.w, L.k_idx, L.k_scale, sh->idx_dtype,
+                                       r, sh->H_I, sh->d_I, scores, ld, status, s);
+            if (st != IC_OK) return st;
+            st = launch_topk(scores, ld, r, sh->k, idx_buf, s);
+            if (st != IC_OK) return st;
+        }
+        ic_status st = run_attn(L.q, L.kmat, sh->k_row_stride, L.vmat, sh->v_row_stride, idx_buf,
+                                sh->k, sh->attn_dtype, r, sh->Hq, sh->d_qk, sh->d_v, sh->scale,
+                                L.out, status, attn_ws, attn_ws_bytes, s);
+        if (st != IC_OK) return st;
+        if (idx_out != nullptr && idx_out[l] != nullptr) {
+            if (cudaMemcpyAsync(idx_out[l], idx_buf, idx_bytes, cudaMemcpyDeviceToDevice, s) !=
+                cudaSuccess)
+                return IC_ERR_CUDA;
+        }
+    }
+    return IC_OK;
+}
+
+}  // extern "C"

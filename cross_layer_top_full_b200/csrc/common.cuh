@@ -1,0 +1,72 @@
+// common.cuh -- shared definitions of the IndexCache CUDA library (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "indexcache.h"
+
+// Bits of the device status word at the start of every workspace.
+#define IC_DEV_INDEX_RANGE 1u
+#define IC_DEV_TIMEOUT 2u
+
+// Launch kinds counted by ic_kernel_launches.
+enum { IC_LK_ALL = 0, IC_LK_INDEXER = 1, IC_LK_TOPK = 2, IC_LK_ATTN = 3, IC_LK_COMBINE = 4 };
+
+namespace ic {
+
+// Host: count one launch of a kind (also counted under IC_LK_ALL).
+void count_launch(int kind);
+
+// Host: map the last CUDA error to a status.
+ic_status last_launch_status();
+
+__device__ __forceinline__ void flag_status(uint32_t* status, uint32_t bit) {
+    if (status) atomicOr(status, bit);
+}
+
+// Element loads of the supported storage types, as float.
+__device__ __forceinline__ float load_as_float(const float* p) { return *p; }
+__device__ __forceinline__ float load_as_float(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ float load_as_float(const __nv_fp8_e4m3* p) { return float(*p); }
+
+__device__ __forceinline__ void store_from_float(float* p, float v) { *p = v; }
+__device__ __forceinline__ void store_from_float(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+__host__ __device__ __forceinline__ int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace ic
+
+// Internal launchers (one per kernel family).  `status` points at the
+// device status word; `scratch` is call-specific workspace after it.
+namespace ic {
+
+ic_status launch_indexer_simt(const void* q_idx, const float* q_scale, const float* w,
+                              const void* k_idx, const float* k_scale, ic_dtype dt, ic_rows r,
+                              int H_I, int d_I, float* scores, int64_t ld, cudaStream_t s);
+
+bool indexer_tc_supported(ic_dtype dt, int H_I, int d_I);
+ic_status launch_indexer_tc(const void* q_idx, const float* q_scale, const float* w,
+                            const void* k_idx, const float* k_scale, ic_dtype dt, ic_rows r,
+                            int H_I, int d_I, float* scores, int64_t ld, uint32_t* status,
+                            cudaStream_t s);
+
+ic_status launch_topk(const float* scores, int64_t ld, ic_rows r, int k, int32_t* idx,
+                      cudaStream_t s);
+
+ic_status launch_attn_simt(const void* q, const void* kmat, int64_t ks, const void* vmat,
+                           int64_t vs, const int32_t* idx, int k, ic_dtype dt, ic_rows r, int Hq,
+                           int d_qk, int d_v, float scale, void* out, uint32_t* status,
+                           cudaStream_t s);
+
+bool attn_tc_supported(const void* kmat, const void* vmat, int64_t ks, int64_t vs, ic_dtype dt,
+                       int Hq, int d_qk, int d_v);
+size_t attn_tc_scratch_bytes(ic_rows r, int k);
+ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_t* idx, int k,
+                         ic_rows r, float scale, void* out, uint32_t* status, void* scratch,
+                         size_t scratch_bytes, cudaStream_t s);
+
+}  // namespace ic

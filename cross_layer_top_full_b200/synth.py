@@ -216,3 +216,62 @@ def layer_inputs(wl: Workload, layer: int, device="cpu", *, indexer: bool = True
             out["k"] = _randn((B, T, wl.d_qk), wl.kv_std, device, wl.seed, "k", layer, dtype=adt)
             out["v"] = _randn((B, T, wl.d_v), wl.kv_std, device, wl.seed, "v", layer, dtype=adt)
     return out
+
+
+def exact_indexer_inputs(B: int, Lq: int, T: int, H_I: int, d_I: int, dtype: str, device="cpu",
+                         seed: int = 0) -> Dict[str, torch.Tensor]:
+    """Indexer inputs whose scores are exact in float32 for any summation order.
+
+    q_I, k_I are integers in [-3, 3]; w = +-2^-j, j in 0..3; with e4m3 the
+    codes hold those integers and the per-token scales are powers of two in
+    {1/2, 1, 2}.  Every product and partial sum is then a multiple of 2^-5
+    below 2^22, so float32 represents it exactly and the top-k is unique up
+    to exact ties (which the smaller-position rule settles).
+    """
+    g = _gen(device, seed, "exact")
+    qI = torch.randint(-3, 4, (B, Lq, H_I, d_I), generator=g, device=device).float()
+    kI = torch.randint(-3, 4, (B, T, d_I), generator=g, device=device).float()
+    sign = torch.randint(0, 2, (B, Lq, H_I), generator=g, device=device).float() * 2 - 1
+    j = torch.randint(0, 4, (B, Lq, H_I), generator=g, device=device).float()
+    out = {"w": (sign * torch.pow(2.0, -j)).contiguous()}
+    if dtype == "e4m3":
+        out["q_I"] = qI.to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+        out["k_I"] = kI.to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+        ex_q = torch.randint(-1, 2, (B, Lq), generator=g, device=device).float()
+        ex_k = torch.randint(-1, 2, (B, T), generator=g, device=device).float()
+        out["q_scale"] = torch.pow(2.0, ex_q).contiguous()
+        out["k_scale"] = torch.pow(2.0, ex_k).contiguous()
+    else:
+        dt = _store_dtype(dtype)
+        out["q_I"] = qI.to(dt).contiguous()
+        out["k_I"] = kI.to(dt).contiguous()
+    return out
+
+
+def random_scores(B: int, Lq: int, T: int, device="cpu", seed: int = 0, ties: bool = False,
+                  ld: Optional[int] = None) -> torch.Tensor:
+    """float32 scores [B, Lq, ld] (ld >= T, default T rounded up to 4).  With
+    ``ties`` the values come from a small set including +0.0 and -0.0, so
+    many scores are equal."""
+    ld = ld or (T + 3) // 4 * 4
+    g = _gen(device, seed, "scores", ties)
+    if ties:
+        pool = torch.tensor([-2.0, -1.0, -0.0, 0.0, 0.0, 0.5, 1.0, 3.0], device=device)
+        pick = torch.randint(0, pool.numel(), (B, Lq, ld), generator=g, device=device)
+        return pool[pick].contiguous()
+    return torch.randn((B, Lq, ld), generator=g, device=device).contiguous()
+
+
+def random_index_sets(B: int, Lq: int, q_start: int, k: int, device="cpu", seed: int = 0,
+                      n_valid: Optional[int] = None) -> torch.Tensor:
+    """int32 [B, Lq, k]: for row t, min(k, t+1, n_valid) distinct positions
+    drawn uniformly from [0, t], ascending, then -1 padding."""
+    g = _gen("cpu", seed, "idxsets")
+    out = torch.full((B, Lq, k), -1, dtype=torch.int32)
+    for b in range(B):
+        for i in range(Lq):
+            t = q_start + i
+            m = min(k, t + 1) if n_valid is None else min(k, t + 1, n_valid)
+            pos = torch.randperm(t + 1, generator=g)[:m].sort().values
+            out[b, i, :m] = pos.to(torch.int32)
+    return out.to(device)

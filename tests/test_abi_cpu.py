@@ -1,0 +1,145 @@
+"""Host-side checks of the C-ABI library that need no GPU.
+
+The library must load, export every function include/indexcache.h
+declares, and reject bad arguments before it touches the device.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import cross_layer_top_full_b200 as ic
+from cross_layer_top_full_b200 import build as icbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(ic.library_path()):
+        icbuild.build()
+    return ic.lib()
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(ic_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared()
+    assert len(declared) >= 12
+    out = subprocess.run(["nm", "-D", "--defined-only", ic.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (ic_[a-z0-9_]+)\b", out))
+    missing = [n for n in declared if n not in exported]
+    assert not missing, missing
+    for n in declared:
+        assert hasattr(lib, n)
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "IC_OK"), (-2, "IC_ERR_PATTERN"), (-6, "IC_ERR_INDEX_RANGE"),
+                       (-7, "IC_ERR_TIMEOUT")]:
+        assert ic.status_string(code) == name
+    assert ic.version() >= 10000
+
+
+def _shape(B=1, L=16, T=16, k=4):
+    return ic.StackShape(ic.Rows(B, L, T - L, T), 4, 32, ic.F32, k, 8, 64, 64, ic.F32, 64, 64, 0.125)
+
+
+class _FakeTensor:
+    """Host memory standing in for a device buffer; the calls below must
+    return before any device access."""
+    def __init__(self, nbytes, align=256):
+        self.buf = ctypes.create_string_buffer(nbytes + align)
+        addr = ctypes.addressof(self.buf)
+        self.addr = (addr + align - 1) // align * align
+        self.nbytes = nbytes
+
+    def data_ptr(self):
+        return self.addr
+
+    def numel(self):
+        return self.nbytes
+
+    def element_size(self):
+        return 1
+
+
+@pytest.mark.parametrize("pattern", ["SFSS", "FSXS", "FSS", "FSSSS", "fsss"])
+def test_stack_rejects_bad_patterns_before_launch(lib, pattern):
+    sh = _shape()
+    ws = _FakeTensor(ic.workspace_size(sh))
+    layers = [dict(q=1, kmat=1, vmat=1, out=1, q_idx=1, w=1, k_idx=1)] * 4
+    with pytest.raises(ic.IcError) as e:
+        ic.layer_stack_forward(pattern, layers, sh, 1, ws, stream=0)
+    assert e.value.code == -2
+
+
+def test_stack_rejects_small_or_misaligned_workspace(lib):
+    sh = _shape()
+    need = ic.workspace_size(sh)
+    assert need >= ic.STATUS_BYTES + 16 * 16 * 4
+    layers = [dict(q=1, kmat=1, vmat=1, out=1, q_idx=1, w=1, k_idx=1)] * 4
+    small = _FakeTensor(need - 1)
+    with pytest.raises(ic.IcError) as e:
+        ic.layer_stack_forward("FSSS", layers, sh, 1, small, stream=0)
+    assert e.value.code == -4
+    code = lib.ic_layer_stack_forward(b"FSSS", 4, (ic.LayerIO * 4)(), ctypes.byref(sh), 1, None,
+                                      _FakeTensor(need + 512).addr + 8, need + 256, None)
+    assert code == -4
+
+
+def test_stack_rejects_missing_layer_pointers(lib):
+    sh = _shape()
+    ws = _FakeTensor(ic.workspace_size(sh))
+    layers = [dict(q=1, kmat=1, vmat=1, out=1, q_idx=1, w=1, k_idx=1)] + \
+             [dict(q=1, kmat=1, vmat=1, out=1)] * 3
+    layers_bad = [dict(q=1, kmat=1, vmat=1, out=1)] * 4      # F layer without indexer inputs
+    with pytest.raises(ic.IcError) as e:
+        ic.layer_stack_forward("FSSS", layers_bad, sh, 1, ws, stream=0)
+    assert e.value.code == -1
+    with pytest.raises(ic.IcError) as e:        # S layers may omit them; idx_buf may not be NULL
+        ic.layer_stack_forward("FSSS", layers, sh, None, ws, stream=0)
+    assert e.value.code == -1
+
+
+def test_single_calls_validate_arguments(lib):
+    r = ic.Rows(1, 8, 4, 10)       # q_start + Lq = 12 > T = 10
+    ws = _FakeTensor(4096)
+    assert lib.ic_topk(1, 12, r, 4, 1, ws.addr, 4096, None) == -1
+    r = ic.Rows(1, 8, 2, 10)
+    assert lib.ic_topk(1, 10, r, 4, 1, ws.addr, 4096, None) == -1      # ld % 4 != 0
+    assert lib.ic_topk(1, 12, r, 0, 1, ws.addr, 4096, None) == -1      # k = 0
+    assert lib.ic_topk(1, 12, r, 4, 1, ws.addr, 100, None) == -4       # workspace too small
+    assert lib.ic_indexer_scores(1, None, 1, 1, None, 7, r, 4, 32, 1, 12, ws.addr, 4096, None) == -1
+    # fp8 needs both scales
+    assert lib.ic_indexer_scores(1, None, 1, 1, None, ic.FP8_E4M3, r, 4, 32, 1, 12, ws.addr, 4096,
+                                 None) == -1
+    # scales on a non-fp8 dtype are an error too
+    assert lib.ic_indexer_scores(1, 1, 1, 1, 1, ic.BF16, r, 4, 32, 1, 12, ws.addr, 4096, None) == -1
+    assert lib.ic_sparse_attn(1, 1, 63, 1, 64, 1, 4, ic.F32, r, 8, 64, 64, 0.1, 1, ws.addr, 4096,
+                              None) == -1                                # row stride < d_qk
+    assert lib.ic_sparse_attn(1, 1, 64, 1, 64, 1, 4, ic.FP8_E4M3, r, 8, 64, 64, 0.1, 1, ws.addr,
+                              4096, None) == -1                          # fp8 attention
+    # empty problems are valid no-ops
+    assert lib.ic_topk(1, 12, ic.Rows(0, 8, 2, 10), 4, 1, ws.addr, 4096, None) == 0
+    assert lib.ic_topk(1, 12, ic.Rows(1, 0, 2, 10), 4, 1, ws.addr, 4096, None) == 0
+
+
+def test_workspace_sizes_grow_with_the_problem(lib):
+    a = ic.workspace_size(_shape(L=16, T=16))
+    b = ic.workspace_size(_shape(L=16, T=1024))
+    assert b - a >= 16 * (1024 - 16) * 4
+    assert ic.topk_workspace_size((1, 4, 0, 4), 2) == ic.STATUS_BYTES
+    latent = ic.sparse_attn_workspace_size((32, 1, 32767, 32768), 2048, 128, 576, 512, ic.BF16)
+    assert latent >= ic.STATUS_BYTES

@@ -1,0 +1,270 @@
+"""GPU parity of each call of the C ABI against the float64 oracle, at sizes
+the oracle finishes in seconds that still span several tiles and ragged
+tails.  Full-size workloads are in test_gpu_workloads.py."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import cross_layer_top_full_b200 as ic
+from cross_layer_top_full_b200 import synth
+from parity_util import (abs_term_sum, check_attention, check_scores, check_topk_band, host64)
+
+pytestmark = pytest.mark.gpu
+
+DT = {"f32": ic.F32, "bf16": ic.BF16, "e4m3": ic.FP8_E4M3}
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    ic.lib()
+    return torch.device("cuda:0")
+
+
+def _ws(nbytes, dev):
+    ws = torch.empty(max(nbytes, ic.STATUS_BYTES), dtype=torch.uint8, device=dev)
+    ic.workspace_init(ws)
+    return ws
+
+
+def _gpu_scores(inp, rows, dtype, dev):
+    B, Lq, q_start, T = rows
+    ld = (T + 3) // 4 * 4
+    scores = torch.full((B, Lq, ld), float("nan"), device=dev)
+    ws = _ws(ic.indexer_workspace_size(rows, inp["q_I"].shape[-2], inp["q_I"].shape[-1], DT[dtype]), dev)
+    ic.indexer_scores(inp["q_I"], inp["w"], inp["k_I"], rows, scores, ws,
+                      q_scale=inp.get("q_scale"), k_scale=inp.get("k_scale"), dtype=DT[dtype])
+    torch.cuda.synchronize()
+    assert ic.read_status(ws) == 0
+    return scores
+
+
+def _oracle_scores(inp, q_start, dtype, rows=None):
+    fp8 = dtype == "e4m3"
+    return oracle.indexer_scores(host64(inp["q_I"]), host64(inp["w"]), host64(inp["k_I"]), q_start,
+                                 host64(inp["q_scale"]) if fp8 else None,
+                                 host64(inp["k_scale"]) if fp8 else None, fp8=fp8, rows=rows)
+
+
+# ------------------------------------------------------------------------- indexer
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "e4m3"])
+@pytest.mark.parametrize("H_I,d_I", [(64, 128), (4, 32), (16, 128)])
+def test_indexer_exact_mode_is_bit_exact(dev, dtype, H_I, d_I):
+    rows = (2, 300, 37, 400)       # ragged: 337 causal keys max, tails in both axes
+    B, Lq, q_start, T = rows
+    inp = synth.exact_indexer_inputs(B, Lq, T, H_I, d_I, dtype, dev, seed=H_I + d_I)
+    got = host64(_gpu_scores(inp, rows, dtype, dev))
+    ref = _oracle_scores(inp, q_start, dtype)
+    for b in range(B):
+        for i in range(Lq):
+            t = q_start + i
+            assert np.array_equal(got[b, i, : t + 1], ref[b, i, : t + 1]), (dtype, b, i)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "e4m3"])
+def test_indexer_general_inputs_within_tolerance(dev, dtype):
+    rows = (3, 130, 5, 140)
+    B, Lq, q_start, T = rows
+    wl = synth.WORKLOADS["decode_b8_t200k_fp8" if dtype == "e4m3" else "prefill_8k_bf16"]
+    g = torch.Generator(device=dev).manual_seed(11)
+    qI = torch.randn(B, Lq, 64, 128, device=dev, generator=g) / 11.3
+    kI = torch.randn(B, T, 128, device=dev, generator=g) / 11.3
+    w = torch.randn(B, Lq, 64, device=dev, generator=g) / 8
+    if dtype == "e4m3":
+        q8, qs = synth.fp8_per_token(qI, 2)
+        k8, ks = synth.fp8_per_token(kI, 2)
+        inp = dict(q_I=q8, k_I=k8, q_scale=qs, k_scale=ks, w=w)
+        vq = oracle.e4m3_decode(host64(q8)) * host64(qs)[..., None, None]
+        vk = oracle.e4m3_decode(host64(k8)) * host64(ks)[..., None]
+    else:
+        dt = torch.float32 if dtype == "f32" else torch.bfloat16
+        inp = dict(q_I=qI.to(dt), k_I=kI.to(dt), w=w)
+        vq, vk = host64(inp["q_I"]), host64(inp["k_I"])
+    got = host64(_gpu_scores(inp, rows, dtype, dev))
+    ref = _oracle_scores(inp, q_start, dtype)
+    absum = abs_term_sum(vq, host64(w), vk)
+    check_scores(got, ref, absum, q_start, rel=1e-3 if dtype == "e4m3" else 1e-4)
+    del wl
+
+
+# ------------------------------------------------------------------------- top-k
+@pytest.mark.parametrize("ties", [False, True])
+@pytest.mark.parametrize("rows,k", [((2, 70, 0, 70), 16),        # short rows, k < and >= t+1
+                                    ((1, 40, 3000, 3040), 2048),  # prefill-like long rows
+                                    ((4, 1, 49999, 50000), 2048), # decode rows beyond smem cache
+                                    ((3, 1, 32767, 32768), 2048), # decode rows, cached
+                                    ((1, 5, 10, 15), 1)])
+def test_topk_is_bit_exact_on_identical_scores(dev, rows, k, ties):
+    B, Lq, q_start, T = rows
+    scores = synth.random_scores(B, Lq, T, dev, seed=k + T, ties=ties)
+    idx = torch.full((B, Lq, k), -7, dtype=torch.int32, device=dev)
+    ws = _ws(ic.topk_workspace_size(rows, k), dev)
+    ic.topk(scores, rows, k, idx, ws)
+    torch.cuda.synchronize()
+    ref = oracle.topk_indices(host64(scores), q_start, k)
+    assert np.array_equal(host64(idx), ref)
+
+
+# ------------------------------------------------------------------------- attention
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("Hq,d_qk,d_v,latent", [(8, 64, 64, False), (128, 576, 512, True),
+                                                (3, 40, 24, False)])
+def test_sparse_attention_within_tolerance(dev, dtype, Hq, d_qk, d_v, latent):
+    rows = (2, 37, 90, 127)        # q_start > 0, ragged
+    B, Lq, q_start, T = rows
+    k = 100
+    torch_dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    g = torch.Generator(device=dev).manual_seed(Hq + d_qk)
+    q = torch.randn(B, Lq, Hq, d_qk, device=dev, generator=g).to(torch_dt)
+    if latent:
+        kv = torch.randn(B, T, d_qk, device=dev, generator=g).to(torch_dt)
+        kmat = vmat = kv
+        ks = vs = d_qk
+    else:
+        kmat = torch.randn(B, T, d_qk, device=dev, generator=g).to(torch_dt)
+        vmat = torch.randn(B, T, d_v, device=dev, generator=g).to(torch_dt)
+        ks, vs = d_qk, d_v
+    idx = synth.random_index_sets(B, Lq, q_start, k, dev, seed=3)
+    idx[0, 0, 40:] = -1            # a row with fewer valid keys than k
+    out = torch.empty(B, Lq, Hq, d_v, device=dev, dtype=torch_dt)
+    scale = d_qk ** -0.5
+    ws = _ws(ic.sparse_attn_workspace_size(rows, k, Hq, d_qk, d_v, DT[dtype]), dev)
+    ic.sparse_attn(q, kmat, ks, vmat, vs, idx, rows, d_v, scale, out, ws)
+    torch.cuda.synchronize()
+    assert ic.read_status(ws) == 0
+    K = host64(kmat)
+    V = host64(vmat)[..., :d_v] if latent else host64(vmat)
+    ref = oracle.sparse_attention(host64(q), K, V, host64(idx), scale)
+    check_attention(host64(out), ref, "attention")
+
+
+def test_attention_flags_and_skips_out_of_range_indices(dev):
+    rows = (1, 4, 10, 14)
+    B, Lq, q_start, T = rows
+    g = torch.Generator(device=dev).manual_seed(0)
+    q = torch.randn(B, Lq, 8, 64, device=dev, generator=g)
+    K = torch.randn(B, T, 64, device=dev, generator=g)
+    V = torch.randn(B, T, 64, device=dev, generator=g)
+    idx = torch.tensor([[[0, 3, 11, -1], [1, 2, 99, -1], [4, -5, 6, 7], [0, 1, 2, 3]]],
+                       dtype=torch.int32, device=dev)   # 11 > t=10, 99 >= T, -5 < -1
+    out = torch.empty(B, Lq, 8, 64, device=dev)
+    ws = _ws(ic.sparse_attn_workspace_size(rows, 4, 8, 64, 64, ic.F32), dev)
+    ic.sparse_attn(q, K, 64, V, 64, idx, rows, 64, 0.125, out, ws)
+    torch.cuda.synchronize()
+    assert ic.read_status(ws) & 1
+    clean = host64(idx).copy()
+    clean[0, 0, 2] = clean[0, 1, 2] = clean[0, 2, 1] = -1
+    ref = oracle.sparse_attention(host64(q), host64(K), host64(V), clean, 0.125)
+    check_attention(host64(out), ref, "out-of-range skip")
+    assert ic.read_status(ws) == 0                       # cleared by the read
+
+
+# ------------------------------------------------------------------------- stack
+def _stack_inputs(wl, dev, layers=None):
+    n = wl.n_layers if layers is None else layers
+    return [synth.layer_inputs(wl, l, dev) for l in range(n)]
+
+
+def _run_stack(wl, pattern, inputs, dev, rows=None, idx_out=True):
+    B, L, q_start, T = (wl.B, wl.L, wl.q_start, wl.T) if rows is None else rows
+    r = ic.Rows(B, L, q_start, T)
+    sh = ic.StackShape(r, wl.H_I, wl.d_I, DT[wl.idx_dtype], wl.k, wl.Hq, wl.d_qk, wl.d_v,
+                       DT[wl.attn_dtype], wl.d_qk, wl.d_qk if wl.latent else wl.d_v, wl.scale)
+    ws = _ws(ic.workspace_size(sh), dev)
+    torch_dt = torch.float32 if wl.attn_dtype == "f32" else torch.bfloat16
+    idx_buf = torch.empty(B, L, wl.k, dtype=torch.int32, device=dev)
+    outs = [torch.empty(B, L, wl.Hq, wl.d_v, dtype=torch_dt, device=dev) for _ in pattern]
+    idx_copies = [torch.empty_like(idx_buf) for _ in pattern] if idx_out else None
+    layers = []
+    for l, inp in enumerate(inputs):
+        kmat = inp["kv"] if wl.latent else inp["k"]
+        vmat = inp["kv"] if wl.latent else inp["v"]
+        layers.append(dict(q_idx=inp.get("q_I"), q_scale=inp.get("q_scale"), w=inp.get("w"),
+                           k_idx=inp.get("k_I"), k_scale=inp.get("k_scale"), q=inp["q"],
+                           kmat=kmat, vmat=vmat, out=outs[l]))
+    before = ic.kernel_launches(1)
+    ic.layer_stack_forward(pattern, layers, sh, idx_buf, ws, idx_out=idx_copies)
+    torch.cuda.synchronize()
+    n_indexer = ic.kernel_launches(1) - before
+    assert ic.read_status(ws) == 0
+    return outs, idx_copies, n_indexer
+
+
+def _oracle_layers(wl, inputs, rows=None):
+    res = []
+    for inp in inputs:
+        d = dict(q=host64(inp["q"]))
+        if wl.latent:
+            kv = host64(inp["kv"])
+            d["K"], d["V"] = kv, kv[..., : wl.d_v]
+        else:
+            d["K"], d["V"] = host64(inp["k"]), host64(inp["v"])
+        for key in ("q_I", "w", "k_I", "q_scale", "k_scale"):
+            if key in inp:
+                d[key] = host64(inp[key])
+        res.append(d)
+    return res
+
+
+@pytest.mark.parametrize("pattern", ["FSSS", "FFFF", "FSFS"])
+def test_prefill_512_fp32_stack_every_row(dev, pattern):
+    wl = synth.WORKLOADS["prefill_512_fp32"]
+    inputs = _stack_inputs(wl, dev)
+    outs, idx_copies, n_ix = _run_stack(wl, pattern, inputs, dev)
+    assert n_ix == pattern.count("F")                           # indexer runs on F layers only
+    ol = _oracle_layers(wl, inputs)
+    last_f = 0
+    for l, kind in enumerate(pattern):
+        gidx = host64(idx_copies[l])
+        if kind == "F":
+            last_f = l
+            sc = oracle.indexer_scores(ol[l]["q_I"], ol[l]["w"], ol[l]["k_I"], wl.q_start)
+            differ = check_topk_band(gidx, sc, wl.q_start, wl.k)
+            ref_idx = oracle.topk_indices(sc, wl.q_start, wl.k)
+        else:                                                   # invariant: reuse, bit for bit
+            assert np.array_equal(gidx, host64(idx_copies[last_f]))
+        same = np.all(gidx == ref_idx, axis=-1)                 # rows with the oracle's exact set
+        ref = oracle.sparse_attention(ol[l]["q"], ol[l]["K"], ol[l]["V"], ref_idx, wl.scale)
+        check_attention(host64(outs[l])[same], ref[same], "layer %d" % l)
+        assert same.mean() > 0.95, same.mean()
+    del differ
+
+
+def test_exact_mode_stack_is_bit_exact_in_indices(dev):
+    """Exact-mode indexer inputs in a 2-layer bf16 stack: GPU indices equal
+    the oracle's for every row, and the S layer reuses them."""
+    B, L, T, H_I, d_I, k = 1, 300, 300, 64, 128, 64
+    wl = synth.Workload("exact", B, L, T, 0, H_I, d_I, k, 8, 64, 64, "bf16", "bf16", False, "FS",
+                        9, 1, 1, 1, 1, 1)
+    inputs = []
+    for l in range(2):
+        inp = synth.exact_indexer_inputs(B, L, T, H_I, d_I, "bf16", dev, seed=20 + l)
+        g = torch.Generator(device=dev).manual_seed(l)
+        inp["q"] = torch.randn(B, L, 8, 64, device=dev, generator=g).bfloat16()
+        inp["k"] = torch.randn(B, T, 64, device=dev, generator=g).bfloat16()
+        inp["v"] = torch.randn(B, T, 64, device=dev, generator=g).bfloat16()
+        inputs.append(inp)
+    outs, idx_copies, n_ix = _run_stack(wl, "FS", inputs, dev)
+    assert n_ix == 1
+    ol = _oracle_layers(wl, inputs)
+    idx_ref, out_ref, n_ref = oracle.layer_stack("FS", ol, 0, k, wl.scale)
+    assert n_ref == 1
+    for l in range(2):
+        assert np.array_equal(host64(idx_copies[l]), idx_ref[l])
+        check_attention(host64(outs[l]), out_ref[l], "exact layer %d" % l)
+
+
+def test_degenerate_rows(dev):
+    """Single candidate (t = 0), k larger than the context, empty batch."""
+    wl = synth.WORKLOADS["prefill_512_fp32"]
+    inputs = [synth.layer_inputs(wl, 0, dev)]
+    rows = (1, 1, 0, 1)
+    for key in ("q_I", "w", "q"):
+        inputs[0][key] = inputs[0][key][:, :1].contiguous()
+    for key in ("k_I", "k", "v"):
+        inputs[0][key] = inputs[0][key][:, :1].contiguous()
+    outs, idx_copies, _ = _run_stack(wl, "F", inputs, dev, rows=rows)
+    assert host64(idx_copies[0])[0, 0].tolist() == [0] + [-1] * (wl.k - 1)
+    assert np.allclose(host64(outs[0])[0, 0], host64(inputs[0]["v"])[0, 0][None, :], atol=1e-6)
