@@ -1,0 +1,521 @@
+"""Benchmark of the IndexCache hot path on B200.
+
+One step = one pass of the whole layer stack (indexer -> top-k on F layers,
+sparse attention on every layer) over one batch of seeded synthetic input,
+through the C ABI (``ic_layer_stack_forward``).  Default workload:
+prefill_8k_bf16 (1 sequence, L=8192, pattern FSSS); the all-F stack (FFFF)
+is timed on the same inputs for the IndexCache comparison.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--pattern P] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own replica
+of the workload (its own sequences, seed offset by rank), no data-path
+collective; the time is the max over ranks and the value counts all ranks'
+tokens ("scaling": "weak").  ``--impl reference`` times the float64 CPU
+oracle on a bounded sample of the same workload (rank 0 only).
+
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import cross_layer_top_full_b200 as ic  # noqa: E402
+from cross_layer_top_full_b200 import synth  # noqa: E402
+
+DT = {"f32": ic.F32, "bf16": ic.BF16, "e4m3": ic.FP8_E4M3}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p["bf16_tflops_sustained"], "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- workload
+class Stack:
+    """Device-resident inputs and buffers of one replica of a workload."""
+
+    def __init__(self, wl, dev, rank=0):
+        self.wl = wl
+        self.dev = dev
+        if rank:
+            import dataclasses
+            wl = dataclasses.replace(wl, seed=wl.seed + 1000 * rank)
+            self.wl = wl
+        self.inputs = [synth.layer_inputs(wl, l, dev) for l in range(wl.n_layers)]
+        torch_dt = torch.float32 if wl.attn_dtype == "f32" else torch.bfloat16
+        self.outs = [torch.empty(wl.B, wl.L, wl.Hq, wl.d_v, dtype=torch_dt, device=dev)
+                     for _ in range(wl.n_layers)]
+        self.rows = ic.Rows(wl.B, wl.L, wl.q_start, wl.T)
+        self.shape = ic.StackShape(self.rows, wl.H_I, wl.d_I, DT[wl.idx_dtype], wl.k, wl.Hq,
+                                   wl.d_qk, wl.d_v, DT[wl.attn_dtype], wl.d_qk,
+                                   wl.d_qk if wl.latent else wl.d_v, wl.scale)
+        self.ws = torch.empty(ic.workspace_size(self.shape), dtype=torch.uint8, device=dev)
+        ic.workspace_init(self.ws)
+        self.idx = torch.empty(wl.B, wl.L, wl.k, dtype=torch.int32, device=dev)
+        self.layers = self._layer_dicts(self.inputs, self.outs)
+        # per-stage calls (same kernels as the stack) for the stage breakdown
+        self.ld = (wl.T + 3) // 4 * 4
+        self.scores = torch.empty(wl.B, wl.L, self.ld, dtype=torch.float32, device=dev)
+
+    def _layer_dicts(self, inputs, outs):
+        wl = self.wl
+        res = []
+        for l, inp in enumerate(inputs):
+            kmat = inp["kv"] if wl.latent else inp["k"]
+            vmat = inp["kv"] if wl.latent else inp["v"]
+            res.append(dict(q_idx=inp.get("q_I"), q_scale=inp.get("q_scale"), w=inp.get("w"),
+                            k_idx=inp.get("k_I"), k_scale=inp.get("k_scale"), q=inp["q"],
+                            kmat=kmat, vmat=vmat, out=outs[l]))
+        return res
+
+    def step(self, pattern, stream=None):
+        ic.layer_stack_forward(pattern, self.layers, self.shape, self.idx, self.ws, stream=stream)
+
+    def stage_step(self, pattern, ev):
+        """The same step as separate C-ABI calls, with CUDA events around each."""
+        wl = self.wl
+        for l, kind in enumerate(pattern):
+            L = self.layers[l]
+            if kind == "F":
+                e0, e1, e2 = ev.new(), ev.new(), ev.new()
+                e0.record()
+                ic.indexer_scores(L["q_idx"], L["w"], L["k_idx"], self.rows, self.scores, self.ws,
+                                  q_scale=L["q_scale"], k_scale=L["k_scale"],
+                                  dtype=DT[wl.idx_dtype])
+                e1.record()
+                ic.topk(self.scores, self.rows, wl.k, self.idx, self.ws)
+                e2.record()
+                ev.add("indexer", e0, e1)
+                ev.add("topk", e1, e2)
+            e3, e4 = ev.new(), ev.new()
+            e3.record()
+            ic.sparse_attn(L["q"], L["kmat"], wl.d_qk, L["vmat"], wl.d_qk if wl.latent else wl.d_v,
+                           self.idx, self.rows, wl.d_v, wl.scale, L["out"], self.ws,
+                           dtype=DT[wl.attn_dtype])
+            e4.record()
+            ev.add("attention", e3, e4)
+
+    def bytes_per_step(self, pattern):
+        """H2D bytes of one step's inputs (F layers carry indexer inputs)."""
+        n = 0
+        for l, kind in enumerate(pattern):
+            for key, t in self.inputs[l].items():
+                if kind == "S" and key in ("q_I", "w", "k_I", "q_scale", "k_scale"):
+                    continue
+                n += t.numel() * t.element_size()
+        return n
+
+
+class Events:
+    def __init__(self):
+        self.pending = []
+
+    def new(self):
+        return torch.cuda.Event(enable_timing=True)
+
+    def add(self, name, a, b):
+        self.pending.append((name, a, b))
+
+    def collect(self):
+        torch.cuda.synchronize()
+        out = {}
+        for name, a, b in self.pending:
+            out.setdefault(name, []).append(a.elapsed_time(b))
+        self.pending = []
+        return out
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+def algorithmic(wl):
+    """Per-launch algorithmic work of each stage (pages' definitions, all rows)."""
+    rows = [wl.q_start + i for i in range(wl.L)]
+    pairs = wl.B * sum(t + 1 for t in rows)                      # causal (query, key) pairs
+    visits = wl.B * sum(min(wl.k, t + 1) for t in rows)          # selected KV rows visited
+    ib = {"f32": 4, "bf16": 2, "e4m3": 1}[wl.idx_dtype]
+    ab = {"f32": 4, "bf16": 2}[wl.attn_dtype]
+    kv_w = wl.d_qk if wl.latent else wl.d_qk + wl.d_v
+    d = {
+        "indexer_flop": 2.0 * wl.H_I * wl.d_I * pairs,
+        "indexer_bytes": wl.B * (wl.T * wl.d_I * ib + wl.L * wl.H_I * (wl.d_I * ib + 4))
+        + 4.0 * pairs,
+        "topk_bytes": 4.0 * pairs + 4.0 * wl.B * wl.L * wl.k,
+        "attn_flop": 2.0 * wl.Hq * (wl.d_qk + wl.d_v) * visits,
+        "attn_bytes": visits * kv_w * ab + wl.B * wl.L * wl.Hq * (wl.d_qk + wl.d_v) * ab
+        + 4.0 * wl.B * wl.L * wl.k,
+        "pairs": pairs, "visits": visits,
+    }
+    return d
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        load = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": float(np.median(load)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle baseline
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def oracle_sample(wl, pattern, budget_s):
+    """Time the float64 oracle (as it stands) on a bounded sample of the
+    workload: prefill -> blocks of consecutive query rows at random offsets of
+    one sequence; decode -> whole sequences, one at a time.  Inputs are drawn
+    on the CPU with the workload's shapes and distributions (the sample's
+    values differ from the GPU run's, its cost per row does not).  Grows the
+    sample until about budget_s seconds of oracle time.  Returns (rows per
+    second, rows done, seconds)."""
+    import dataclasses
+    import oracle
+    rng = np.random.default_rng(0)
+    done, spent, n = 0, 0.0, 1
+    while spent < budget_s:
+        if wl.L > 1:
+            n = min(n, wl.L)
+            r0 = int(rng.integers(0, wl.L - n + 1))
+            sub = dataclasses.replace(wl, B=1, L=n, q_start=wl.q_start + r0, chunk=0)
+        else:
+            sub = dataclasses.replace(wl, B=1, seed=wl.seed + int(rng.integers(1 << 20)))
+        inputs = _oracle_inputs(sub)
+        t0 = time.perf_counter()
+        oracle.layer_stack(pattern, inputs, sub.q_start, sub.k, sub.scale,
+                           fp8=sub.idx_dtype == "e4m3")
+        dt = time.perf_counter() - t0
+        done += sub.B * sub.L
+        spent += dt
+        if wl.L > 1:
+            n = max(1, min(256, int(n * min(8.0, max(1.5, 0.5 * (budget_s - spent) / max(dt, 1e-3))))))
+    return done / spent, done, spent
+
+
+def _oracle_inputs(wl):
+    res = []
+    for l in range(wl.n_layers):
+        inp = synth.layer_inputs(wl, l, "cpu")
+        d = {}
+        for key in ("q_I", "w", "k_I", "q_scale", "k_scale", "q"):
+            if key in inp:
+                t = inp[key]
+                d[key] = t.numpy() if t.dtype == torch.uint8 else t.double().numpy()
+        if wl.latent:
+            kv = inp["kv"].double().numpy()
+            d["K"], d["V"] = kv, kv[..., : wl.d_v]
+        else:
+            d["K"], d["V"] = inp["k"].double().numpy(), inp["v"].double().numpy()
+        res.append(d)
+    return res
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill_8k_bf16")
+    ap.add_argument("--pattern", default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = synth.WORKLOADS[args.workload]
+    pattern = args.pattern or wl.pattern
+    tokens_per_step = wl.B * wl.L
+
+    if args.impl == "reference":
+        return run_reference(args, wl, pattern, rank, world)
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    st = Stack(wl, dev, rank)
+    all_f = "F" * len(pattern)
+
+    def timed(fn, steps):
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        if pg:
+            t = torch.tensor([ms], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    for _ in range(max(3, args.warmup)):
+        st.step(pattern)
+        st.step(all_f)
+    torch.cuda.synchronize()
+
+    # main timed region: the IndexCache pattern through the C ABI
+    clocks = ClockSampler(local)
+    clocks.start()
+    n0 = ic.kernel_launches(0)
+    ms = timed(lambda: st.step(pattern), args.steps)
+    launches = ic.kernel_launches(0) - n0
+    ms_all_f = timed(lambda: st.step(all_f), args.steps)
+    clk = clocks.stop()
+
+    # stage breakdown (same kernels as separate calls, events on the launch stream)
+    ev = Events()
+    for _ in range(args.steps):
+        st.stage_step(pattern, ev)
+    stages = ev.collect()
+
+    # end to end from pinned host buffers through the public API
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(st, pattern, args.steps, dev, pg)
+
+    per_step_ms = ms / args.steps
+    value = tokens_per_step * world / (per_step_ms / 1e3)
+    hbm, tf_burst, tf_sus, peak_src = _peaks()
+    work = algorithmic(wl)
+    avg = {k: float(np.mean(v)) for k, v in stages.items()}
+    dom = max(avg, key=lambda k: sum(stages[k]))
+    if dom == "attention":
+        tensor_path = wl.attn_dtype == "bf16"
+        if tensor_path and wl.L > 1:
+            roof = {"bound": "tensor", "achieved": work["attn_flop"] / (avg[dom] * 1e-3) / 1e12,
+                    "peak": tf_sus, "unit": "TFLOP/s"}
+        else:
+            roof = {"bound": "hbm", "achieved": work["attn_bytes"] / (avg[dom] * 1e-3) / 1e9,
+                    "peak": hbm, "unit": "GB/s"}
+    elif dom == "indexer":
+        if wl.L > 1:
+            roof = {"bound": "tensor", "achieved": work["indexer_flop"] / (avg[dom] * 1e-3) / 1e12,
+                    "peak": tf_sus, "unit": "TFLOP/s"}
+        else:
+            roof = {"bound": "hbm", "achieved": work["indexer_bytes"] / (avg[dom] * 1e-3) / 1e9,
+                    "peak": hbm, "unit": "GB/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": work["topk_bytes"] / (avg[dom] * 1e-3) / 1e9,
+                "peak": hbm, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dom
+    roof["ms_per_launch"] = avg[dom]
+    roof["peak_source"] = "%s (%s)" % (peak_src, "sustained bf16" if roof["unit"] == "TFLOP/s"
+                                       else "copy bandwidth")
+    roof["traffic"] = _traffic(dom, args.workload)
+
+    if rank != 0:
+        _finish(pg)
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rps, done, spent = oracle_sample(wl, pattern, args.cpu_budget)
+        cpu = {"value": rps, "unit": "tok/s", "cores": _blas_threads(), "kind": "oracle",
+               "sample": "%d query rows of %s through all %d layers of %s (float64 NumPy, %.1f s)"
+                         % (done, wl.name, len(pattern), pattern, spent)}
+    line = {
+        "metric": "prefill tok/s (IndexCache pattern) with all-F comparison; roofline of the "
+                  "dominant kernel" if wl.L > 1 else "decode tok/s (IndexCache pattern)",
+        "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": per_step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.attn_dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "pattern": pattern, "B": wl.B, "L": wl.L, "T": wl.T,
+                   "H_I": wl.H_I, "d_I": wl.d_I, "k": wl.k, "Hq": wl.Hq, "d_qk": wl.d_qk,
+                   "d_v": wl.d_v, "indexer_dtype": wl.idx_dtype, "parallelism": "replicas x%d" % world,
+                   "l2": "inputs larger than L2 (%.2f GB read per step)" % (st.bytes_per_step(pattern) / 1e9)},
+        "all_f": {"pattern": all_f, "ms_per_step": ms_all_f / args.steps,
+                  "value": tokens_per_step * world / (ms_all_f / args.steps / 1e3),
+                  "speedup_of_pattern": ms_all_f / ms},
+        "stages_ms": {k: {"per_launch": avg[k], "launches_per_step": len(v) / args.steps}
+                      for k, v in stages.items()},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    _finish(pg)
+
+
+def _traffic(kernel, workload):
+    """DRAM bytes per launch of the kernel from the committed ncu summary of
+    the current kernels (profiles/traffic.json), else None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            return json.load(f).get(workload, {}).get(kernel)
+    except Exception:
+        return None
+
+
+def run_e2e(st, pattern, steps, dev, pg):
+    """Same metric through the public API from pinned host buffers: every step
+    copies that step's inputs host->device, runs the stack and reads the last
+    layer's output back."""
+    host = []
+    h2d = 0
+    for l, kind in enumerate(pattern):
+        d = {}
+        for key, t in st.inputs[l].items():
+            if kind == "S" and key in ("q_I", "w", "k_I", "q_scale", "k_scale"):
+                continue
+            d[key] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            d[key].copy_(t)
+            h2d += t.numel() * t.element_size()
+        host.append(d)
+    out_host = torch.empty(st.outs[-1].shape, dtype=st.outs[-1].dtype, pin_memory=True)
+    d2h = out_host.numel() * out_host.element_size()
+
+    def step():
+        for l, d in enumerate(host):
+            for key, t in d.items():
+                st.inputs[l][key].copy_(t, non_blocking=True)
+        st.step(pattern)
+        out_host.copy_(st.outs[-1], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    world = pg.get_world_size() if pg else 1
+    wl = st.wl
+    del host
+    return {"value": wl.B * wl.L * world / (ms / steps / 1e3), "unit": "tok/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def run_reference(args, wl, pattern, rank, world):
+    if rank != 0:
+        return
+    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(wl, pattern, budget / 4)
+    rates, done_all, spent_all = [], 0, 0.0
+    for _ in range(args.steps):
+        rps, done, spent = oracle_sample(wl, pattern, budget)
+        rates.append(rps)
+        done_all += done
+        spent_all += spent
+    value = done_all / spent_all
+    cores = _blas_threads()
+    line = {
+        "impl": "reference",
+        "metric": "prefill tok/s (IndexCache pattern) with all-F comparison; roofline of the "
+                  "dominant kernel" if wl.L > 1 else "decode tok/s (IndexCache pattern)",
+        "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * wl.B * wl.L / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "pattern": pattern, "B": wl.B, "L": wl.L, "T": wl.T,
+                   "k": wl.k},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                         "sample": "%d sampled query rows of %s through all layers of %s per run "
+                                   "(float64 NumPy)" % (done_all, wl.name, pattern)},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _finish(pg):
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -13,11 +13,13 @@
 
 namespace ic {
 
-static std::atomic<uint64_t> g_launches[5];
+static std::atomic<uint64_t> g_launches[IC_LK_KINDS];
 
 void count_launch(int kind) {
     g_launches[IC_LK_ALL].fetch_add(1, std::memory_order_relaxed);
-    if (kind > 0 && kind < 5) g_launches[kind].fetch_add(1, std::memory_order_relaxed);
+    if (kind == IC_LK_INDEXER_TC) g_launches[IC_LK_INDEXER].fetch_add(1, std::memory_order_relaxed);
+    if (kind == IC_LK_ATTN_TC) g_launches[IC_LK_ATTN].fetch_add(1, std::memory_order_relaxed);
+    if (kind > 0 && kind < IC_LK_KINDS) g_launches[kind].fetch_add(1, std::memory_order_relaxed);
 }
 
 ic_status last_launch_status() {
@@ -108,7 +110,7 @@ const char* ic_status_string(ic_status st) {
 int ic_version(void) { return 10000; }
 
 uint64_t ic_kernel_launches(int kind) {
-    if (kind < 0 || kind > 4) return 0;
+    if (kind < 0 || kind >= IC_LK_KINDS) return 0;
     return g_launches[kind].load(std::memory_order_relaxed);
 }
 

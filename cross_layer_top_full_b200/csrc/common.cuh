@@ -13,7 +13,10 @@
 #define IC_DEV_TIMEOUT 2u
 
 // Launch kinds counted by ic_kernel_launches.
-enum { IC_LK_ALL = 0, IC_LK_INDEXER = 1, IC_LK_TOPK = 2, IC_LK_ATTN = 3, IC_LK_COMBINE = 4 };
+enum {
+    IC_LK_ALL = 0, IC_LK_INDEXER = 1, IC_LK_TOPK = 2, IC_LK_ATTN = 3, IC_LK_COMBINE = 4,
+    IC_LK_INDEXER_TC = 5, IC_LK_ATTN_TC = 6, IC_LK_KINDS = 7
+};
 
 namespace ic {
 

@@ -91,8 +91,10 @@ ic_status ic_workspace_init(void* ws, size_t ws_bytes, void* stream);
 ic_status ic_read_status(void* ws, void* stream, int32_t* device_status);
 
 /* Number of kernels this library has launched in this process, by kind:
- * 0 = all, 1 = indexer, 2 = top-k, 3 = attention, 4 = split-k combine.
- * A host-side diagnostic counter (thread-safe). */
+ * 0 = all, 1 = indexer, 2 = top-k, 3 = attention, 4 = split-k combine,
+ * 5 = indexer launches that took the tensor-core path, 6 = attention
+ * launches that took the tensor-core path.  A host-side diagnostic counter
+ * (thread-safe). */
 uint64_t ic_kernel_launches(int kind);
 
 /* ------------------------------------------------------------------------ */

@@ -33,10 +33,14 @@ def _gpu_scores(inp, rows, dtype, dev):
     B, Lq, q_start, T = rows
     ld = (T + 3) // 4 * 4
     scores = torch.full((B, Lq, ld), float("nan"), device=dev)
-    ws = _ws(ic.indexer_workspace_size(rows, inp["q_I"].shape[-2], inp["q_I"].shape[-1], DT[dtype]), dev)
+    H_I, d_I = inp["q_I"].shape[-2], inp["q_I"].shape[-1]
+    ws = _ws(ic.indexer_workspace_size(rows, H_I, d_I, DT[dtype]), dev)
+    tc0 = ic.kernel_launches(5)
     ic.indexer_scores(inp["q_I"], inp["w"], inp["k_I"], rows, scores, ws,
                       q_scale=inp.get("q_scale"), k_scale=inp.get("k_scale"), dtype=DT[dtype])
     torch.cuda.synchronize()
+    tensor_core = dtype != "f32" and d_I == 128 and H_I in (16, 32, 64, 128)
+    assert ic.kernel_launches(5) - tc0 == (1 if tensor_core else 0)
     assert ic.read_status(ws) == 0
     return scores
 
@@ -138,6 +142,30 @@ def test_sparse_attention_within_tolerance(dev, dtype, Hq, d_qk, d_v, latent):
     V = host64(vmat)[..., :d_v] if latent else host64(vmat)
     ref = oracle.sparse_attention(host64(q), K, V, host64(idx), scale)
     check_attention(host64(out), ref, "attention")
+
+
+@pytest.mark.parametrize("rows,k", [((3, 1, 999, 1000), 512),      # decode: split-k + combine
+                                    ((2, 3, 4000, 4003), 2048),    # few rows, long k
+                                    ((1, 160, 0, 160), 64),        # prefill, early rows short
+                                    ((2, 1, 40, 41), 2048)])       # fewer keys than k
+def test_latent_attention_tensor_core_path(dev, rows, k):
+    B, Lq, q_start, T = rows
+    g = torch.Generator(device=dev).manual_seed(k + T)
+    q = torch.randn(B, Lq, 128, 576, device=dev, generator=g).bfloat16()
+    kv = (torch.randn(B, T, 576, device=dev, generator=g) / 24 ** 0.5).bfloat16()
+    idx = synth.random_index_sets(B, Lq, q_start, k, dev, seed=k)
+    if Lq > 1:
+        idx[0, 1, 5:9] = -1                      # holes inside a row are masked
+    out = torch.empty(B, Lq, 128, 512, device=dev, dtype=torch.bfloat16)
+    ws = _ws(ic.sparse_attn_workspace_size(rows, k, 128, 576, 512, ic.BF16), dev)
+    n0, tc0 = ic.kernel_launches(3), ic.kernel_launches(6)
+    ic.sparse_attn(q, kv, 576, kv, 576, idx, rows, 512, 576 ** -0.5, out, ws)
+    torch.cuda.synchronize()
+    assert ic.kernel_launches(3) - n0 == 1 and ic.kernel_launches(6) - tc0 == 1
+    assert ic.read_status(ws) == 0
+    kvh = host64(kv)
+    ref = oracle.sparse_attention(host64(q), kvh, kvh[..., :512], host64(idx), 576 ** -0.5)
+    check_attention(host64(out), ref, "latent attention")
 
 
 def test_attention_flags_and_skips_out_of_range_indices(dev):
