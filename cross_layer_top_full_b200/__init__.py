@@ -20,7 +20,8 @@ __all__ = [
     "F32", "BF16", "FP8_E4M3", "STATUS_BYTES",
     "status_string", "version", "kernel_launches", "workspace_init", "read_status",
     "indexer_workspace_size", "indexer_scores", "topk_workspace_size", "topk",
-    "sparse_attn_workspace_size", "sparse_attn", "workspace_size", "layer_stack_forward",
+    "sparse_attn_workspace_size", "sparse_attn", "sparse_attn_noalloc", "workspace_size",
+    "layer_stack_forward",
 ]
 
 F32, BF16, FP8_E4M3 = 0, 1, 2
@@ -77,6 +78,8 @@ _SIG = {
     "ic_sparse_attn": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P, ctypes.c_int64, _P, ctypes.c_int,
                                       ctypes.c_int, Rows, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+    "ic_sparse_attn_noalloc": (ctypes.c_int, [_P, _P, _P, ctypes.c_int, Rows, ctypes.c_float, _P,
+                                              _P, _P]),
     "ic_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(StackShape)]),
     "ic_layer_stack_forward": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_int,
                                               ctypes.POINTER(LayerIO), ctypes.POINTER(StackShape),
@@ -213,6 +216,18 @@ def sparse_attn(q, kmat, k_row_stride: int, vmat, v_row_stride: int, idx, rows, 
                                 _ptr(idx), k, dt, _rows(rows), Hq, d_qk, d_v, float(scale),
                                 _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream)),
            "ic_sparse_attn")
+
+
+def sparse_attn_noalloc(q, kv, idx, rows, scale: float, out, *, device_status=None,
+                        stream=None) -> None:
+    """Latent sparse MQA attention (bf16, 128 heads, 576-wide KV rows) without
+    a workspace: for callers that may not allocate device memory.  Its split-k
+    partials live in a fixed device array inside the library, shared by all
+    calls (serialise calls on one stream)."""
+    k = idx.shape[-1]
+    _check(lib().ic_sparse_attn_noalloc(_ptr(q), _ptr(kv), _ptr(idx), k, _rows(rows),
+                                        float(scale), _ptr(out), _ptr(device_status),
+                                        _stream(stream)), "ic_sparse_attn_noalloc")
 
 
 def workspace_size(shape: StackShape) -> int:

@@ -181,6 +181,36 @@ ic_status ic_sparse_attn(const void* q, const void* kmat, int64_t k_row_stride,
                          ic_dtype dt, ic_rows r, int Hq, int d_qk, int d_v, float scale,
                          void* out, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Workspace-free variant of ic_sparse_attn for the latent MQA layout
+ * (IC_BF16, Hq = 128, d_qk = 576, d_v = 512, K and V rows in one 576-wide
+ * KV row: kv + (b*T + s)*576).  The IndexCache pages have no counterpart of
+ * this call; it exists for callers that may not allocate device memory where
+ * they run attention (an engine whose memory pool owns the whole GPU, a
+ * plugin that only receives input and output buffers, a step where a
+ * cudaMalloc and its possible device synchronisation are not acceptable).
+ *
+ * Same arguments, layouts and results as ic_sparse_attn with
+ * kmat = vmat = kv and row strides 576, except that the split-k partials of
+ * decode live in a fixed device array inside the library of
+ * IC_NOALLOC_SCRATCH_BYTES bytes (about 16 MiB; every GPU that loads the
+ * library holds it until the process exits), enough for
+ * B*Lq*splits <= 64 partial rows.  A call that would need more returns
+ * IC_ERR_WORKSPACE before launching anything; use ic_sparse_attn with a
+ * workspace instead.  This function allocates nothing.
+ *   device_status  NULL, or a DEVICE int32 that receives the call's status
+ *                  bits (as ic_read_status reports them) when it completes.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the array and it keeps the last call's contents
+ * (the status word is cleared at the start of each call): calls whose kernels
+ * overlap on the GPU race on it, so serialise them (one stream, one thread).
+ */
+#define IC_NOALLOC_SCRATCH_BYTES ((16u << 20) + (64u << 10) + 512u)
+ic_status ic_sparse_attn_noalloc(const void* q, const void* kv, const int32_t* idx, int k,
+                                 ic_rows r, float scale, void* out, int32_t* device_status,
+                                 void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* a3  The layer stack with the F/S branch                                   */
 /* ------------------------------------------------------------------------ */
