@@ -10,12 +10,17 @@
   score, every position scoring above tau + 1e-3|tau| is kept and every kept
   position scores at least tau - 1e-3|tau|; no duplicates, all in [0, t],
   ascending, -1 padded, exactly min(k, t+1) kept.
-* attention: max |gpu - oracle| <= 1e-2 and ||gpu - oracle||_2 <= 1e-2 ||oracle||_2.
+* attention: "within 1e-2 max abs and 1e-2 relative" read elementwise as
+  |gpu - oracle| <= 1e-2 + 1e-2 |oracle| (the allclose form), plus the
+  aggregate ||gpu - oracle||_2 <= 1e-2 ||oracle||_2.  A pure 1e-2 absolute
+  bound cannot hold for bf16 outputs of magnitude >= 2, whose rounding step
+  alone is 2^-7 or more.
 """
 import numpy as np
 import torch
 
-ATTN_MAX_ABS = 1e-2
+ATTN_ATOL = 1e-2
+ATTN_RTOL = 1e-2
 ATTN_REL_L2 = 1e-2
 TOPK_BAND = 1e-3
 
@@ -89,7 +94,11 @@ def check_topk_band(idx: np.ndarray, ref_scores: np.ndarray, q_start: int, k: in
 
 def check_attention(gpu: np.ndarray, ref: np.ndarray, what: str = "") -> None:
     d = np.abs(gpu - ref)
-    mx = float(d.max()) if d.size else 0.0
+    excess = d - (ATTN_ATOL + ATTN_RTOL * np.abs(ref))
+    worst = float(excess.max()) if d.size else -1.0
     rel = float(np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-30))
-    assert mx <= ATTN_MAX_ABS, "%s max|diff| = %g" % (what, mx)
+    if worst > 0:
+        at = np.unravel_index(int(np.argmax(excess)), d.shape)
+        raise AssertionError("%s |diff| %g > %g + %g*|ref| at %s (ref %g)"
+                             % (what, d[at], ATTN_ATOL, ATTN_RTOL, at, ref[at]))
     assert rel <= ATTN_REL_L2, "%s rel L2 = %g" % (what, rel)
