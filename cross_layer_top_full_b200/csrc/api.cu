@@ -6,6 +6,7 @@
 // the cache unchanged, every layer runs sparse attention (IndexCache summary,
 // es page, section 2 "Arquitectura del Método"; it page, section 2
 // "Architettura e Funzionamento").
+#include <algorithm>
 #include <atomic>
 #include <cstring>
 
@@ -73,6 +74,15 @@ ic_status run_indexer(const void* q_idx, const float* q_scale, const float* w, c
         return launch_indexer_tc(q_idx, q_scale, w, k_idx, k_scale, dt, r, H_I, d_I, scores, ld,
                                  status, s);
     return launch_indexer_simt(q_idx, q_scale, w, k_idx, k_scale, dt, r, H_I, d_I, scores, ld, s);
+}
+
+ic_status run_topk(const float* scores, int64_t ld, ic_rows r, int k, int32_t* idx, void* scratch,
+                   size_t scratch_bytes, cudaStream_t s) {
+    // the multi-CTA path reads 16-byte vectors: it needs 16-byte aligned rows
+    if (topk_multi_applies(r, k) && scratch != nullptr && ((uintptr_t)scores & 15) == 0 &&
+        scratch_bytes >= topk_multi_scratch_bytes(r, k))
+        return launch_topk_multi(scores, ld, r, k, idx, scratch, s);
+    return launch_topk_rows(scores, ld, r, k, idx, s);
 }
 
 ic_status run_attn(const void* q, const void* kmat, int64_t ks, const void* vmat, int64_t vs,
@@ -159,8 +169,7 @@ ic_status ic_indexer_scores(const void* q_idx, const float* q_scale, const float
 }
 
 size_t ic_topk_workspace_size(ic_rows r, int k) {
-    (void)r; (void)k;
-    return IC_STATUS_BYTES;
+    return IC_STATUS_BYTES + align_up(topk_multi_scratch_bytes(r, k));
 }
 
 ic_status ic_topk(const float* scores, int64_t ld_scores, ic_rows r, int k, int32_t* idx,
@@ -170,7 +179,8 @@ ic_status ic_topk(const float* scores, int64_t ld_scores, ic_rows r, int k, int3
     if (!ws_ok(ws, ws_bytes, ic_topk_workspace_size(r, k))) return IC_ERR_WORKSPACE;
     if (rows_empty(r)) return IC_OK;
     if (!scores || !idx) return IC_ERR_INVALID_ARG;
-    return launch_topk(scores, ld_scores, r, k, idx, (cudaStream_t)stream);
+    return run_topk(scores, ld_scores, r, k, idx, scratch_of(ws), ws_bytes - IC_STATUS_BYTES,
+                    (cudaStream_t)stream);
 }
 
 size_t ic_sparse_attn_workspace_size(ic_rows r, int k, int Hq, int d_qk, int d_v, ic_dtype dt) {
@@ -195,8 +205,10 @@ ic_status ic_sparse_attn(const void* q, const void* kmat, int64_t k_row_stride, 
 size_t ic_workspace_size(const ic_stack_shape* sh) {
     if (sh == nullptr) return 0;
     const ic_rows& r = sh->rows;
-    return IC_STATUS_BYTES + align_up(scores_bytes(r)) +
-           align_up(attn_scratch(r, sh->k, sh->Hq, sh->d_qk, sh->d_v, sh->attn_dtype));
+    // top-k and attention run one after the other: they share the scratch region
+    const size_t tail = std::max(align_up(attn_scratch(r, sh->k, sh->Hq, sh->d_qk, sh->d_v, sh->attn_dtype)),
+                                 align_up(topk_multi_scratch_bytes(r, sh->k)));
+    return IC_STATUS_BYTES + align_up(scores_bytes(r)) + tail;
 }
 
 ic_status ic_layer_stack_forward(const char* pattern, int n_layers, const ic_layer_io* layers,
@@ -242,7 +254,7 @@ ic_status ic_layer_stack_forward(const char* pattern, int n_layers, const ic_lay
             ic_status st = run_indexer(L.q_idx, L.q_scale, L.w, L.k_idx, L.k_scale, sh->idx_dtype,
                                        r, sh->H_I, sh->d_I, scores, ld, status, s);
             if (st != IC_OK) return st;
-            st = launch_topk(scores, ld, r, sh->k, idx_buf, s);
+            st = run_topk(scores, ld, r, sh->k, idx_buf, attn_ws, attn_ws_bytes, s);
             if (st != IC_OK) return st;
         }
         ic_status st = run_attn(L.q, L.kmat, sh->k_row_stride, L.vmat, sh->v_row_stride, idx_buf,

@@ -57,8 +57,12 @@ ic_status launch_indexer_tc(const void* q_idx, const float* q_scale, const float
                             int H_I, int d_I, float* scores, int64_t ld, uint32_t* status,
                             cudaStream_t s);
 
-ic_status launch_topk(const float* scores, int64_t ld, ic_rows r, int k, int32_t* idx,
-                      cudaStream_t s);
+ic_status launch_topk_rows(const float* scores, int64_t ld, ic_rows r, int k, int32_t* idx,
+                           cudaStream_t s);
+bool topk_multi_applies(ic_rows r, int k);
+size_t topk_multi_scratch_bytes(ic_rows r, int k);
+ic_status launch_topk_multi(const float* scores, int64_t ld, ic_rows r, int k, int32_t* idx,
+                            void* scratch, cudaStream_t s);
 
 ic_status launch_attn_simt(const void* q, const void* kmat, int64_t ks, const void* vmat,
                            int64_t vs, const int32_t* idx, int k, ic_dtype dt, ic_rows r, int Hq,

@@ -47,10 +47,16 @@ struct Cfg {
     static constexpr int B_BYTES = N * D_I * ESZ;            // one query block
     static constexpr int STAGES_RAW = (SMEM_BUDGET - B_BYTES) / A_BYTES;
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
-    static constexpr int TMEM_COLS = (2 * N) < 32 ? 32 : 2 * N;
+    // One token per accumulator (decode): four accumulators and the two
+    // epilogue warpgroups take alternate key tiles.  Several tokens (prefill):
+    // two accumulators and each warpgroup takes half of every tile's tokens.
+    static constexpr bool ALT_TILES = NTOK == 1;
+    static constexpr int NACC = ALT_TILES ? 4 : 2;
+    static constexpr int TMEM_COLS = (NACC * N) < 32 ? 32 : NACC * N;
     static constexpr int K_STEP_BYTES = 32;                  // K per MMA: 16 bf16 / 32 e4m3
-    static constexpr int EPI_GROUPS = NTOK >= 2 ? 2 : 1;
-    static constexpr int TOK_PER_GROUP = NTOK / EPI_GROUPS;
+    static constexpr int EPI_GROUPS = 2;
+    static constexpr int TOK_PER_GROUP = ALT_TILES ? 1 : NTOK / 2;
+    static constexpr int ACC_EMPTY_ARRIVALS = ALT_TILES ? 4 : 8;
     static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
     static_assert(STAGES >= 2, "pipeline depth");
     static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation is a power of two");
@@ -63,7 +69,7 @@ struct Work {
 struct __align__(8) Bars {
     uint64_t a_full[8], a_empty[8];
     uint64_t b_full, b_empty;
-    uint64_t acc_full[2], acc_empty[2];
+    uint64_t acc_full[4], acc_empty[4];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -97,10 +103,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
                                                ~uintptr_t(1023));
     uint8_t* a_smem = smem;                                  // [STAGES][ATOMS][BM][128B]
     uint8_t* b_smem = a_smem + C::STAGES * C::A_BYTES;       // [ATOMS][N][128B]
-    float* w_smem = reinterpret_cast<float*>(b_smem + C::B_BYTES);   // [NTOK][H]
-    float* qs_smem = w_smem + NTOK * H;                              // [NTOK]
+    // per epilogue warp: its tokens' head weights and query scales
+    float* w_smem = reinterpret_cast<float*>(b_smem + C::B_BYTES);   // [8][TOK_PER_GROUP][H]
+    float* qs_smem = w_smem + N_EPI_WARPS * C::TOK_PER_GROUP * H;    // [8][TOK_PER_GROUP]
     Bars* bars = reinterpret_cast<Bars*>(
-        (reinterpret_cast<uintptr_t>(qs_smem + NTOK) + 15) & ~uintptr_t(15));
+        (reinterpret_cast<uintptr_t>(qs_smem + N_EPI_WARPS * C::TOK_PER_GROUP) + 15) & ~uintptr_t(15));
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -113,9 +120,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
         }
         mbar_init(&bars->b_full, 1);
         mbar_init(&bars->b_empty, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < C::NACC; ++s) {
             mbar_init(&bars->acc_full[s], 1);
-            mbar_init(&bars->acc_empty[s], 4 * C::EPI_GROUPS);
+            mbar_init(&bars->acc_empty[s], C::ACC_EMPTY_ARRIVALS);
         }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
@@ -189,9 +196,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
                 bool ok = true;
                 for (int kt = kt0; kt < kt1; ++kt, ++a_it, ++acc_it) {
                     const int s = a_it % C::STAGES;
-                    const int acc = acc_it & 1;
+                    const int acc = acc_it % C::NACC;
                     if (!mbar_wait(&bars->a_full[s], (a_it / C::STAGES) & 1, status, abort) ||
-                        !mbar_wait(&bars->acc_empty[acc], ((acc_it >> 1) & 1) ^ 1, status, abort)) {
+                        !mbar_wait(&bars->acc_empty[acc], ((acc_it / C::NACC) & 1) ^ 1, status, abort)) {
                         ok = false;
                         break;
                     }
@@ -226,28 +233,31 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
         const int ew = warp - 2;                     // 0..7
         const int group = ew >> 2;                   // which half of the tokens
         const int quad = warp & 3;                   // TMEM lanes 32*quad .. +31
-        const int gt = threadIdx.x - 64 - group * 128;  // thread index within the group
         if (group < C::EPI_GROUPS) {
             uint32_t acc_it = 0;
             for (int id = blockIdx.x; id < wk.n_items; id += gridDim.x) {
                 int b, i0, kt0, kt1;
                 if (!decode_item(id, wk, B, Lq, q_start, NTOK, b, i0, kt0, kt1)) continue;
-                // stage this item's head weights (and query scales) for my tokens
-                asm volatile("bar.sync %0, 128;" ::"r"(1 + group));
-                for (int e = gt; e < C::TOK_PER_GROUP * H; e += 128) {
-                    const int j = group * C::TOK_PER_GROUP + e / H;
-                    const int i = i0 + j;
-                    w_smem[j * H + e % H] = i < Lq ? w[((int64_t)b * Lq + i) * H + e % H] : 0.f;
+                // stage this item's head weights (and query scales) of my tokens
+                // in this warp's own buffer: only the warp itself reads it
+                float* w_w = w_smem + ew * C::TOK_PER_GROUP * H;
+                float* qs_w = qs_smem + ew * C::TOK_PER_GROUP;
+                __syncwarp();
+                const int tok0 = C::ALT_TILES ? 0 : group * C::TOK_PER_GROUP;   // my first token
+                for (int e = lane; e < C::TOK_PER_GROUP * H; e += 32) {
+                    const int i = i0 + tok0 + e / H;
+                    w_w[e] = i < Lq ? w[((int64_t)b * Lq + i) * H + e % H] : 0.f;
                 }
-                if (FP8 && gt < C::TOK_PER_GROUP) {
-                    const int j = group * C::TOK_PER_GROUP + gt;
-                    qs_smem[j] = i0 + j < Lq ? q_scale[(int64_t)b * Lq + i0 + j] : 0.f;
+                if (FP8 && lane < C::TOK_PER_GROUP) {
+                    const int i = i0 + tok0 + lane;
+                    qs_w[lane] = i < Lq ? q_scale[(int64_t)b * Lq + i] : 0.f;
                 }
-                asm volatile("bar.sync %0, 128;" ::"r"(1 + group));
+                __syncwarp();
                 bool ok = true;
                 for (int kt = kt0; kt < kt1; ++kt, ++acc_it) {
-                    const int acc = acc_it & 1;
-                    if (!mbar_wait(&bars->acc_full[acc], (acc_it >> 1) & 1, status, abort)) {
+                    if (C::ALT_TILES && (int)(acc_it & 1) != group) continue;   // the other warpgroup's tile
+                    const int acc = acc_it % C::NACC;
+                    if (!warp_wait(&bars->acc_full[acc], (acc_it / C::NACC) & 1, status, abort)) {
                         ok = false;
                         break;
                     }
@@ -256,7 +266,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
                     const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * C::N;
 #pragma unroll
                     for (int jj = 0; jj < C::TOK_PER_GROUP; ++jj) {
-                        const int j = group * C::TOK_PER_GROUP + jj;
+                        const int j = tok0 + jj;
                         if constexpr (H >= 32) {
 #pragma unroll
                             for (int h0 = 0; h0 < H; h0 += 32) {
@@ -282,9 +292,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
                     if (FP8 && s < T) ks = k_scale[(int64_t)b * T + s];
 #pragma unroll
                     for (int jj = 0; jj < C::TOK_PER_GROUP; ++jj) {
-                        const int j = group * C::TOK_PER_GROUP + jj;
+                        const int j = tok0 + jj;
                         const int i = i0 + j;
-                        const float4* wv = reinterpret_cast<const float4*>(w_smem + j * H);
+                        const float4* wv = reinterpret_cast<const float4*>(w_w + jj * H);
                         float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
                         for (int h = 0; h < H; h += 4) {
@@ -295,7 +305,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
                             acc1 = fmaf(ww.w, fmaxf(d[jj][h + 3], 0.f), acc1);
                         }
                         float sc = acc0 + acc1;
-                        if (FP8) sc *= qs_smem[j] * ks;
+                        if (FP8) sc *= qs_w[jj] * ks;
                         if (i < Lq && s <= q_start + i)
                             scores[((int64_t)b * Lq + i) * ld + s] = sc;
                     }
@@ -376,7 +386,7 @@ ic_status launch_cfg(const void* q_idx, const float* q_scale, const float* w, co
     if (items > 0x7fffffff) return IC_ERR_UNSUPPORTED;
     wk.n_items = (int)items;
     const size_t smem = 1024 + (size_t)C::STAGES * C::A_BYTES + C::B_BYTES +
-                        sizeof(float) * (NTOK * H + NTOK + 4) + sizeof(Bars);
+                        sizeof(float) * (N_EPI_WARPS * C::TOK_PER_GROUP * (H + 1) + 4) + sizeof(Bars);
     auto kern = indexer_tc_kernel<H, NTOK, FP8>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)

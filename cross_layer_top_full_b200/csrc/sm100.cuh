@@ -339,3 +339,109 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 }  // namespace sm100
 }  // namespace ic
+
+namespace ic {
+namespace sm100 {
+
+// Shared-memory matrix descriptor for the 64-byte swizzled K-major layout:
+// rows of 64 B, 8-row core groups 512 B apart, layout type 4 (SWIZZLE_64B).
+__device__ __forceinline__ uint64_t desc_sw64(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)(16u >> 4) << 16;
+    d |= (uint64_t)(512u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)4u << 61;
+    return d;
+}
+
+__device__ __forceinline__ void st_cluster_v4_b32(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                                  uint32_t d) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b),
+                 "r"(c), "r"(d)
+                 : "memory");
+}
+
+}  // namespace sm100
+}  // namespace ic
+
+namespace ic {
+namespace sm100 {
+
+// Asynchronous 16-byte store into another CTA's shared memory; when it lands
+// it counts 16 bytes of transaction on that CTA's mbarrier (no fence or
+// arrive needed on the sending side).
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c,
+                                            uint32_t d, uint32_t cluster_bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+            cluster_addr),
+        "r"(a), "r"(b), "r"(c), "r"(d), "r"(cluster_bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
+// 2^x on the special-function unit (approximate, flushes denormals).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+}  // namespace sm100
+}  // namespace ic
+
+namespace ic {
+namespace sm100 {
+
+// Warp-uniform bounded waits: lane 0 waits, the outcome is broadcast, and
+// __syncwarp orders the other lanes' later reads after lane 0's acquire.
+// Every lane gets the same answer, so a timeout can never leave part of a
+// warp inside a warp-synchronous operation.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                          volatile int* abort) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status, abort) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                                  volatile int* abort) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_cluster(bar, parity, status, abort) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+}  // namespace sm100
+}  // namespace ic
+
+namespace ic {
+namespace sm100 {
+
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into
+// another CTA's shared memory of the cluster; completion is counted in bytes
+// on that CTA's mbarrier.  No multicast.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
+                                                  uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst_cluster),
+        "r"(src_cta), "r"(bytes), "r"(bar_cluster)
+        : "memory");
+}
+
+}  // namespace sm100
+}  // namespace ic

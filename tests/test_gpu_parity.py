@@ -99,6 +99,8 @@ def test_indexer_general_inputs_within_tolerance(dev, dtype):
                                     ((1, 40, 3000, 3040), 2048),  # prefill-like long rows
                                     ((4, 1, 49999, 50000), 2048), # decode rows beyond smem cache
                                     ((3, 1, 32767, 32768), 2048), # decode rows, cached
+                                    ((2, 3, 40000, 40003), 2048), # few long rows of unequal length
+                                    ((1, 2, 199998, 200000), 2048),
                                     ((1, 5, 10, 15), 1)])
 def test_topk_is_bit_exact_on_identical_scores(dev, rows, k, ties):
     B, Lq, q_start, T = rows
@@ -108,6 +110,24 @@ def test_topk_is_bit_exact_on_identical_scores(dev, rows, k, ties):
     ic.topk(scores, rows, k, idx, ws)
     torch.cuda.synchronize()
     ref = oracle.topk_indices(host64(scores), q_start, k)
+    assert np.array_equal(host64(idx), ref)
+
+
+def test_topk_long_rows_of_equal_scores(dev):
+    """Every score equal (a mix of +0.0 and -0.0): the candidate bin of the
+    multi-CTA path overflows and the row is resolved in one CTA; the answer is
+    the k smallest positions."""
+    rows = (2, 1, 99999, 100000)
+    k = 2048
+    g = torch.Generator(device=dev).manual_seed(4)
+    scores = torch.zeros(2, 1, 100000, device=dev)
+    scores[torch.rand(2, 1, 100000, generator=g, device=dev) < 0.5] = -0.0
+    idx = torch.full((2, 1, k), -7, dtype=torch.int32, device=dev)
+    ws = _ws(ic.topk_workspace_size(rows, k), dev)
+    ic.topk(scores, rows, k, idx, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(host64(idx)[:, 0], np.tile(np.arange(k), (2, 1)))
+    ref = oracle.topk_indices(host64(scores), 99999, k)
     assert np.array_equal(host64(idx), ref)
 
 
