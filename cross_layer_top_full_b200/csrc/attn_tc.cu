@@ -14,36 +14,42 @@
 // every selected row (value columns 256r..256r+255 and rope columns
 // 512+32r..512+32r+31), computes the partial logits S_r = Q_r K_r^T on the
 // tensor core, scales them to base-2 units and swaps them with its partner
-// through distributed shared memory as float16 (both CTAs round their own
-// half the same way and add the halves in the same order, so both run the
-// very same online softmax).  Each then accumulates its own 256 value
-// columns, O_r += P V_r, in TMEM.  No key byte is gathered twice and no flop
-// is done twice.
+// through distributed shared memory as float16.  Both CTAs add the two
+// halves in float32 (a commutative single rounding, so both get the very
+// same logits) and run the same online softmax.  Each then accumulates its
+// own 256 value columns, O_r += P V_r, in TMEM.  No key byte is gathered
+// twice and no flop is done twice.
 //
-// Per CTA (416 threads), persistent over work units (one unit = one query
+// Per CTA (352 threads), persistent over work units (one unit = one query
 // row, or one split of a row's indices in decode):
-//   warps 0-3  gather: per unit, one pass over the unit's indices computes
-//              the per-block validity masks and the block count; then
-//              16-byte cp.async of the selected rows' columns into swizzled
-//              tiles (3 stages of 64 keys); invalid rows are zero-filled;
-//   warps 4-11 softmax, two warpgroups (thread = head = TMEM lane; warpgroup
-//              w takes keys 32w..32w+31 of each 64-key block): partial S
-//              from TMEM, rounded to float16 and sent straight into the
-//              partner's tile with st.async (counted in bytes on the
-//              partner's mbarrier, no fence or arrive on the sender), row
-//              max over all 64 keys computed by both warpgroups, online
-//              softmax in base
-//              2 with lazy rescaling (O is rescaled only when the running max
-//              grows by more than 2^8), P as bf16 written back into TMEM over
-//              its S columns, final normalisation and store;
-//   warp 12    TMEM allocation, TMA load of Q_r (the next unit's Q is loaded
-//              while the current unit finishes), single-thread MMA issue:
-//              S(j) = Q_r K_r(j)^T (K = 288), then O += P(j-1) V_r(j-1) with
-//              P read from TMEM ("TS" form), software-pipelined so the tensor
-//              core works on block j while block j-1 is in softmax.
-// TMEM: O at columns 0..255, two S/P buffers at 256..319 and 320..383.
-// Shared memory: Q_r 72 KB, 3 KV stages of 36 KB, 2 float16 logit tiles of
-// 16 KB (written by the partner), per-unit masks, barriers (~219 KB).
+//   warps 0-1  gather: per unit, one pass over the unit's indices computes
+//              the per-block validity masks and the block count; then TMA
+//              four-row gathers (tile::gather4) of the selected rows' columns
+//              into 128-byte-swizzled tiles (3 stages of 64 keys); an
+//              invalid index becomes an out-of-range row, which TMA fills
+//              with zeros;
+//   warps 2-5  exchange (thread = head = TMEM lane): partial S of a 64-key
+//              block from TMEM -> base-2 float16, sent straight into the
+//              partner's inbox with st.async (counted in bytes on the
+//              partner's mbarrier) and stored back into TMEM for the
+//              softmax warps; they run ahead of the softmax warps, so the
+//              exchange latency of block j+1 hides behind the softmax of j;
+//   warps 6-9  softmax (thread = head): own + partner logits, row max,
+//              online softmax in base 2 with lazy rescaling (O is rescaled
+//              only when the running max grows by more than 2^8), P as bf16
+//              into TMEM over the S columns, final normalisation and store;
+//   warp 10    TMEM allocation, TMA load of Q_r (the next unit's Q is loaded
+//              while the current unit finishes), and single-thread issue of
+//              S(j) = Q_r K_r(j)^T (K = 288) as soon as block j is gathered;
+//   warp 11    single-thread issue of O += P(j) V_r(j) and l += P(j) 1 (the
+//              row sums, on the tensor core against a ones operand), P read
+//              from TMEM ("TS" form), as soon as P(j) is ready.  Two issuing
+//              threads keep a P V from waiting behind the gather of a later
+//              block.
+// TMEM: O at columns 0..255, three S/P buffers at 256..447, l at 448..463.
+// Shared memory: Q_r 72 KB, 3 KV stages of 36 KB, 2 float16 inbox tiles of
+// 16 KB (written by the partner), a 2 KB ones operand, per-unit masks,
+// barriers (~221 KB).
 //
 // Decode (few query rows): each row's k indices are split over several CTA
 // pairs, which write unnormalised (O, m, l) partials; a small combine kernel
@@ -70,37 +76,44 @@ constexpr int KV_ATOM = NB * 128;    // one 64-column slice of a key block
 constexpr int KV_ROPE = NB * 64;     // the 32 rope columns of a key block
 constexpr int KV_STAGE = 4 * KV_ATOM + KV_ROPE;     // 36 KB
 constexpr int NSTAGE = 3;
+constexpr int NSBUF = 3;                            // S/P buffers in TMEM
 constexpr int X_TILE = HQ * NB * 2;                 // 16 KB of float16 logits
+constexpr int X_QUAD = X_TILE / 4;                  // the 32 rows of one TMEM lane quadrant
+constexpr int ONES_BYTES = 16 * 128;                // 16 x 64 bf16 ones: the row-sum operand
 constexpr int MAX_UNIT_BLOCKS = 64;                 // at most 4096 indices per unit
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = 4 * Q_ATOM + Q_ROPE;         // 72 KB
 constexpr int OFF_X = OFF_KV + NSTAGE * KV_STAGE;   // partner's float16 logits
-constexpr int OFF_MASK = OFF_X + 2 * X_TILE;
+constexpr int OFF_ONES = OFF_X + 2 * X_TILE;
+constexpr int OFF_MASK = OFF_ONES + ONES_BYTES;
 constexpr int OFF_BARS = OFF_MASK + 2 * MAX_UNIT_BLOCKS * 8;
-constexpr int N_THREADS = 416;
+constexpr int N_THREADS = 384;                      // 2 gather, 4 exchange, 4 softmax, 2 MMA warps
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t TM_O = 0;
-constexpr uint32_t TM_S = 256;                      // S/P buffer s at TM_S + 64 s
+constexpr uint32_t TM_S = 256;                      // S/P buffer b at TM_S + 64 b
+constexpr uint32_t TM_L = TM_S + 64 * NSBUF;        // 16 columns, all equal to l
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_THRESHOLD = 8.f;            // log2 units
-constexpr float HALF_MAX = 65504.f;
+static_assert(OFF_ONES % 1024 == 0, "ones operand alignment");
+static_assert(TM_L + 16 <= TMEM_COLS, "tensor memory budget");
 
 struct __align__(8) AttnBars {
     uint64_t q_full, q_empty;
     uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
-    uint64_t s_full[2], s_free[2];
-    uint64_t p_full[2];
-    uint64_t x_full[2];
-    uint64_t o_done, o_final, o_free;
+    uint64_t s_full[NSBUF], s_free[NSBUF];
+    uint64_t own_full[NSBUF][4];    // exchange warp q -> softmax warp q: own float16 logits in TMEM
+    uint64_t p_full[NSBUF];         // softmax warps -> MMA: P in TMEM
+    uint64_t x_full[2][4];          // [inbox slot][quad]: the partner's 32 rows (counted in bytes)
+    uint64_t peer_free[2][4];       // the partner's softmax warp q has read its inbox slot
+    uint64_t o_done[2];             // P V of block g finished (barrier g & 1)
+    uint64_t o_final, o_free;
     uint64_t info_full[2], info_empty[2];
-    uint64_t drain;
+    uint64_t drain[2];
+    uint64_t scan_done[2];          // gather warps: per-unit reduction of the last valid index
     uint32_t tmem_base;
     int abort;
     int n_blocks[2];
-    int red[2][4];
-    uint64_t scan_done[2];      // gather warps: per-unit reduction of the last valid index
-    uint64_t l_ready[2];        // softmax warpgroups: per-unit row sums published
-    float half_l[2][2][HQ];     // [unit parity][warpgroup][row] row sum at the end of a unit
+    int red[2][2];
 };
 
 constexpr size_t SMEM_BYTES = 1024 + OFF_BARS + sizeof(AttnBars);
@@ -108,26 +121,37 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 __device__ __forceinline__ bool idx_valid(int v, int t, int T) { return v >= 0 && v <= t && v < T; }
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b, float& ra, float& rb) {
-    __nv_bfloat16 x = __float2bfloat16_rn(a), y = __float2bfloat16_rn(b);
-    ra = __bfloat162float(x);
-    rb = __bfloat162float(y);
-    return (uint32_t)__bfloat16_as_ushort(x) | ((uint32_t)__bfloat16_as_ushort(y) << 16);
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-// float16 pair of two base-2 logits (clamped to the float16 range), and the
-// rounded values back as float
-__device__ __forceinline__ uint32_t pack_half(float a, float b, float& ra, float& rb) {
-    const __half x = __float2half_rn(fminf(fmaxf(a, -HALF_MAX), HALF_MAX));
-    const __half y = __float2half_rn(fminf(fmaxf(b, -HALF_MAX), HALF_MAX));
-    ra = __half2float(x);
-    rb = __half2float(y);
-    return (uint32_t)__half_as_ushort(x) | ((uint32_t)__half_as_ushort(y) << 16);
+// float16 pair {lo = a, hi = b}, saturated to the finite float16 range
+__device__ __forceinline__ uint32_t half2_sat(float a, float b) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
 }
 
-__device__ __forceinline__ void unpack_half(uint32_t w, float& a, float& b) {
-    a = __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
-    b = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+// a (float16, exact in float32) + c, one float32 rounding
+__device__ __forceinline__ float add_f16_f32(unsigned short a, float c) {
+    float d;
+    asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(a), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// both logits of a key pair: own (float16 pair) + partner (float16 pair)
+__device__ __forceinline__ void sum_pair(uint32_t own, uint32_t par, float& s0, float& s1) {
+    const float o0 = __half2float(__ushort_as_half((unsigned short)(own & 0xffffu)));
+    const float o1 = __half2float(__ushort_as_half((unsigned short)(own >> 16)));
+    s0 = add_f16_f32((unsigned short)(par & 0xffffu), o0);
+    s1 = add_f16_f32((unsigned short)(par >> 16), o1);
 }
 
 struct AttnArgs {
@@ -160,6 +184,7 @@ __device__ __forceinline__ Unit decode_unit(const AttnArgs& a, int seq) {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(N_THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_qr,
+               const __grid_constant__ CUtensorMap map_kv, const __grid_constant__ CUtensorMap map_kvr,
                const AttnArgs args) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -179,40 +204,48 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         mbar_init(&bars->q_full, 1);
         mbar_init(&bars->q_empty, 1);
         for (int s = 0; s < NSTAGE; ++s) {
-            mbar_init(&bars->kv_full[s], 128);
+            mbar_init(&bars->kv_full[s], 2);
             mbar_init(&bars->kv_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < NSBUF; ++s) {
             mbar_init(&bars->s_full[s], 1);
             mbar_init(&bars->s_free[s], 1);
-            mbar_init(&bars->p_full[s], 8);
-            mbar_init(&bars->x_full[s], 1);
-            mbar_init(&bars->info_full[s], 1);
-            mbar_init(&bars->info_empty[s], 9);
+            mbar_init(&bars->p_full[s], 4);
+            for (int q = 0; q < 4; ++q) mbar_init(&bars->own_full[s][q], 1);
         }
-        mbar_init(&bars->o_done, 1);
-        mbar_init(&bars->o_final, 1);
-        mbar_init(&bars->o_free, 8);
-        mbar_init(&bars->drain, 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars->scan_done[s], 4);
-            mbar_init(&bars->l_ready[s], 8);
+            for (int q = 0; q < 4; ++q) {
+                mbar_init(&bars->x_full[s][q], 1);
+                mbar_init(&bars->peer_free[s][q], 1);
+            }
+            mbar_init(&bars->o_done[s], 1);
+            mbar_init(&bars->info_full[s], 1);
+            mbar_init(&bars->info_empty[s], 10);
+            mbar_init(&bars->scan_done[s], 2);
         }
+        mbar_init(&bars->o_final, 1);
+        mbar_init(&bars->o_free, 4);
+        mbar_init(&bars->drain[0], 1);
+        mbar_init(&bars->drain[1], 1);
         bars->abort = 0;
         fence_mbar_init();
     }
-    if (warp == 12) tmem_alloc<TMEM_COLS>(&bars->tmem_base);
+    {
+        // the row-sum operand: bf16 ones, read by the tensor core
+        uint32_t* ones = reinterpret_cast<uint32_t*>(smem + OFF_ONES);
+        for (int i = threadIdx.x; i < ONES_BYTES / 4; i += N_THREADS) ones[i] = 0x3f803f80u;
+        fence_proxy_async_smem();
+    }
+    if (warp == 10) tmem_alloc<TMEM_COLS>(&bars->tmem_base);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     cluster_sync();  // the partner's barriers are initialised before any remote arrive
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp < 4) {
+    if (warp < 2) {
         // ------------------------------------------------------------ gather
         const int gt = threadIdx.x;
-        const int krow = gt >> 1;                 // key row of the block this thread fills
-        const int half = gt & 1;                  // which half of the row's 16-byte chunks
         uint32_t g = 0;
         int n = 0;
         for (int seq = pair; seq < args.n_units; seq += n_pairs, ++n) {
@@ -223,7 +256,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             // validity masks of the unit's blocks and its last valid index
             int last = -1;
             const int n_ent = u.e1 - u.e0;
-            for (int base = 0; base < n_ent; base += 128) {
+            for (int base = 0; base < n_ent; base += 64) {
                 const int e = u.e0 + base + gt;
                 const int v = e < u.e1 ? idx_row[e] : -1;
                 const bool ok = idx_valid(v, u.t, args.T);
@@ -239,48 +272,109 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->scan_done[ip]);
             if (!warp_wait(&bars->scan_done[ip], (n >> 1) & 1, status, abort)) break;
-            last = max(max(bars->red[ip][0], bars->red[ip][1]), max(bars->red[ip][2], bars->red[ip][3]));
+            last = max(bars->red[ip][0], bars->red[ip][1]);
             const int nb = last < 0 ? 0 : (last - u.e0) / NB + 1;
             if (gt == 0) {
                 bars->n_blocks[ip] = nb;
                 mbar_arrive(&bars->info_full[ip]);
             }
-            const __nv_bfloat16* kv_b = args.kv + (int64_t)u.b * args.T * KVW;
+            // warp w fills key rows 32w..32w+31 of each block: lane L < 8 gathers
+            // rows 4L..4L+3 of its half with five tile::gather4 copies (four
+            // 64-column value slices and the 32 rope columns)
+            const int oob_row = args.B * args.T;                 // zero-filled by TMA
+            const int grp = lane & 7;
             bool ok_all = true;
             for (int j = 0; j < nb; ++j, ++g) {
                 const int s = g % NSTAGE;
-                const int e = u.e0 + j * NB + krow;
-                const int v = e < u.e1 ? idx_row[e] : -1;   // issued before the wait
+                const int e = u.e0 + j * NB + gt;
+                const int v_lane = e < u.e1 ? idx_row[e] : -1;   // issued before the wait
                 if (!warp_wait(&bars->kv_empty[s], ((g / NSTAGE) & 1) ^ 1, status, abort)) {
                     ok_all = false;
                     break;
                 }
-                const bool ok = idx_valid(v, u.t, args.T);
-                const __nv_bfloat16* src = kv_b + (int64_t)(ok ? v : 0) * KVW;
-                const uint32_t nbytes = ok ? 16u : 0u;
-                const uint32_t stage = smem_base + OFF_KV + s * KV_STAGE;
+                const int row_lane = idx_valid(v_lane, u.t, args.T) ? u.b * args.T + v_lane : oob_row;
+                const int r0 = __shfl_sync(0xffffffffu, row_lane, 4 * grp);
+                const int r1 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 1);
+                const int r2 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 2);
+                const int r3 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 3);
+                if (lane == 0) mbar_arrive_expect_tx(&bars->kv_full[s], KV_STAGE / 2);
+                __syncwarp();
+                if (lane < 8) {
+                    const int krow = 32 * warp + 4 * grp;
+                    const uint32_t stage = smem_base + OFF_KV + s * KV_STAGE;
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {       // value columns: atoms 2*half, 2*half+1
-                    const int a = 2 * half + (c >> 3), ch = c & 7;
-                    cp_async16(stage + a * KV_ATOM + krow * 128 + ((ch ^ (krow & 7)) << 4),
-                               src + r * 256 + a * 64 + ch * 8, nbytes);
+                    for (int a = 0; a < 4; ++a)
+                        tma_gather4(stage + a * KV_ATOM + krow * 128, &map_kv, &bars->kv_full[s],
+                                    (int)r * 256 + a * 64, r0, r1, r2, r3);
+                    tma_gather4(stage + 4 * KV_ATOM + krow * 64, &map_kvr, &bars->kv_full[s],
+                                512 + (int)r * 32, r0, r1, r2, r3);
                 }
-#pragma unroll
-                for (int c = 2 * half; c < 2 * half + 2; ++c)   // rope columns (64-byte rows)
-                    cp_async16(stage + 4 * KV_ATOM + krow * 64 + ((c ^ ((krow >> 1) & 3)) << 4),
-                               src + 512 + r * 32 + c * 8, nbytes);
-                cp_async_arrive_noinc(&bars->kv_full[s]);
             }
             if (!ok_all) break;
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
-    } else if (warp < 12) {
-        // ------------------------------------------------------------ softmax
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ exchange
         const int quad = warp & 3;                // TMEM lanes 32*quad .. +31
-        const int wg = (warp - 4) >> 2;           // warpgroup: keys 32*wg .. 32*wg+31 of a block
         const int h = quad * 32 + lane;           // head of this thread
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
-        const bool arm = warp == 4 && lane == 0;  // arms x_full with the expected bytes
+        const uint32_t x_remote = map_to_rank(smem_base + OFF_X + h * 128, peer);
+        uint32_t g = 0;
+        int n = 0;
+        bool ok = true;
+        for (int seq = pair; seq < args.n_units && ok; seq += n_pairs, ++n) {
+            const int ip = n & 1;
+            if (!warp_wait(&bars->info_full[ip], (n >> 1) & 1, status, abort)) break;
+            const int nb = bars->n_blocks[ip];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->info_empty[ip]);
+            for (int j = 0; j < nb; ++j, ++g) {
+                const int sb = g % NSBUF;
+                const int slot = g & 1;
+                if (!warp_wait(&bars->s_full[sb], (g / NSBUF) & 1, status, abort)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t own[NB / 2];
+                {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(t_lane + TM_S + 64 * sb, r0);
+                    tmem_ld32(t_lane + TM_S + 64 * sb + 32, r1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) {
+                        own[x] = half2_sat(__uint_as_float(r0[2 * x]) * args.scale_log2,
+                                           __uint_as_float(r0[2 * x + 1]) * args.scale_log2);
+                        own[16 + x] = half2_sat(__uint_as_float(r1[2 * x]) * args.scale_log2,
+                                                __uint_as_float(r1[2 * x + 1]) * args.scale_log2);
+                    }
+                }
+                // own float16 logits for the softmax warp of this quadrant (the
+                // store completes while the partner's copy is sent)
+                tmem_st32(t_lane + TM_S + 64 * sb + 32, own);
+                // the partner's softmax warp must have read this inbox slot (block g-2)
+                if (!warp_wait_cluster(&bars->peer_free[slot][quad], ((g >> 1) & 1) ^ 1, status, abort)) {
+                    ok = false;
+                    break;
+                }
+                // row h of the partner's inbox; each 16-byte st.async counts its
+                // bytes on the partner's x_full (no fence or arrive on this side)
+                const uint32_t xr = x_remote + slot * X_TILE;
+                const uint32_t br = map_to_rank(smem_u32(&bars->x_full[slot][quad]), peer);
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_async_v4(xr + ((c ^ (h & 7)) << 4), own[4 * c], own[4 * c + 1], own[4 * c + 2],
+                                own[4 * c + 3], br);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
+            }
+        }
+    } else if (warp < 10) {
+        // ------------------------------------------------------------ softmax
+        const int quad = warp & 3;
+        const int h = quad * 32 + lane;
+        const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+        const uint32_t free_remote0 = map_to_rank(smem_u32(&bars->peer_free[0][quad]), peer);
+        const uint32_t free_remote1 = map_to_rank(smem_u32(&bars->peer_free[1][quad]), peer);
         uint32_t g = 0, o_use = 0;
         int n = 0;
         bool ok = true;
@@ -289,150 +383,129 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             const int ip = n & 1;
             if (!warp_wait(&bars->info_full[ip], (n >> 1) & 1, status, abort)) { ok = false; break; }
             const int nb = bars->n_blocks[ip];
-            float m_use = -INFINITY, l = 0.f;
+            float m_use = 0.f;      // running max (log2 units); meaningful once m_set
+            bool m_set = false;
             for (int j = 0; j < nb; ++j, ++g) {
-                const int s = g & 1;
-                const uint32_t ph = (g >> 1) & 1;
-                if (arm) mbar_arrive_expect_tx(&bars->x_full[s], X_TILE);
-                if (!warp_wait(&bars->s_full[s], ph, status, abort)) { ok = false; break; }
-                tc_fence_after();
-                // own partial logits of all 64 keys -> base-2 units -> float16;
-                // this warpgroup sends its 32 to the partner
-                float xo[NB];
-                uint32_t hw[NB / 2];
-                {
-                    uint32_t r0[32], r1[32];
-                    tmem_ld32(t_lane + TM_S + 64 * s, r0);
-                    tmem_ld32(t_lane + TM_S + 64 * s + 32, r1);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        hw[x] = pack_half(__uint_as_float(r0[2 * x]) * args.scale_log2,
-                                          __uint_as_float(r0[2 * x + 1]) * args.scale_log2,
-                                          xo[2 * x], xo[2 * x + 1]);
-                        hw[16 + x] = pack_half(__uint_as_float(r1[2 * x]) * args.scale_log2,
-                                               __uint_as_float(r1[2 * x + 1]) * args.scale_log2,
-                                               xo[32 + 2 * x], xo[32 + 2 * x + 1]);
-                    }
-                }
-                {
-                    // my warpgroup's 32 values go straight into row h of the
-                    // partner's tile s; each 16-byte st.async counts its bytes on
-                    // the partner's x_full[s] (no fence or arrive on this side)
-                    const uint32_t x_remote = map_to_rank(smem_base + OFF_X + s * X_TILE + h * 128, peer);
-                    const uint32_t bar_remote = map_to_rank(smem_u32(&bars->x_full[s]), peer);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int c = 4 * wg + q;
-                        const uint32_t w0 = wg ? hw[16 + 4 * q] : hw[4 * q];
-                        const uint32_t w1 = wg ? hw[17 + 4 * q] : hw[4 * q + 1];
-                        const uint32_t w2 = wg ? hw[18 + 4 * q] : hw[4 * q + 2];
-                        const uint32_t w3 = wg ? hw[19 + 4 * q] : hw[4 * q + 3];
-                        st_async_v4(x_remote + ((c ^ (h & 7)) << 4), w0, w1, w2, w3, bar_remote);
-                    }
-                }
+                const int sb = g % NSBUF;
+                const int slot = g & 1;
+                if (lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD);
                 const uint32_t m_lo = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j];
                 const uint32_t m_hi = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j + 1];
-                if (!warp_wait_cluster(&bars->x_full[s], ph, status, abort)) { ok = false; break; }
-                const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + s * X_TILE + h * 128);
-                float xs[NB];
+                if (!warp_wait(&bars->own_full[sb][quad], (g / NSBUF) & 1, status, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t own[NB / 2], par[NB / 2];
+                tmem_ld32(t_lane + TM_S + 64 * sb + 32, own);
+                if (!warp_wait_cluster(&bars->x_full[slot][quad], (g >> 1) & 1, status, abort)) {
+                    ok = false;
+                    break;
+                }
+                {
+                    const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + slot * X_TILE + h * 128);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 w4 = xp[c ^ (h & 7)];
-                    const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float p0, p1;
-                        unpack_half(wv[e], p0, p1);
-                        const int kk = 8 * c + 2 * e;
-                        // canonical order: half 0 + half 1 on both CTAs
-                        const float s0 = r == 0 ? xo[kk] + p0 : p0 + xo[kk];
-                        const float s1 = r == 0 ? xo[kk + 1] + p1 : p1 + xo[kk + 1];
-                        const uint32_t mw = kk < 32 ? m_lo : m_hi;
-                        xs[kk] = ((mw >> (kk & 31)) & 1u) ? s0 : -INFINITY;
-                        xs[kk + 1] = ((mw >> ((kk + 1) & 31)) & 1u) ? s1 : -INFINITY;
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 w4 = xp[c ^ (h & 7)];
+                        par[4 * c] = w4.x;
+                        par[4 * c + 1] = w4.y;
+                        par[4 * c + 2] = w4.z;
+                        par[4 * c + 3] = w4.w;
                     }
                 }
-                // row max over all 64 keys (both warpgroups compute it: no exchange)
-                float mx[32];
+                tmem_ld_wait();
+                // full logits of the 64 keys (log2 units), masked keys -> -inf
+                float sv[NB];
 #pragma unroll
-                for (int x = 0; x < 32; ++x) mx[x] = fmaxf(xs[2 * x], xs[2 * x + 1]);
+                for (int x = 0; x < NB / 2; ++x) sum_pair(own[x], par[x], sv[2 * x], sv[2 * x + 1]);
+                if ((m_lo & m_hi) != 0xffffffffu) {
 #pragma unroll
-                for (int w = 16; w > 0; w >>= 1)
+                    for (int kk = 0; kk < NB; ++kk) {
+                        const uint32_t mw = kk < 32 ? m_lo : m_hi;
+                        if (!((mw >> (kk & 31)) & 1u)) sv[kk] = -INFINITY;
+                    }
+                }
+                float mx[21];
 #pragma unroll
-                    for (int x = 0; x < w; ++x) mx[x] = fmaxf(mx[x], mx[x + w]);
-                const float mloc = mx[0];
-                float alpha = 1.f;
+                for (int x = 0; x < 21; ++x) mx[x] = max3(sv[3 * x], sv[3 * x + 1], sv[3 * x + 2]);
+                float mloc = max3(mx[0], mx[1], sv[63]);
+#pragma unroll
+                for (int x = 2; x + 1 < 21; x += 2) mloc = max3(mloc, mx[x], mx[x + 1]);
+                mloc = fmaxf(mloc, mx[20]);
+                // every inbox value of this slot has been consumed (mloc depends on
+                // all of them): hand the slot back to the partner's exchange warp
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote_relaxed(slot ? free_remote1 : free_remote0);
                 bool rescale = false;
-                if (mloc > m_use + RESCALE_THRESHOLD || (m_use == -INFINITY && mloc > -INFINITY)) {
-                    alpha = m_use == -INFINITY ? 0.f : ex2_approx(m_use - mloc);
+                float alpha = 1.f;
+                if (mloc > -INFINITY && (!m_set || mloc > m_use + RESCALE_THRESHOLD)) {
+                    rescale = m_set;             // O and l hold earlier blocks only if m was set
+                    alpha = m_set ? ex2_approx(m_use - mloc) : 0.f;
                     m_use = mloc;
-                    rescale = true;
+                    m_set = true;
                 }
-                uint32_t pw[16];
-                float ps[4] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t pw[NB / 2];
 #pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    const float a0 = wg ? xs[32 + 2 * x] : xs[2 * x];
-                    const float a1 = wg ? xs[33 + 2 * x] : xs[2 * x + 1];
-                    const float p0 = a0 == -INFINITY ? 0.f : ex2_approx(a0 - m_use);
-                    const float p1 = a1 == -INFINITY ? 0.f : ex2_approx(a1 - m_use);
-                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                    pw[x] = *reinterpret_cast<const uint32_t*>(&pb);
-                    ps[x & 3] += __low2float(pb) + __high2float(pb);
-                }
-                l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-                if (rescale && j > 0) {
-                    // O must hold P(j-1) V(j-1) before it is rescaled; each
-                    // warpgroup rescales its 128 of the 256 value columns
-                    if (!warp_wait(&bars->o_done, (g - 1) & 1, status, abort)) { ok = false; break; }
+                for (int x = 0; x < NB / 2; ++x)
+                    pw[x] = pack_bf16(ex2_approx(sv[2 * x] - m_use), ex2_approx(sv[2 * x + 1] - m_use));
+                if (rescale) {
+                    // O and l must hold P V of block g-1 before they are rescaled
+                    if (!warp_wait(&bars->o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, status, abort)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
 #pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < 8; ++c) {
                         uint32_t o[32];
-                        const uint32_t col = TM_O + 128 * wg + 32 * c;
-                        tmem_ld32(t_lane + col, o);
+                        tmem_ld32(t_lane + TM_O + 32 * c, o);
                         tmem_ld_wait();
 #pragma unroll
                         for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-                        tmem_st32(t_lane + col, o);
+                        tmem_st32(t_lane + TM_O + 32 * c, o);
                     }
+                    uint32_t lr[16];
+                    tmem_ld16(t_lane + TM_L, lr);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) lr[x] = __float_as_uint(__uint_as_float(lr[x]) * alpha);
+                    tmem_st16(t_lane + TM_L, lr);
                 }
-                tmem_st16(t_lane + TM_S + 64 * s + 16 * wg, pw);
+                tmem_st32(t_lane + TM_S + 64 * sb, pw);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->p_full[s]);
+                if (lane == 0) mbar_arrive(&bars->p_full[sb]);
             }
             if (!ok) break;
             // ---------------------------------------------------------- unit epilogue
             const bool split = args.splits > 1;
-            bars->half_l[ip][wg][h] = l;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->l_ready[ip]);
-            if (!warp_wait(&bars->l_ready[ip], (n >> 1) & 1, status, abort)) { ok = false; break; }
-            const float l_all = bars->half_l[ip][0][h] + bars->half_l[ip][1][h];
+            float l_all = 0.f;
             if (nb > 0) {
                 if (!warp_wait(&bars->o_final, o_use & 1, status, abort)) { ok = false; break; }
                 tc_fence_after();
+                {
+                    uint32_t lr[16];
+                    tmem_ld16(t_lane + TM_L, lr);
+                    tmem_ld_wait();
+                    l_all = m_set ? __uint_as_float(lr[0]) : 0.f;
+                }
                 const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     uint32_t o[32];
-                    const int ocol = 128 * wg + 32 * c;          // column of O in TMEM
-                    tmem_ld32(t_lane + TM_O + ocol, o);
+                    tmem_ld32(t_lane + TM_O + 32 * c, o);
                     tmem_ld_wait();
-                    const int col = (int)r * 256 + ocol;        // column of the output row
+                    const int col = (int)r * 256 + 32 * c;     // column of the output row
                     if (!split) {
                         uint4* dst = reinterpret_cast<uint4*>(args.out + ((int64_t)u.row * HQ + h) * DV + col);
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
-                            float d0, d1;
                             uint4 pk;
-                            pk.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv, d0, d1);
-                            pk.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv, d0, d1);
-                            pk.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv, d0, d1);
-                            pk.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv, d0, d1);
+                            pk.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+                            pk.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+                            pk.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+                            pk.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
                             dst[v] = pk;
                         }
                     } else {
@@ -449,19 +522,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 ++o_use;
             } else if (!split) {
                 // no valid key: the output row is zero
-                uint4* dst = reinterpret_cast<uint4*>(args.out + ((int64_t)u.row * HQ + h) * DV + r * 256 + 128 * wg);
-                for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+                uint4* dst = reinterpret_cast<uint4*>(args.out + ((int64_t)u.row * HQ + h) * DV + r * 256);
+                for (int v = 0; v < 32; ++v) dst[v] = make_uint4(0, 0, 0, 0);
             }
-            if (split && r == 0 && wg == 0)
-                args.part_ml[(int64_t)u.unit * HQ + h] = make_float2(m_use, nb > 0 ? l_all : 0.f);
+            if (split && r == 0) args.part_ml[(int64_t)u.unit * HQ + h] = make_float2(m_use, l_all);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->info_empty[ip]);
         }
-    } else {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 10) {
+        // ------------------------------------------------------------ S = Q K^T issuer
         if (lane == 0) {
             constexpr uint32_t id_s = idesc_f32acc(1, 1, HQ, NB);            // S = Q K^T
-            constexpr uint32_t id_pv = idesc_f32acc(1, 1, HQ, 256, 0, 1);    // O += P V (V MN-major)
             const uint32_t q_addr = smem_base + OFF_Q;
             uint32_t g = 0, o_use = 0;
             bool issued = false, ok = true;
@@ -475,25 +546,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                                 u.row * HQ);
                 tma_load_2d(smem + OFF_Q + 4 * Q_ATOM, &map_qr, &bars->q_full, 512 + (int)r * 32,
                             u.row * HQ);
-            };
-            auto pv = [&](uint32_t gg, bool first) -> bool {
-                const int s = gg & 1;
-                if (!mbar_wait(&bars->p_full[s], (gg >> 1) & 1, status, abort)) return false;
-                if (first && o_use > 0 &&
-                    !mbar_wait(&bars->o_free, (o_use - 1) & 1, status, abort))
-                    return false;
-                tc_fence_after();
-                const uint32_t v_addr = smem_base + OFF_KV + (gg % NSTAGE) * KV_STAGE;
-#pragma unroll
-                for (int kk = 0; kk < NB / 16; ++kk) {
-                    const uint64_t db = desc_sw128(v_addr + kk * 16 * 128, 8192, 1024);
-                    mma_bf16_ts(tmem + TM_O, tmem + TM_S + 64 * s + kk * 8, db, id_pv,
-                                (!first || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(&bars->kv_empty[gg % NSTAGE]);
-                mma_commit(&bars->s_free[s]);
-                mma_commit(&bars->o_done);
-                return true;
             };
             int n = 0;
             for (int seq = pair; seq < args.n_units && ok; seq += n_pairs, ++n) {
@@ -514,64 +566,101 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 q_loaded_next = false;
                 if (!mbar_wait(&bars->q_full, o_use & 1, status, abort)) break;
                 for (int j = 0; j < nb; ++j, ++g) {
-                    const int s = g & 1;
+                    const int sb = g % NSBUF;
                     const int ks = g % NSTAGE;
                     if (!mbar_wait(&bars->kv_full[ks], (g / NSTAGE) & 1, status, abort) ||
-                        !mbar_wait(&bars->s_free[s], ((g >> 1) & 1) ^ 1, status, abort)) {
+                        !mbar_wait(&bars->s_free[sb], ((g / NSBUF) & 1) ^ 1, status, abort)) {
                         ok = false;
                         break;
                     }
-                    fence_proxy_async_smem();  // cp.async data -> tensor-core reads
                     tc_fence_after();
                     const uint32_t kv_addr = smem_base + OFF_KV + ks * KV_STAGE;
+                    const uint32_t s_tm = tmem + TM_S + 64 * sb;
 #pragma unroll
                     for (int a = 0; a < 4; ++a) {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint64_t da = desc_sw128(q_addr + a * Q_ATOM + kk * 32, 16, 1024);
                             const uint64_t db = desc_sw128(kv_addr + a * KV_ATOM + kk * 32, 16, 1024);
-                            mma_bf16(tmem + TM_S + 64 * s, da, db, id_s, (a | kk) != 0);
+                            mma_bf16(s_tm, da, db, id_s, (a | kk) != 0);
                         }
                     }
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk) {
                         const uint64_t da = desc_sw64(q_addr + 4 * Q_ATOM + kk * 32);
                         const uint64_t db = desc_sw64(kv_addr + 4 * KV_ATOM + kk * 32);
-                        mma_bf16(tmem + TM_S + 64 * s, da, db, id_s, 1u);
+                        mma_bf16(s_tm, da, db, id_s, 1u);
                     }
                     issued = true;
-                    mma_commit(&bars->s_full[s]);
-                    if (j == nb - 1) {
-                        // Q is free once these MMAs finish: fetch the next unit's Q now
-                        mma_commit(&bars->q_empty);
-                        if (seq + n_pairs < args.n_units) {
-                            const int n1 = n + 1;
-                            if (!mbar_wait(&bars->info_full[n1 & 1], (n1 >> 1) & 1, status, abort)) {
-                                ok = false;
-                                break;
-                            }
-                            nb_next = bars->n_blocks[n1 & 1];
-                            mbar_arrive(&bars->info_empty[n1 & 1]);
-                            if (nb_next > 0) {
-                                if (!mbar_wait(&bars->q_empty, o_use & 1, status, abort)) {
-                                    ok = false;
-                                    break;
-                                }
-                                load_q(seq + n_pairs);
-                                q_loaded_next = true;
-                            }
-                        }
-                    }
-                    if (j >= 1 && !pv(g - 1, j == 1)) { ok = false; break; }
+                    mma_commit(&bars->s_full[sb]);
                 }
                 if (!ok) break;
-                if (!pv(g - 1, nb == 1)) break;
+                // Q is free once these MMAs finish: fetch the next unit's Q now
+                mma_commit(&bars->q_empty);
+                if (seq + n_pairs < args.n_units) {
+                    const int n1 = n + 1;
+                    if (!mbar_wait(&bars->info_full[n1 & 1], (n1 >> 1) & 1, status, abort)) break;
+                    nb_next = bars->n_blocks[n1 & 1];
+                    mbar_arrive(&bars->info_empty[n1 & 1]);
+                    if (nb_next > 0) {
+                        if (!mbar_wait(&bars->q_empty, o_use & 1, status, abort)) break;
+                        load_q(seq + n_pairs);
+                        q_loaded_next = true;
+                    }
+                }
+                ++o_use;
+            }
+            if (issued) {
+                mma_commit(&bars->drain[0]);   // every MMA this thread issued has finished
+                mbar_wait(&bars->drain[0], 0, status, abort);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ O += P V, l += P 1 issuer
+        if (lane == 0) {
+            constexpr uint32_t id_pv = idesc_f32acc(1, 1, HQ, 256, 0, 1);    // O += P V (V MN-major)
+            constexpr uint32_t id_l = idesc_f32acc(1, 1, HQ, 16);            // l += P 1
+            const uint32_t ones_addr = smem_base + OFF_ONES;
+            uint32_t g = 0, o_use = 0;
+            bool issued = false, ok = true;
+            int n = 0;
+            for (int seq = pair; seq < args.n_units && ok; seq += n_pairs, ++n) {
+                if (!mbar_wait(&bars->info_full[n & 1], (n >> 1) & 1, status, abort)) break;
+                const int nb = bars->n_blocks[n & 1];
+                mbar_arrive(&bars->info_empty[n & 1]);
+                if (nb == 0) continue;
+                for (int j = 0; j < nb; ++j, ++g) {
+                    const int sb = g % NSBUF;
+                    if (!mbar_wait(&bars->p_full[sb], (g / NSBUF) & 1, status, abort) ||
+                        (j == 0 && o_use > 0 && !mbar_wait(&bars->o_free, (o_use - 1) & 1, status, abort))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t v_addr = smem_base + OFF_KV + (g % NSTAGE) * KV_STAGE;
+                    const uint32_t p_tm = tmem + TM_S + 64 * sb;
+#pragma unroll
+                    for (int kk = 0; kk < NB / 16; ++kk) {
+                        const uint64_t db = desc_sw128(v_addr + kk * 16 * 128, 8192, 1024);
+                        mma_bf16_ts(tmem + TM_O, p_tm + kk * 8, db, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < NB / 16; ++kk) {
+                        const uint64_t dl = desc_sw128(ones_addr + kk * 32, 16, 1024);
+                        mma_bf16_ts(tmem + TM_L, p_tm + kk * 8, dl, id_l, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    issued = true;
+                    mma_commit(&bars->kv_empty[g % NSTAGE]);
+                    mma_commit(&bars->s_free[sb]);
+                    mma_commit(&bars->o_done[g & 1]);
+                }
+                if (!ok) break;
                 mma_commit(&bars->o_final);
                 ++o_use;
             }
             if (issued) {
-                mma_commit(&bars->drain);   // every MMA of this CTA has finished
-                mbar_wait(&bars->drain, 0, status, abort);
+                mma_commit(&bars->drain[1]);
+                mbar_wait(&bars->drain[1], 0, status, abort);
             }
         }
     }
@@ -579,7 +668,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // the partner no longer writes into this CTA's shared memory
-    if (warp == 12) {
+    if (warp == 10) {
         tc_fence_after();
         tmem_dealloc<TMEM_COLS>(tmem);
     }
@@ -708,6 +797,22 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return IC_ERR_CUDA;
 
+    // KV rows for the gathers: one box row of 64 value columns (128-byte
+    // swizzle) or of the 32 rope columns (64-byte swizzle)
+    CUtensorMap map_kv, map_kvr;
+    cuuint64_t kdims[2] = {(cuuint64_t)KVW, (cuuint64_t)r.B * r.T};
+    cuuint32_t kbox[2] = {64, 1};
+    cuuint32_t kbox_r[2] = {32, 1};
+    if ((int64_t)r.B * r.T >= 0x7fffffff) return IC_ERR_UNSUPPORTED;
+    if (fn(&map_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv), kdims, strides, kbox,
+           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return IC_ERR_CUDA;
+    if (fn(&map_kvr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv), kdims, strides, kbox_r,
+           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return IC_ERR_CUDA;
+
     AttnArgs a;
     a.kv = static_cast<const __nv_bfloat16*>(kv);
     a.idx = idx;
@@ -736,7 +841,7 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
                              (int)SMEM_BYTES) != cudaSuccess)
         return IC_ERR_CUDA;
     const int64_t pairs = std::min<int64_t>(units, std::max(1, sm_count() / 2));
-    attn_tc_kernel<<<(unsigned)(2 * pairs), N_THREADS, SMEM_BYTES, s>>>(map_q, map_qr, a);
+    attn_tc_kernel<<<(unsigned)(2 * pairs), N_THREADS, SMEM_BYTES, s>>>(map_q, map_qr, map_kv, map_kvr, a);
     count_launch(IC_LK_ATTN_TC);
     ic_status st = last_launch_status();
     if (st != IC_OK || a.splits <= 1) return st;

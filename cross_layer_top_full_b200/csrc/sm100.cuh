@@ -109,6 +109,20 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
+// Four-row gather (tile::gather4): rows r0..r3 of a 2D tensor map whose box
+// is one row high, columns c0 .. c0 + box width - 1, written as four
+// consecutive box rows at smem_dst (the map's swizzle is applied by address);
+// completion counted on `bar` in bytes.  This CTA only, no multicast.
+__device__ __forceinline__ void tma_gather4(uint32_t smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int r0, int r1, int r2, int r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
+        "r"(r3)
+        : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 template <int NCOLS>
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem) {
@@ -284,6 +298,14 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, f
 // Arrive (release at cluster scope) on an mbarrier of another CTA of the cluster.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+// Remote arrive without release semantics: for a consumer that hands a
+// buffer back after every value it read has been used (so the reads are
+// complete), with no writes of its own to publish.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                  : "memory");
 }
 
