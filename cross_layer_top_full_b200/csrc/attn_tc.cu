@@ -87,7 +87,20 @@ constexpr int OFF_X = OFF_KV + NSTAGE * KV_STAGE;   // partner's float16 logits
 constexpr int OFF_ONES = OFF_X + 2 * X_TILE;
 constexpr int OFF_MASK = OFF_ONES + ONES_BYTES;
 constexpr int OFF_BARS = OFF_MASK + 2 * MAX_UNIT_BLOCKS * 8;
-constexpr int N_THREADS = 384;                      // 2 gather, 4 exchange, 4 softmax, 2 MMA warps
+#ifndef IC_ATTN_GATHER_WARPS
+#define IC_ATTN_GATHER_WARPS 4
+#endif
+#ifndef IC_ATTN_GATHER_TMA
+#define IC_ATTN_GATHER_TMA 1
+#endif
+constexpr int GW = IC_ATTN_GATHER_WARPS;            // gather warps (2 or 4)
+constexpr bool GATHER_TMA = IC_ATTN_GATHER_TMA != 0;  // TMA four-row gathers, else coalesced cp.async
+static_assert(GW == 2 || GW == 4, "gather warps");
+constexpr int KPW = NB / GW;                        // key rows of a block per gather warp
+constexpr int W_X = GW, W_Y = GW + 4, W_S = GW + 8, W_PV = GW + 9;   // first warp of each role
+constexpr int N_THREADS = 32 * (GW + 10);           // gather, 4 exchange, 4 softmax, 2 MMA warps
+constexpr int KV_FULL_ARRIVALS = GATHER_TMA ? GW : 32 * GW;
+static_assert(W_PV + 1 == N_THREADS / 32, "warp roles");
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t TM_O = 0;
 constexpr uint32_t TM_S = 256;                      // S/P buffer b at TM_S + 64 b
@@ -113,7 +126,7 @@ struct __align__(8) AttnBars {
     uint32_t tmem_base;
     int abort;
     int n_blocks[2];
-    int red[2][2];
+    int red[2][4];
 };
 
 constexpr size_t SMEM_BYTES = 1024 + OFF_BARS + sizeof(AttnBars);
@@ -204,7 +217,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         mbar_init(&bars->q_full, 1);
         mbar_init(&bars->q_empty, 1);
         for (int s = 0; s < NSTAGE; ++s) {
-            mbar_init(&bars->kv_full[s], 2);
+            mbar_init(&bars->kv_full[s], KV_FULL_ARRIVALS);
             mbar_init(&bars->kv_empty[s], 1);
         }
         for (int s = 0; s < NSBUF; ++s) {
@@ -221,7 +234,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             mbar_init(&bars->o_done[s], 1);
             mbar_init(&bars->info_full[s], 1);
             mbar_init(&bars->info_empty[s], 10);
-            mbar_init(&bars->scan_done[s], 2);
+            mbar_init(&bars->scan_done[s], GW);
         }
         mbar_init(&bars->o_final, 1);
         mbar_init(&bars->o_free, 4);
@@ -236,14 +249,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         for (int i = threadIdx.x; i < ONES_BYTES / 4; i += N_THREADS) ones[i] = 0x3f803f80u;
         fence_proxy_async_smem();
     }
-    if (warp == 10) tmem_alloc<TMEM_COLS>(&bars->tmem_base);
+    if (warp == W_S) tmem_alloc<TMEM_COLS>(&bars->tmem_base);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     cluster_sync();  // the partner's barriers are initialised before any remote arrive
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp < 2) {
+    if (warp < GW) {
         // ------------------------------------------------------------ gather
         const int gt = threadIdx.x;
         uint32_t g = 0;
@@ -256,7 +269,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             // validity masks of the unit's blocks and its last valid index
             int last = -1;
             const int n_ent = u.e1 - u.e0;
-            for (int base = 0; base < n_ent; base += 64) {
+            for (int base = 0; base < n_ent; base += 32 * GW) {
                 const int e = u.e0 + base + gt;
                 const int v = e < u.e1 ? idx_row[e] : -1;
                 const bool ok = idx_valid(v, u.t, args.T);
@@ -272,47 +285,91 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->scan_done[ip]);
             if (!warp_wait(&bars->scan_done[ip], (n >> 1) & 1, status, abort)) break;
-            last = max(bars->red[ip][0], bars->red[ip][1]);
+            last = bars->red[ip][0];
+#pragma unroll
+            for (int w = 1; w < GW; ++w) last = max(last, bars->red[ip][w]);
             const int nb = last < 0 ? 0 : (last - u.e0) / NB + 1;
             if (gt == 0) {
                 bars->n_blocks[ip] = nb;
                 mbar_arrive(&bars->info_full[ip]);
             }
-            // warp w fills key rows 32w..32w+31 of each block: lane L < 8 gathers
-            // rows 4L..4L+3 of its half with five tile::gather4 copies (four
-            // 64-column value slices and the 32 rope columns)
-            const int oob_row = args.B * args.T;                 // zero-filled by TMA
-            const int grp = lane & 7;
+            // warp w fills key rows KPW*w .. KPW*w + KPW-1 of each block; lane
+            // L < KPW holds the row of key KPW*w + L (the indices of block j+1
+            // are loaded while block j is issued).  An invalid index becomes
+            // the out-of-range row B*T (zero-filled by TMA) or a zero-byte
+            // cp.async source (zero-filled as well).
+            const int oob_row = args.B * args.T;
             bool ok_all = true;
+            const int key = warp * KPW + lane;
+            int v_next = (lane < KPW && u.e0 + key < u.e1) ? idx_row[u.e0 + key] : -1;
             for (int j = 0; j < nb; ++j, ++g) {
                 const int s = g % NSTAGE;
-                const int e = u.e0 + j * NB + gt;
-                const int v_lane = e < u.e1 ? idx_row[e] : -1;   // issued before the wait
+                const int v_lane = v_next;
+                if (j + 1 < nb) {
+                    const int e1 = u.e0 + (j + 1) * NB + key;
+                    v_next = (lane < KPW && e1 < u.e1) ? idx_row[e1] : -1;
+                }
+                const int row_lane = idx_valid(v_lane, u.t, args.T) ? u.b * args.T + v_lane : oob_row;
                 if (!warp_wait(&bars->kv_empty[s], ((g / NSTAGE) & 1) ^ 1, status, abort)) {
                     ok_all = false;
                     break;
                 }
-                const int row_lane = idx_valid(v_lane, u.t, args.T) ? u.b * args.T + v_lane : oob_row;
-                const int r0 = __shfl_sync(0xffffffffu, row_lane, 4 * grp);
-                const int r1 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 1);
-                const int r2 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 2);
-                const int r3 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 3);
-                if (lane == 0) mbar_arrive_expect_tx(&bars->kv_full[s], KV_STAGE / 2);
-                __syncwarp();
-                if (lane < 8) {
-                    const int krow = 32 * warp + 4 * grp;
-                    const uint32_t stage = smem_base + OFF_KV + s * KV_STAGE;
+                const uint32_t stage = smem_base + OFF_KV + s * KV_STAGE;
+                if constexpr (GATHER_TMA) {
+                    // (KPW/4) groups of 4 rows x (four 64-column value slices + the 32
+                    // rope columns) tile::gather4 copies; copy c (group c / 5, slice
+                    // c % 5) is issued by lane c % 32
+                    constexpr int OPS = KPW / 4 * 5;
+                    if (lane == 0) mbar_arrive_expect_tx(&bars->kv_full[s], KPW / 4 * (4 * 512 + 256));
+                    __syncwarp();
 #pragma unroll
-                    for (int a = 0; a < 4; ++a)
-                        tma_gather4(stage + a * KV_ATOM + krow * 128, &map_kv, &bars->kv_full[s],
-                                    (int)r * 256 + a * 64, r0, r1, r2, r3);
-                    tma_gather4(stage + 4 * KV_ATOM + krow * 64, &map_kvr, &bars->kv_full[s],
-                                512 + (int)r * 32, r0, r1, r2, r3);
+                    for (int c0 = 0; c0 < OPS; c0 += 32) {
+                        const int c = c0 + lane;
+                        const int grp = (c < OPS ? c : 0) / 5, sl = c % 5;
+                        const int r0 = __shfl_sync(0xffffffffu, row_lane, 4 * grp);
+                        const int r1 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 1);
+                        const int r2 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 2);
+                        const int r3 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 3);
+                        if (c < OPS) {
+                            const int krow = KPW * warp + 4 * grp;
+                            if (sl < 4)
+                                tma_gather4(stage + sl * KV_ATOM + krow * 128, &map_kv, &bars->kv_full[s],
+                                            (int)r * 256 + sl * 64, r0, r1, r2, r3);
+                            else
+                                tma_gather4(stage + 4 * KV_ATOM + krow * 64, &map_kvr, &bars->kv_full[s],
+                                            512 + (int)r * 32, r0, r1, r2, r3);
+                        }
+                    }
+                } else {
+                    // one warp instruction per row for the 512 value bytes (lane =
+                    // 16-byte chunk), then 8 rows per instruction for the 64 rope bytes
+                    const int a_val = lane >> 3, ch_val = lane & 7;
+#pragma unroll 4
+                    for (int rr = 0; rr < KPW; ++rr) {
+                        const int krow = KPW * warp + rr;
+                        const int row = __shfl_sync(0xffffffffu, row_lane, rr);
+                        const bool valid = row != oob_row;
+                        cp_async16(stage + a_val * KV_ATOM + krow * 128 + ((ch_val ^ (krow & 7)) << 4),
+                                   args.kv + (int64_t)(valid ? row : 0) * KVW + r * 256 + lane * 8,
+                                   valid ? 16u : 0u);
+                    }
+#pragma unroll
+                    for (int i = 0; i < KPW / 8; ++i) {
+                        const int rr = 8 * i + (lane >> 2), chr = lane & 3;
+                        const int krow = KPW * warp + rr;
+                        const int row = __shfl_sync(0xffffffffu, row_lane, rr);
+                        const bool valid = row != oob_row;
+                        cp_async16(stage + 4 * KV_ATOM + krow * 64 + ((chr ^ ((krow >> 1) & 3)) << 4),
+                                   args.kv + (int64_t)(valid ? row : 0) * KVW + 512 + r * 32 + chr * 8,
+                                   valid ? 16u : 0u);
+                    }
+                    cp_async_arrive_noinc(&bars->kv_full[s]);
                 }
             }
             if (!ok_all) break;
         }
-    } else if (warp < 6) {
+        if constexpr (!GATHER_TMA) asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp < W_X + 4) {
         // ------------------------------------------------------------ exchange
         const int quad = warp & 3;                // TMEM lanes 32*quad .. +31
         const int h = quad * 32 + lane;           // head of this thread
@@ -368,7 +425,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
             }
         }
-    } else if (warp < 10) {
+    } else if (warp < W_S) {
         // ------------------------------------------------------------ softmax
         const int quad = warp & 3;
         const int h = quad * 32 + lane;
@@ -529,7 +586,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->info_empty[ip]);
         }
-    } else if (warp == 10) {
+    } else if (warp == W_S) {
         // ------------------------------------------------------------ S = Q K^T issuer
         if (lane == 0) {
             constexpr uint32_t id_s = idesc_f32acc(1, 1, HQ, NB);            // S = Q K^T
@@ -573,6 +630,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                         ok = false;
                         break;
                     }
+                    if constexpr (!GATHER_TMA) fence_proxy_async_smem();  // cp.async data -> tensor core
                     tc_fence_after();
                     const uint32_t kv_addr = smem_base + OFF_KV + ks * KV_STAGE;
                     const uint32_t s_tm = tmem + TM_S + 64 * sb;
@@ -668,7 +726,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // the partner no longer writes into this CTA's shared memory
-    if (warp == 10) {
+    if (warp == W_S) {
         tc_fence_after();
         tmem_dealloc<TMEM_COLS>(tmem);
     }
