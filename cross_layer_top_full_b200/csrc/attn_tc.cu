@@ -266,18 +266,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             const int32_t* idx_row = args.idx + (int64_t)u.row * args.k;
             const int ip = n & 1;
             if (!warp_wait(&bars->info_empty[ip], ((n >> 1) & 1) ^ 1, status, abort)) break;
-            // validity masks of the unit's blocks and its last valid index
+            // validity masks of the unit's blocks and its last valid index; the
+            // loads go out SCAN_BATCH at a time so the scan costs a few memory
+            // round trips, not one per 32*GW indices
             int last = -1;
             const int n_ent = u.e1 - u.e0;
-            for (int base = 0; base < n_ent; base += 32 * GW) {
-                const int e = u.e0 + base + gt;
-                const int v = e < u.e1 ? idx_row[e] : -1;
-                const bool ok = idx_valid(v, u.t, args.T);
-                if (!ok && v != -1 && r == 0) flag_status(status, IC_DEV_INDEX_RANGE);
-                if (ok) last = e;
-                const uint32_t bal = __ballot_sync(0xffffffffu, ok);
-                const int word = base / 32 + warp;
-                if (lane == 0 && word < 2 * MAX_UNIT_BLOCKS) masks[ip * 2 * MAX_UNIT_BLOCKS + word] = bal;
+            constexpr int SCAN_BATCH = 8;
+            for (int base0 = 0; base0 < n_ent; base0 += SCAN_BATCH * 32 * GW) {
+                int v[SCAN_BATCH];
+#pragma unroll
+                for (int q = 0; q < SCAN_BATCH; ++q) {
+                    const int e = u.e0 + base0 + q * 32 * GW + gt;
+                    v[q] = e < u.e1 ? idx_row[e] : -1;
+                }
+#pragma unroll
+                for (int q = 0; q < SCAN_BATCH; ++q) {
+                    const int base = base0 + q * 32 * GW;
+                    if (base >= n_ent) break;
+                    const int e = u.e0 + base + gt;
+                    const bool ok = idx_valid(v[q], u.t, args.T);
+                    if (!ok && v[q] != -1 && r == 0) flag_status(status, IC_DEV_INDEX_RANGE);
+                    if (ok) last = e;
+                    const uint32_t bal = __ballot_sync(0xffffffffu, ok);
+                    const int word = base / 32 + warp;
+                    if (lane == 0 && word < 2 * MAX_UNIT_BLOCKS) masks[ip * 2 * MAX_UNIT_BLOCKS + word] = bal;
+                }
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
