@@ -51,16 +51,35 @@ def _peaks():
 
 
 # ----------------------------------------------------------------------------- workload
+def replica_workload(wl, rank):
+    """The workload replica of one rank: same shapes, its own sequences
+    (seed offset by rank), no data shared between ranks."""
+    import dataclasses
+    return dataclasses.replace(wl, seed=wl.seed + 1000 * rank) if rank else wl
+
+
+def max_over_ranks(ms, pg, dev):
+    """Slowest rank's time (every rank gets it); ``pg`` is torch.distributed
+    or None for one process."""
+    if not pg:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms_per_step):
+    """Units per second processed by all ranks together."""
+    return units_per_rank * world / (ms_per_step / 1e3)
+
+
 class Stack:
     """Device-resident inputs and buffers of one replica of a workload."""
 
     def __init__(self, wl, dev, rank=0):
+        wl = replica_workload(wl, rank)
         self.wl = wl
         self.dev = dev
-        if rank:
-            import dataclasses
-            wl = dataclasses.replace(wl, seed=wl.seed + 1000 * rank)
-            self.wl = wl
         self.inputs = [synth.layer_inputs(wl, l, dev) for l in range(wl.n_layers)]
         torch_dt = torch.float32 if wl.attn_dtype == "f32" else torch.bfloat16
         self.outs = [torch.empty(wl.B, wl.L, wl.Hq, wl.d_v, dtype=torch_dt, device=dev)
@@ -167,6 +186,39 @@ def algorithmic(wl):
     return d
 
 
+def roofline(wl, work, total_ms, launches, per_pass=1):
+    """Roofline line of the dominant stage.  total_ms / launches: summed
+    event time and launch count per stage over the measured passes; work:
+    algorithmic work of one pass of a stage over all rows (``algorithmic``;
+    summed over the chunks of a chunked run), which takes ``per_pass``
+    launches."""
+    hbm, tf_burst, tf_sus, peak_src = _peaks()
+    dom = max(total_ms, key=lambda k: total_ms[k])
+    passes = launches[dom] / per_pass
+    per_pass_ms = total_ms[dom] / passes
+    if dom == "attention":
+        tensor = wl.attn_dtype == "bf16" and wl.L > 1
+        num = work["attn_flop"] if tensor else work["attn_bytes"]
+    elif dom == "indexer":
+        tensor = wl.L > 1
+        num = work["indexer_flop"] if tensor else work["indexer_bytes"]
+    else:
+        tensor = False
+        num = work["topk_bytes"]
+    if tensor:
+        roof = {"bound": "tensor", "achieved": num / (per_pass_ms * 1e-3) / 1e12, "peak": tf_sus,
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": num / (per_pass_ms * 1e-3) / 1e9, "peak": hbm,
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dom
+    roof["ms_per_launch"] = total_ms[dom] / launches[dom]
+    roof["peak_source"] = "%s (%s)" % (peak_src, "sustained bf16" if roof["unit"] == "TFLOP/s"
+                                       else "copy bandwidth")
+    return roof, dom
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     def __init__(self, index):
@@ -248,15 +300,23 @@ def oracle_sample(wl, pattern, budget_s):
     if wl.L == 1 and wl.T * len(pattern) > 2_000_000:
         sub_pattern = pattern[:4]
     layer_share = len(sub_pattern) / len(pattern)
+    dec_inputs = None
     while spent < budget_s:
         if wl.L > 1:
             n = min(n, wl.L)
             r0 = int(rng.integers(0, wl.L - n + 1))
-            sub = dataclasses.replace(wl, B=1, L=n, q_start=wl.q_start + r0, chunk=0)
+            # rows r0..r0+n-1 of one sequence against their causal prefix
+            sub = dataclasses.replace(wl, B=1, L=n, q_start=wl.q_start + r0,
+                                      T=wl.q_start + r0 + n, chunk=0)
+            inputs = _oracle_inputs(sub)
         else:
-            sub = dataclasses.replace(wl, B=1, seed=wl.seed + int(rng.integers(1 << 20)),
-                                      pattern=sub_pattern)
-        inputs = _oracle_inputs(sub)
+            # one sequence, drawn once and timed repeatedly (drawing it costs
+            # more than the oracle pass; the cost per pass does not change)
+            if dec_inputs is None:
+                sub = dataclasses.replace(wl, B=1, seed=wl.seed + int(rng.integers(1 << 20)),
+                                          pattern=sub_pattern)
+                dec_inputs = _oracle_inputs(sub)
+            inputs = dec_inputs
         t0 = time.perf_counter()
         oracle.layer_stack(sub.pattern, inputs, sub.q_start, sub.k, sub.scale,
                            fp8=sub.idx_dtype == "e4m3")
@@ -264,7 +324,11 @@ def oracle_sample(wl, pattern, budget_s):
         done += sub.B * sub.L
         spent += dt
         if wl.L > 1:
-            n = max(1, min(256, int(n * min(8.0, max(1.5, 0.5 * (budget_s - spent) / max(dt, 1e-3))))))
+            # a row's cost grows with its causal length: plan the next block
+            # (at most half the remaining budget) from the cost per row at the
+            # longest prefix the next draw can have
+            per_row_max = dt / n * (wl.q_start + wl.L) / max(1, sub.T)
+            n = max(1, min(256, int(0.5 * (budget_s - spent) / max(per_row_max, 1e-6))))
     return done / spent * layer_share, done, spent
 
 
@@ -322,6 +386,8 @@ def main():
                                 device_id=dev)
         pg = dist
 
+    if wl.chunk:
+        return run_chunked(args, wl, pattern, dev, pg, rank, world)
     st = Stack(wl, dev, rank)
     all_f = "F" * len(pattern)
 
@@ -335,12 +401,7 @@ def main():
             fn()
         b.record()
         torch.cuda.synchronize()
-        ms = a.elapsed_time(b)
-        if pg:
-            t = torch.tensor([ms], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(a.elapsed_time(b), pg, dev)
 
     for _ in range(max(3, args.warmup)):
         st.step(pattern)
@@ -392,35 +453,15 @@ def main():
         e2e = run_e2e(st, pattern, args.steps, dev, pg)
 
     per_step_ms = ms / args.steps
-    value = tokens_per_step * world / (per_step_ms / 1e3)
-    hbm, tf_burst, tf_sus, peak_src = _peaks()
+    value = whole_job_rate(tokens_per_step, world, per_step_ms)
     work = algorithmic(wl)
     avg = {k: float(np.mean(v)) for k, v in stages.items()}
-    dom = max(avg, key=lambda k: sum(stages[k]))
-    if dom == "attention":
-        tensor_path = wl.attn_dtype == "bf16"
-        if tensor_path and wl.L > 1:
-            roof = {"bound": "tensor", "achieved": work["attn_flop"] / (avg[dom] * 1e-3) / 1e12,
-                    "peak": tf_sus, "unit": "TFLOP/s"}
-        else:
-            roof = {"bound": "hbm", "achieved": work["attn_bytes"] / (avg[dom] * 1e-3) / 1e9,
-                    "peak": hbm, "unit": "GB/s"}
-    elif dom == "indexer":
-        if wl.L > 1:
-            roof = {"bound": "tensor", "achieved": work["indexer_flop"] / (avg[dom] * 1e-3) / 1e12,
-                    "peak": tf_sus, "unit": "TFLOP/s"}
-        else:
-            roof = {"bound": "hbm", "achieved": work["indexer_bytes"] / (avg[dom] * 1e-3) / 1e9,
-                    "peak": hbm, "unit": "GB/s"}
-    else:
-        roof = {"bound": "hbm", "achieved": work["topk_bytes"] / (avg[dom] * 1e-3) / 1e9,
-                "peak": hbm, "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["kernel"] = dom
-    roof["ms_per_launch"] = avg[dom]
-    roof["peak_source"] = "%s (%s)" % (peak_src, "sustained bf16" if roof["unit"] == "TFLOP/s"
-                                       else "copy bandwidth")
+    roof, dom = roofline(wl, work, {k: sum(v) for k, v in stages.items()},
+                         {k: len(v) for k, v in stages.items()})
     roof["traffic"] = _traffic(dom, args.workload)
+    # decode: share of the step spent choosing keys (indexer + top-k)
+    total_stage = sum(sum(v) for v in stages.values())
+    sel_share = (sum(stages.get("indexer", [])) + sum(stages.get("topk", []))) / total_stage
 
     if rank != 0:
         _finish(pg)
@@ -448,11 +489,217 @@ def main():
                   "speedup_of_pattern": ms_all_f / ms},
         "stages_ms": {k: {"per_launch": avg[k], "launches_per_step": len(v) / args.steps}
                       for k, v in stages.items()},
+        "indexer_share_of_step": sel_share,
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
         "cuda_graph": bool(args.graph),
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    _finish(pg)
+
+
+def run_chunked(args, wl, pattern, dev, pg, rank, world):
+    """Chunked prefill: the sequence's L query rows go through the layer stack
+    in chunks of wl.chunk rows, chunk c against its causal prefix (q_start =
+    c*chunk, T = (c+1)*chunk), the index cache living per chunk.  One step =
+    every chunk through every layer.  All per-(layer, chunk) queries and all
+    layers' keys stay resident on the device.  After timing, an untimed pass
+    runs every S layer's own indexer and top-k and reports the overlap of its
+    own selection with the reused one (per row: |own & reused| / min(k, t+1)),
+    mean and minimum over all rows, per S layer."""
+    import dataclasses
+    C, nch, nl = wl.chunk, wl.L // wl.chunk, len(pattern)
+    all_f = "F" * nl
+    shared_q = bool(wl.kI_noise)              # indexer queries shared by all layers
+    need = (nl * nch * C * wl.Hq * wl.d_qk * 2 + nl * wl.T * (wl.d_qk + wl.d_I) * 2
+            + (1 if shared_q else nl) * nch * C * wl.H_I * (wl.d_I * 2 + 4)
+            + nl * C * wl.Hq * wl.d_v * 2 + C * wl.T * 4)
+    free = torch.cuda.mem_get_info(dev)[0]
+    if need > 0.95 * free:
+        raise SystemExit("chunked workload needs %.1f GB on the device, %.1f GB free"
+                         % (need / 1e9, free / 1e9))
+    outs = [torch.empty(1, C, wl.Hq, wl.d_v, dtype=torch.bfloat16, device=dev) for _ in range(nl)]
+    idx_buf = torch.empty(1, C, wl.k, dtype=torch.int32, device=dev)
+    shapes, rows = [], []
+    for c in range(nch):
+        r = ic.Rows(1, C, c * C, (c + 1) * C)
+        rows.append(r)
+        shapes.append(ic.StackShape(r, wl.H_I, wl.d_I, DT[wl.idx_dtype], wl.k, wl.Hq, wl.d_qk,
+                                    wl.d_v, DT[wl.attn_dtype], wl.d_qk, wl.d_qk, wl.scale))
+    ws = torch.empty(ic.workspace_size(shapes[-1]), dtype=torch.uint8, device=dev)
+    ic.workspace_init(ws)
+    ld = (wl.T + 3) // 4 * 4
+    scores = torch.empty(1, C, ld, dtype=torch.float32, device=dev)
+    t_start = time.time()
+
+    def progress(msg):
+        print("[chunked %6.1f s] %s" % (time.time() - t_start, msg), file=sys.stderr, flush=True)
+
+    keys, qs, qI, wI = [], [], {}, {}
+    for l in range(nl):
+        inp = synth.layer_inputs(wl, l, dev, chunk=0)
+        keys.append((inp["k_I"], inp["kv"]))
+        ql = [inp["q"]]
+        if l == 0 or not shared_q:
+            qI[(l, 0)], wI[(l, 0)] = inp["q_I"], inp["w"]
+        if l == 0:
+            # load every kernel of the stack (and its code on the device) before
+            # the bulk of the inputs fills the memory
+            ic.layer_stack_forward("F", [dict(q_idx=inp["q_I"], w=inp["w"], k_idx=inp["k_I"],
+                                              q=inp["q"], kmat=inp["kv"], vmat=inp["kv"],
+                                              out=outs[0])], shapes[0], idx_buf, ws)
+            torch.cuda.synchronize()
+        del inp
+        for c in range(1, nch):
+            d = synth.chunk_queries(wl, l, c, dev, indexer=(l == 0 or not shared_q))
+            ql.append(d["q"])
+            if "q_I" in d:
+                qI[(l, c)], wI[(l, c)] = d["q_I"], d["w"]
+            del d
+        qs.append(ql)
+        torch.cuda.empty_cache()   # float32 temporaries of the generator
+    qkey = (lambda l, c: (0, c)) if shared_q else (lambda l, c: (l, c))
+    progress("inputs resident (%.1f GB)" % (need / 1e9))
+
+    def layer_dicts(pat, c):
+        res = []
+        for l, kind in enumerate(pat):
+            kI, kv = keys[l]
+            d = dict(q=qs[l][c], kmat=kv, vmat=kv, out=outs[l])
+            if kind == "F":
+                d.update(q_idx=qI[qkey(l, c)], w=wI[qkey(l, c)], k_idx=kI)
+            res.append(d)
+        return res
+
+    calls = {p: [layer_dicts(p, c) for c in range(nch)] for p in (pattern, all_f)}
+
+    def step(pat):
+        for c in range(nch):
+            ic.layer_stack_forward(pat, calls[pat][c], shapes[c], idx_buf, ws)
+
+    def timed(fn, steps):
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b), pg, dev)
+
+    for _ in range(max(3, args.warmup)):
+        step(pattern)
+        step(all_f)
+    progress("warm-up done")
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    n0 = ic.kernel_launches(0)
+    ms = timed(lambda: step(pattern), args.steps)
+    launches = ic.kernel_launches(0) - n0
+    ms_all_f = timed(lambda: step(all_f), args.steps)
+    clk = clocks.stop()
+
+    # stage breakdown: the same kernels as separate calls, events around each
+    ev = Events()
+    for c in range(nch):
+        r = rows[c]
+        for l, kind in enumerate(pattern):
+            kI, kv = keys[l]
+            if kind == "F":
+                e0, e1, e2 = ev.new(), ev.new(), ev.new()
+                e0.record()
+                ic.indexer_scores(qI[qkey(l, c)], wI[qkey(l, c)], kI, r, scores, ws,
+                                  dtype=DT[wl.idx_dtype])
+                e1.record()
+                ic.topk(scores, r, wl.k, idx_buf, ws)
+                e2.record()
+                ev.add("indexer", e0, e1)
+                ev.add("topk", e1, e2)
+            e3, e4 = ev.new(), ev.new()
+            e3.record()
+            ic.sparse_attn(qs[l][c], kv, wl.d_qk, kv, wl.d_qk, idx_buf, r, wl.d_v, wl.scale,
+                           outs[l], ws, dtype=DT[wl.attn_dtype])
+            e4.record()
+            ev.add("attention", e3, e4)
+    stages = ev.collect()
+    progress("timed steps and stage pass done")
+
+    # algorithmic work of one layer pass over all chunks
+    work = {}
+    for c in range(nch):
+        sub = dataclasses.replace(wl, L=C, q_start=c * C, T=(c + 1) * C, chunk=0)
+        for k, v in algorithmic(sub).items():
+            work[k] = work.get(k, 0.0) + v
+    roof, dom = roofline(wl, work, {k: sum(v) for k, v in stages.items()},
+                         {k: len(v) for k, v in stages.items()}, per_pass=nch)
+    roof["traffic"] = _traffic(dom, args.workload)
+
+    # untimed: top-k overlap of each S layer's own selection with the reused one
+    own = torch.empty_like(idx_buf)
+    acc = {}
+    for c in range(nch):
+        r = rows[c]
+        t_row = torch.arange(c * C, (c + 1) * C, device=dev)
+        m = torch.clamp(t_row + 1, max=wl.k).to(torch.float64)
+        off = (torch.arange(C, device=dev, dtype=torch.int64) * (wl.T + 1))[:, None]
+        for l, kind in enumerate(pattern):
+            kI = keys[l][0]
+            ic.indexer_scores(qI[qkey(l, c)], wI[qkey(l, c)], kI, r, scores, ws,
+                              dtype=DT[wl.idx_dtype])
+            ic.topk(scores, r, wl.k, own if kind == "S" else idx_buf, ws)
+            if kind == "F":
+                continue
+            a = idx_buf[0].to(torch.int64)
+            b = own[0].to(torch.int64)
+            a = torch.where(a >= 0, a + off, torch.full_like(a, -1))
+            b = torch.where(b >= 0, b + off, torch.full_like(b, -2))
+            hit = torch.isin(b.flatten(), a.flatten()).view(C, wl.k).sum(1).to(torch.float64)
+            frac = hit / m
+            s_, n_, mn = acc.get(l, (0.0, 0, 1.0))
+            acc[l] = (s_ + float(frac.sum()), n_ + C, min(mn, float(frac.min())))
+    overlap = {"layer_%d" % l: {"mean": v[0] / v[1], "min": v[2]} for l, v in sorted(acc.items())}
+    torch.cuda.synchronize()
+    progress("overlap pass done")
+
+    if rank != 0:
+        _finish(pg)
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rps, done, spent = oracle_sample(wl, pattern, args.cpu_budget)
+        cpu = {"value": rps, "unit": "tok/s", "cores": _blas_threads(), "kind": "oracle",
+               "sample": "%d query rows of %s at random positions through all %d layers of %s "
+                         "(float64 NumPy, %.1f s)" % (done, wl.name, nl, pattern, spent)}
+    per_step_ms = ms / args.steps
+    avg = {k: float(np.mean(v)) for k, v in stages.items()}
+    line = {
+        "metric": "chunked prefill tok/s (IndexCache pattern) with all-F comparison; roofline of "
+                  "the dominant kernel; top-k overlap of S layers",
+        "value": wl.B * wl.L * world / (per_step_ms / 1e3), "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": per_step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.attn_dtype,
+        "data": "synthetic",
+        "config": {"workload": wl.name, "pattern": pattern, "B": wl.B, "L": wl.L, "chunk": C,
+                   "T": wl.T, "H_I": wl.H_I, "d_I": wl.d_I, "k": wl.k, "Hq": wl.Hq,
+                   "d_qk": wl.d_qk, "d_v": wl.d_v, "indexer_dtype": wl.idx_dtype,
+                   "k_I_per_layer": "base + %.1f x noise at the base's scale" % wl.kI_noise,
+                   "parallelism": "replicas x%d" % world,
+                   "l2": "inputs larger than L2 (%.1f GB resident)" % (need / 1e9)},
+        "all_f": {"pattern": all_f, "ms_per_step": ms_all_f / args.steps,
+                  "value": wl.B * wl.L * world / (ms_all_f / args.steps / 1e3),
+                  "speedup_of_pattern": ms_all_f / ms},
+        "stages_ms": {k: {"per_launch": avg[k], "launches_per_step": len(v)}
+                      for k, v in stages.items()},
+        "topk_overlap_s_layers": overlap,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": None,
+        "e2e_note": "not measured for this workload: one step reads %.0f GB of query inputs"
+                    % (need / 1e9),
+        "gpu_launches": launches,
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)
@@ -515,11 +762,7 @@ def run_e2e(st, pattern, steps, dev, pg):
         step()
     b.record()
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(a.elapsed_time(b), pg, dev)
     world = pg.get_world_size() if pg else 1
     wl = st.wl
     del host

@@ -26,6 +26,7 @@ __all__ = [
 
 F32, BF16, FP8_E4M3 = 0, 1, 2
 STATUS_BYTES = 256
+CUDA_ERROR = -5
 _STATUS = {0: "IC_OK", -1: "IC_ERR_INVALID_ARG", -2: "IC_ERR_PATTERN", -3: "IC_ERR_UNSUPPORTED",
            -4: "IC_ERR_WORKSPACE", -5: "IC_ERR_CUDA", -6: "IC_ERR_INDEX_RANGE",
            -7: "IC_ERR_TIMEOUT"}
@@ -38,9 +39,10 @@ def library_path() -> str:
 
 
 class IcError(RuntimeError):
-    def __init__(self, code: int, where: str):
+    def __init__(self, code: int, where: str, detail: str = ""):
         self.code = code
-        super().__init__("%s failed: %s (%d)" % (where, _STATUS.get(code, "?"), code))
+        super().__init__("%s failed: %s (%d)%s" % (where, _STATUS.get(code, "?"), code,
+                                                   " [%s]" % detail if detail else ""))
 
 
 class Rows(ctypes.Structure):
@@ -64,6 +66,7 @@ class LayerIO(ctypes.Structure):
 _P = ctypes.c_void_p
 _SIG = {
     "ic_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "ic_last_error": (ctypes.c_char_p, []),
     "ic_version": (ctypes.c_int, []),
     "ic_kernel_launches": (ctypes.c_uint64, [ctypes.c_int]),
     "ic_workspace_init": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
@@ -133,7 +136,8 @@ def _nbytes(x) -> int:
 
 def _check(code: int, where: str) -> None:
     if code != 0:
-        raise IcError(code, where)
+        detail = lib().ic_last_error().decode() if code == CUDA_ERROR else ""
+        raise IcError(code, where, detail)
 
 
 def _rows(rows) -> Rows:

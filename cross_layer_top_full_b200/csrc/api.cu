@@ -8,6 +8,7 @@
 // "Architettura e Funzionamento").
 #include <algorithm>
 #include <atomic>
+#include <cstdio>
 #include <cstring>
 
 #include "common.cuh"
@@ -23,8 +24,24 @@ void count_launch(int kind) {
     if (kind > 0 && kind < IC_LK_KINDS) g_launches[kind].fetch_add(1, std::memory_order_relaxed);
 }
 
+namespace {
+thread_local char tl_error[256] = "";
+}
+
+const char* tl_error_text() { return tl_error; }
+
+ic_status cuda_error(const char* where) {
+    const cudaError_t e = cudaGetLastError();
+    snprintf(tl_error, sizeof(tl_error), "%s: %s", where,
+             e == cudaSuccess ? "CUDA driver call failed" : cudaGetErrorString(e));
+    return cuda_error("api");
+}
+
 ic_status last_launch_status() {
-    return cudaGetLastError() == cudaSuccess ? IC_OK : IC_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) return IC_OK;
+    snprintf(tl_error, sizeof(tl_error), "kernel launch: %s", cudaGetErrorString(e));
+    return cuda_error("api");
 }
 
 namespace {
@@ -103,6 +120,8 @@ using namespace ic;
 
 extern "C" {
 
+const char* ic_last_error(void) { return ic::tl_error_text(); }
+
 const char* ic_status_string(ic_status st) {
     switch (st) {
         case IC_OK: return "IC_OK";
@@ -127,7 +146,7 @@ uint64_t ic_kernel_launches(int kind) {
 ic_status ic_workspace_init(void* ws, size_t ws_bytes, void* stream) {
     if (!ws_ok(ws, ws_bytes, IC_STATUS_BYTES)) return IC_ERR_WORKSPACE;
     if (cudaMemsetAsync(ws, 0, IC_STATUS_BYTES, (cudaStream_t)stream) != cudaSuccess)
-        return IC_ERR_CUDA;
+        return cuda_error("api");
     return IC_OK;
 }
 
@@ -136,11 +155,11 @@ ic_status ic_read_status(void* ws, void* stream, int32_t* device_status) {
     cudaStream_t s = (cudaStream_t)stream;
     uint32_t v = 0;
     if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        return IC_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return IC_ERR_CUDA;
+        return cuda_error("api");
+    if (cudaStreamSynchronize(s) != cudaSuccess) return cuda_error("api");
     if (v != 0) {
-        if (cudaMemsetAsync(ws, 0, sizeof(v), s) != cudaSuccess) return IC_ERR_CUDA;
-        if (cudaStreamSynchronize(s) != cudaSuccess) return IC_ERR_CUDA;
+        if (cudaMemsetAsync(ws, 0, sizeof(v), s) != cudaSuccess) return cuda_error("api");
+        if (cudaStreamSynchronize(s) != cudaSuccess) return cuda_error("api");
     }
     *device_status = (int32_t)v;
     if (v & IC_DEV_INDEX_RANGE) return IC_ERR_INDEX_RANGE;
@@ -264,7 +283,7 @@ ic_status ic_layer_stack_forward(const char* pattern, int n_layers, const ic_lay
         if (idx_out != nullptr && idx_out[l] != nullptr) {
             if (cudaMemcpyAsync(idx_out[l], idx_buf, idx_bytes, cudaMemcpyDeviceToDevice, s) !=
                 cudaSuccess)
-                return IC_ERR_CUDA;
+                return cuda_error("api");
         }
     }
     return IC_OK;

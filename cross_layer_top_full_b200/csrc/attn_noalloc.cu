@@ -62,16 +62,16 @@ extern "C" ic_status ic_sparse_attn_noalloc(const void* q, const void* kv, const
     const size_t need = attn_tc_scratch_bytes(r, k);
     if (need > IC_NOALLOC_SCRATCH_BYTES - kStatusBytes) return IC_ERR_WORKSPACE;
     char* base = static_cast<char*>(scratch_address());
-    if (base == nullptr) return IC_ERR_CUDA;
+    if (base == nullptr) return cuda_error("attn_noalloc");
     cudaStream_t s = (cudaStream_t)stream;
     uint32_t* status = reinterpret_cast<uint32_t*>(base);
-    if (cudaMemsetAsync(status, 0, sizeof(uint32_t), s) != cudaSuccess) return IC_ERR_CUDA;
+    if (cudaMemsetAsync(status, 0, sizeof(uint32_t), s) != cudaSuccess) return cuda_error("attn_noalloc");
     ic_status st = launch_attn_tc(q, kv, 576, idx, k, r, scale, out, status, base + kStatusBytes,
                                   IC_NOALLOC_SCRATCH_BYTES - kStatusBytes, s);
     if (st != IC_OK) return st;
     if (device_status != nullptr &&
         cudaMemcpyAsync(device_status, status, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) !=
             cudaSuccess)
-        return IC_ERR_CUDA;
+        return cuda_error("attn_noalloc");
     return IC_OK;
 }

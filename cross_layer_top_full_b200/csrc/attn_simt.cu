@@ -128,7 +128,7 @@ ic_status launch_typed(const void* q, const void* kmat, int64_t ks, const void* 
     if (smem > 48 * 1024) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
-            return IC_ERR_CUDA;
+            return cuda_error("attn_simt");
     }
     dim3 grid((unsigned)((int64_t)r.B * r.Lq), ceil_div(Hq, HEADS_PER_CTA));
     kern<<<grid, 32 * HEADS_PER_CTA, smem, s>>>(

@@ -852,7 +852,7 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
     if (((uintptr_t)q & 15) || ((uintptr_t)kv & 15) || ((uintptr_t)out & 15))
         return IC_ERR_INVALID_ARG;
     auto fn = encode_fn();
-    if (fn == nullptr) return IC_ERR_CUDA;
+    if (fn == nullptr) return cuda_error("attn_tc");
     CUtensorMap map_q, map_qr;
     cuuint64_t dims[2] = {(cuuint64_t)KVW, (cuuint64_t)r.B * r.Lq * HQ};
     cuuint64_t strides[1] = {(cuuint64_t)KVW * 2};
@@ -862,11 +862,11 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
     if (fn(&map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box,
            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return IC_ERR_CUDA;
+        return cuda_error("attn_tc");
     if (fn(&map_qr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box_r,
            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return IC_ERR_CUDA;
+        return cuda_error("attn_tc");
 
     // KV rows for the gathers: one box row of 64 value columns (128-byte
     // swizzle) or of the 32 rope columns (64-byte swizzle)
@@ -878,11 +878,11 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
     if (fn(&map_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv), kdims, strides, kbox,
            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return IC_ERR_CUDA;
+        return cuda_error("attn_tc");
     if (fn(&map_kvr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv), kdims, strides, kbox_r,
            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return IC_ERR_CUDA;
+        return cuda_error("attn_tc");
 
     AttnArgs a;
     a.kv = static_cast<const __nv_bfloat16*>(kv);
@@ -910,7 +910,7 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
     }
     if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES) != cudaSuccess)
-        return IC_ERR_CUDA;
+        return cuda_error("attn_tc");
     const int64_t pairs = std::min<int64_t>(units, std::max(1, sm_count() / 2));
     attn_tc_kernel<<<(unsigned)(2 * pairs), N_THREADS, SMEM_BYTES, s>>>(map_q, map_qr, map_kv, map_kvr, a);
     count_launch(IC_LK_ATTN_TC);

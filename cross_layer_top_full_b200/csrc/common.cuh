@@ -25,6 +25,10 @@ void count_launch(int kind);
 
 // Host: map the last CUDA error to a status.
 ic_status last_launch_status();
+// Records the pending CUDA runtime error (or, for a failed driver call, the
+// site alone) as this thread's last error text and returns IC_ERR_CUDA.
+ic_status cuda_error(const char* where);
+const char* tl_error_text();
 
 __device__ __forceinline__ void flag_status(uint32_t* status, uint32_t bit) {
     if (status) atomicOr(status, bit);

@@ -71,7 +71,7 @@ ic_status launch_typed(const void* q_idx, const float* q_scale, const float* w, 
     if (smem > 48 * 1024) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
-            return IC_ERR_CUDA;
+            return cuda_error("indexer_simt");
     }
     const int last_t = r.q_start + r.Lq - 1;
     if (ceil_div(last_t + 1, KT) > 65535) return IC_ERR_UNSUPPORTED;

@@ -371,8 +371,8 @@ ic_status launch_cfg(const void* q_idx, const float* q_scale, const float* w, co
                      cudaStream_t s) {
     using C = Cfg<H, NTOK, FP8>;
     CUtensorMap map_k, map_q;
-    if (!make_map(&map_k, k_idx, (int64_t)r.B * r.T, FP8, BM)) return IC_ERR_CUDA;
-    if (!make_map(&map_q, q_idx, (int64_t)r.B * r.Lq * H, FP8, C::N)) return IC_ERR_CUDA;
+    if (!make_map(&map_k, k_idx, (int64_t)r.B * r.T, FP8, BM)) return cuda_error("indexer_tc");
+    if (!make_map(&map_q, q_idx, (int64_t)r.B * r.Lq * H, FP8, C::N)) return cuda_error("indexer_tc");
     Work wk;
     wk.n_groups = ceil_div(r.Lq, NTOK);
     const int max_tiles = ceil_div(r.q_start + r.Lq, BM);
@@ -390,7 +390,7 @@ ic_status launch_cfg(const void* q_idx, const float* q_scale, const float* w, co
     auto kern = indexer_tc_kernel<H, NTOK, FP8>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
-        return IC_ERR_CUDA;
+        return cuda_error("indexer_tc");
     const int grid = (int)std::min<int64_t>(items, sms);
     kern<<<grid, N_THREADS, smem, s>>>(map_k, map_q, w, q_scale, k_scale, scores, ld, r.B, r.Lq,
                                        r.q_start, r.T, wk, status);

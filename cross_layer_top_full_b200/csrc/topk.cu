@@ -46,10 +46,12 @@ ic_status launch_topk_rows(const float* scores, int64_t ld, ic_rows r, int k, in
     const int n_max = r.q_start + r.Lq;  // candidates of the last row
     const int cache = n_max <= SMEM_KEYS_MAX ? n_max : 0;
     const size_t smem = (size_t)cache * sizeof(uint32_t);
-    if (smem > 48 * 1024) {
+    // the default dynamic limit leaves room for the static SelectState: opt in
+    // whenever static + dynamic could pass 48 KB
+    if (smem + sizeof(SelectState<NT / 32>) > 48 * 1024) {
         if (cudaFuncSetAttribute(topk_radix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
-            return IC_ERR_CUDA;
+            return cuda_error("topk");
     }
     const int64_t rows = (int64_t)r.B * r.Lq;
     topk_radix_kernel<<<(unsigned)rows, NT, smem, s>>>(scores, ld, r.Lq, r.q_start, k, idx, cache);

@@ -479,13 +479,13 @@ ic_status launch_topk_multi(const float* scores, int64_t ld, ic_rows r, int k, i
     MultiWs ws = carve(scratch, rows, nch);
     // per-call state that must start at zero: row histograms and control words
     if (cudaMemsetAsync(ws.hist, 0, sizeof(uint32_t) * rows * (HBINS + RW_WORDS), s) != cudaSuccess)
-        return IC_ERR_CUDA;
+        return cuda_error("topk_multi");
     const size_t smem2 = sizeof(uint32_t) * std::max<size_t>(2 * CAPG + (size_t)nch, 2 * CAPS);
     if (cudaFuncSetAttribute(topk_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem2) != cudaSuccess ||
         cudaFuncSetAttribute(topk_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(sizeof(uint32_t) * NW * HBINS)) != cudaSuccess)
-        return IC_ERR_CUDA;
+        return cuda_error("topk_multi");
     dim3 grid(nch, (unsigned)rows);
     topk_hist_kernel<<<grid, NT, sizeof(uint32_t) * NW * HBINS, s>>>(scores, ld, r.Lq, r.q_start, k, ws);
     count_launch(IC_LK_TOPK);

@@ -218,6 +218,32 @@ def layer_inputs(wl: Workload, layer: int, device="cpu", *, indexer: bool = True
     return out
 
 
+def chunk_queries(wl: Workload, layer: int, chunk: int, device="cpu", *,
+                  indexer: bool = True) -> Dict[str, torch.Tensor]:
+    """Query-side inputs of one chunk of a chunked workload, drawn exactly as
+    ``layer_inputs(wl, layer, device, chunk=chunk)`` draws them: 'q'
+    [B,chunk,Hq,d_qk] and, with ``indexer``, 'q_I' [B,chunk,H_I,d_I] and 'w'
+    [B,chunk,H_I] (+ 'q_scale' for e4m3).  Keys are not drawn."""
+    assert wl.chunk, "chunked workload expected"
+    B, qrows = wl.B, wl.chunk
+    out: Dict[str, torch.Tensor] = {}
+    if indexer:
+        if wl.kI_noise:
+            qkey, wkey = ("qI_shared", chunk), ("w_shared", chunk)
+        else:
+            qkey, wkey = ("qI", layer, chunk), ("w", layer, chunk)
+        qI = _randn((B, qrows, wl.H_I, wl.d_I), wl.qI_std, device, wl.seed, *qkey)
+        out["w"] = _randn((B, qrows, wl.H_I), wl.w_std, device, wl.seed, *wkey)
+        if wl.idx_dtype == "e4m3":
+            out["q_I"], out["q_scale"] = fp8_per_token(qI, 2)
+        else:
+            out["q_I"] = qI.to(_store_dtype(wl.idx_dtype)).contiguous()
+        del qI
+    out["q"] = _randn((B, qrows, wl.Hq, wl.d_qk), wl.q_std, device, wl.seed, "q", layer, chunk,
+                      dtype=_store_dtype(wl.attn_dtype))
+    return out
+
+
 def exact_indexer_inputs(B: int, Lq: int, T: int, H_I: int, d_I: int, dtype: str, device="cpu",
                          seed: int = 0) -> Dict[str, torch.Tensor]:
     """Indexer inputs whose scores are exact in float32 for any summation order.

@@ -78,6 +78,12 @@ typedef struct {
 /* Human-readable name of a status code (static string, never NULL). */
 const char* ic_status_string(ic_status st);
 
+/* Text of the last CUDA failure seen by a call of this library on the
+ * calling thread ("<source>: <CUDA error string>"), behind the most recent
+ * IC_ERR_CUDA; "" if none.  Per-thread static storage, valid until the next
+ * failing call on the same thread; never NULL. */
+const char* ic_last_error(void);
+
 /* Library version, major*10000 + minor*100 + patch. */
 int ic_version(void);
 
