@@ -67,6 +67,7 @@ _P = ctypes.c_void_p
 _SIG = {
     "ic_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ic_last_error": (ctypes.c_char_p, []),
+    "ic_selftest_wait_timeout": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "ic_version": (ctypes.c_int, []),
     "ic_kernel_launches": (ctypes.c_uint64, [ctypes.c_int]),
     "ic_workspace_init": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
@@ -177,6 +178,13 @@ def read_status(ws, stream=None) -> int:
     if code not in (0, -6, -7):
         raise IcError(code, "ic_read_status")
     return int(v.value)
+
+
+def selftest_wait_timeout(ws, stream=None) -> None:
+    """Launch the failure-path self-test (a pipeline wait that never
+    completes and gives up after about 1 s); read the result with read_status."""
+    _check(lib().ic_selftest_wait_timeout(_ptr(ws), _nbytes(ws), _stream(stream)),
+           "ic_selftest_wait_timeout")
 
 
 def indexer_workspace_size(rows, H_I: int, d_I: int, dtype: int) -> int:

@@ -16,6 +16,12 @@
 #ifndef IC_WAIT_LIMIT_NS
 #define IC_WAIT_LIMIT_NS 1000000000ull  // 1 s
 #endif
+// Suspend-time hint of the waiting try_wait: a waiting warp sleeps until the
+// phase completes (or this many ns pass) instead of re-issuing the poll, so
+// it leaves the issue slots to the warps doing work.  0 = no hint.
+#ifndef IC_WAIT_SUSPEND_NS
+#define IC_WAIT_SUSPEND_NS 20000u
+#endif
 
 namespace ic {
 namespace sm100 {
@@ -73,6 +79,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with the suspend-time hint (blocks until the phase completes or
+// the hint's time passes)
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+#if IC_WAIT_SUSPEND_NS
+    uint32_t ok = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(IC_WAIT_SUSPEND_NS)
+        : "memory");
+    return ok != 0;
+#else
+    return mbar_try_wait(bar, parity);
+#endif
+}
+
 // Wait until the phase with the given parity of `bar` has completed.
 // Returns false (and flags IC_DEV_TIMEOUT, raises *abort) on timeout, or
 // returns false at once if *abort is already raised.
@@ -81,7 +105,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t n = 0;; ++n) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity)) return true;
         if ((n & 63u) == 63u) {
             if (*abort) return false;
             if (globaltimer() - t0 > IC_WAIT_LIMIT_NS) {
@@ -321,13 +345,29 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
     return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_try_wait_cluster_sleep(uint64_t* bar, uint32_t parity) {
+#if IC_WAIT_SUSPEND_NS
+    uint32_t ok = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(IC_WAIT_SUSPEND_NS)
+        : "memory");
+    return ok != 0;
+#else
+    return mbar_try_wait_cluster(bar, parity);
+#endif
+}
+
 // Bounded wait with cluster-scope acquire (for barriers other CTAs arrive on).
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* status,
                                                   volatile int* abort) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t n = 0;; ++n) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (mbar_try_wait_cluster_sleep(bar, parity)) return true;
         if ((n & 63u) == 63u) {
             if (*abort) return false;
             if (globaltimer() - t0 > IC_WAIT_LIMIT_NS) {

@@ -96,6 +96,13 @@ ic_status ic_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * it.  Returns IC_OK when no bit was set, else the error of the lowest bit. */
 ic_status ic_read_status(void* ws, void* stream, int32_t* device_status);
 
+/* Failure-path self-test: launches one CTA whose pipeline wait (the
+ * library's bounded mbarrier wait) never completes.  After about 1 s the
+ * wait gives up, bit 1 (wait timeout) of the status word of `ws` is set and
+ * the kernel returns normally; read it with ic_read_status.  Faults and
+ * hangs nothing; the context stays usable.  ws_bytes >= IC_STATUS_BYTES. */
+ic_status ic_selftest_wait_timeout(void* ws, size_t ws_bytes, void* stream);
+
 /* Number of kernels this library has launched in this process, by kind:
  * 0 = all, 1 = indexer, 2 = top-k, 3 = attention, 4 = split-k combine,
  * 5 = indexer launches that took the tensor-core path, 6 = attention

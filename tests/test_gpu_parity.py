@@ -320,3 +320,20 @@ def test_degenerate_rows(dev):
     outs, idx_copies, _ = _run_stack(wl, "F", inputs, dev, rows=rows)
     assert host64(idx_copies[0])[0, 0].tolist() == [0] + [-1] * (wl.k - 1)
     assert np.allclose(host64(outs[0])[0, 0], host64(inputs[0]["v"])[0, 0][None, :], atol=1e-6)
+
+
+# ------------------------------------------------------------------------- failure path
+def test_stalled_wait_ends_with_timeout_status_and_usable_context(dev):
+    """A pipeline wait that nothing completes gives up after its bounded time:
+    the status word reports the timeout bit (2), the kernel returns, and the
+    context keeps working (a top-k afterwards is still bit-exact)."""
+    ws = _ws(1 << 16, dev)
+    ic.selftest_wait_timeout(ws)
+    torch.cuda.synchronize()
+    assert ic.read_status(ws) == 2
+    rows, k = (1, 8, 100, 108), 16
+    scores = synth.random_scores(1, 8, 108, dev, seed=5)
+    idx = torch.full((1, 8, k), -7, dtype=torch.int32, device=dev)
+    ic.topk(scores, rows, k, idx, _ws(ic.topk_workspace_size(rows, k), dev))
+    torch.cuda.synchronize()
+    assert np.array_equal(host64(idx), oracle.topk_indices(host64(scores), 100, k))
