@@ -1,0 +1,82 @@
+"""Algorithmic work counts behind the bench's roofline lines (CPU).
+
+Each count is re-derived here from the workload's shape in closed form
+(sums of arithmetic series), independently of bench.algorithmic's loops:
+  causal pairs of L rows starting at q_start: sum_{t=q0}^{q0+L-1} (t+1);
+  selected-row visits: sum_t min(k, t+1);
+  indexer flop = 2*H_I*d_I per pair, attention flop = 2*Hq*(d_qk+d_v) per visit.
+"""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from cross_layer_top_full_b200 import synth  # noqa: E402
+
+
+def _pairs(q0, L):
+    a, b = q0 + 1, q0 + L            # sum of (t+1) for t = q0 .. q0+L-1
+    return (a + b) * L // 2
+
+
+def _visits(q0, L, k):
+    lo, hi = q0, q0 + L - 1          # t range; min(k, t+1) = t+1 for t < k
+    n_small = max(0, min(hi, k - 1) - lo + 1)
+    small = _pairs(lo, n_small) if n_small else 0
+    return small + k * (L - n_small)
+
+
+@pytest.mark.parametrize("name", ["prefill_512_fp32", "prefill_8k_bf16", "decode_b32_t32k_bf16",
+                                  "decode_b8_t200k_fp8"])
+def test_counts_match_closed_forms(name):
+    wl = synth.WORKLOADS[name]
+    w = bench.algorithmic(wl)
+    pairs = wl.B * _pairs(wl.q_start, wl.L)
+    visits = wl.B * _visits(wl.q_start, wl.L, wl.k)
+    assert w["pairs"] == pairs
+    assert w["visits"] == visits
+    assert w["indexer_flop"] == pytest.approx(2 * wl.H_I * wl.d_I * pairs)
+    assert w["attn_flop"] == pytest.approx(2 * wl.Hq * (wl.d_qk + wl.d_v) * visits)
+
+
+def test_prefill_8k_figures():
+    """L = 8192 from position 0, H_I = 64, d_I = 128, k = 2048, 128 heads, 576/512."""
+    w = bench.algorithmic(synth.WORKLOADS["prefill_8k_bf16"])
+    assert w["pairs"] == 8192 * 8193 // 2                       # 33.56 M causal pairs
+    assert w["indexer_flop"] == pytest.approx(0.5498e12, rel=1e-3)
+    # rows t < 2047 see t+1 keys, the other 6145 rows see 2048
+    assert w["visits"] == 2048 * 2049 // 2 + 2048 * (8192 - 2048)
+    assert w["attn_flop"] == pytest.approx(4.088e12, rel=1e-3)
+
+
+def test_decode_bytes():
+    """Decode: the indexer reads every cached key once; attention gathers k rows."""
+    c2 = bench.algorithmic(synth.WORKLOADS["decode_b32_t32k_bf16"])
+    assert c2["pairs"] == 32 * 32768
+    kI = 32 * 32768 * 128 * 2
+    assert c2["indexer_bytes"] == pytest.approx(kI + 32 * 64 * (128 * 2 + 4) + 4 * 32 * 32768)
+    kv = 32 * 2048 * 576 * 2
+    assert c2["attn_bytes"] == pytest.approx(kv + 32 * 128 * (576 + 512) * 2 + 4 * 32 * 2048)
+    c4 = bench.algorithmic(synth.WORKLOADS["decode_b8_t200k_fp8"])
+    assert c4["indexer_bytes"] == pytest.approx(8 * 200000 * 128 + 8 * 64 * (128 + 4)
+                                                + 4 * 8 * 200000)
+    assert c4["attn_bytes"] == pytest.approx(8 * 2048 * 1152 + 8 * 128 * 1088 * 2 + 4 * 8 * 2048)
+
+
+def test_roofline_line_uses_the_dominant_stage():
+    wl = synth.WORKLOADS["prefill_8k_bf16"]
+    work = bench.algorithmic(wl)
+    roof, dom = bench.roofline(wl, work, {"indexer": 0.5, "topk": 0.5, "attention": 40.0},
+                               {"indexer": 1, "topk": 1, "attention": 4})
+    assert dom == "attention" and roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s"
+    assert roof["achieved"] == pytest.approx(work["attn_flop"] / 10e-3 / 1e12)
+    assert roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"])
+    wl = synth.WORKLOADS["decode_b32_t32k_bf16"]
+    roof, dom = bench.roofline(wl, bench.algorithmic(wl), {"indexer": 0.2, "topk": 0.1,
+                                                           "attention": 0.6},
+                               {"indexer": 2, "topk": 2, "attention": 8})
+    assert dom == "attention" and roof["bound"] == "hbm" and roof["unit"] == "GB/s"
