@@ -20,36 +20,41 @@
 // own 256 value columns, O_r += P V_r, in TMEM.  No key byte is gathered
 // twice and no flop is done twice.
 //
-// Per CTA (352 threads), persistent over work units (one unit = one query
+// Per CTA (448 threads), persistent over work units (one unit = one query
 // row, or one split of a row's indices in decode):
-//   warps 0-1  gather: per unit, one pass over the unit's indices computes
-//              the per-block validity masks and the block count; then TMA
-//              four-row gathers (tile::gather4) of the selected rows' columns
-//              into 128-byte-swizzled tiles (3 stages of 64 keys); an
-//              invalid index becomes an out-of-range row, which TMA fills
-//              with zeros;
-//   warps 2-5  exchange (thread = head = TMEM lane): partial S of a 64-key
-//              block from TMEM -> base-2 float16, sent straight into the
-//              partner's inbox with st.async (counted in bytes on the
-//              partner's mbarrier) and stored back into TMEM for the
-//              softmax warps; they run ahead of the softmax warps, so the
-//              exchange latency of block j+1 hides behind the softmax of j;
-//   warps 6-9  softmax (thread = head): own + partner logits, row max,
+//   warps 0-3  gather: per unit, one batched pass over the unit's indices
+//              computes the per-block validity masks and the block count;
+//              then TMA four-row gathers (tile::gather4) of the selected
+//              rows' columns into 128-byte-swizzled tiles (4 stages of 64
+//              keys); an invalid index becomes an out-of-range row, which
+//              TMA fills with zeros;
+//   warps 4-7  exchange (thread = head = TMEM lane): at the start of a unit,
+//              the unit's Q_r columns that the S MMA reads from TMEM (value
+//              slice 3 and the 32 rope columns); per 64-key block, partial S
+//              from TMEM -> base-2 float16, sent straight into the partner's
+//              inbox with st.async (counted in bytes on the partner's
+//              mbarrier) and stored back into TMEM for the softmax warps;
+//              they run ahead of the softmax warps, so the exchange latency
+//              of block j+1 hides behind the softmax of block j;
+//   warps 8-11 softmax (thread = head): own + partner logits, row max,
 //              online softmax in base 2 with lazy rescaling (O is rescaled
 //              only when the running max grows by more than 2^8), P as bf16
-//              into TMEM over the S columns, final normalisation and store;
-//   warp 10    TMEM allocation, TMA load of Q_r (the next unit's Q is loaded
-//              while the current unit finishes), and single-thread issue of
-//              S(j) = Q_r K_r(j)^T (K = 288) as soon as block j is gathered;
-//   warp 11    single-thread issue of O += P(j) V_r(j) and l += P(j) 1 (the
-//              row sums, on the tensor core against a ones operand), P read
-//              from TMEM ("TS" form), as soon as P(j) is ready.  Two issuing
-//              threads keep a P V from waiting behind the gather of a later
-//              block.
-// TMEM: O at columns 0..255, three S/P buffers at 256..447, l at 448..463.
-// Shared memory: Q_r 72 KB, 3 KV stages of 36 KB, 2 float16 inbox tiles of
-// 16 KB (written by the partner), a 2 KB ones operand, per-unit masks,
-// barriers (~221 KB).
+//              into TMEM over the S columns, the row sum l of the same
+//              rounded P, final normalisation and store;
+//   warp 12    TMEM allocation, TMA load of Q_r's value slices 0-2 (the next
+//              unit's while the current unit finishes), and single-thread
+//              issue of S(j) = Q_r K_r(j)^T (K = 288; A from shared memory for
+//              slices 0-2, from TMEM for slice 3 and the rope columns) as
+//              soon as block j is gathered;
+//   warp 13    single-thread issue of O += P(j) V_r(j), P read from TMEM
+//              ("TS" form), as soon as P(j) is ready.  Two issuing threads
+//              keep a P V from waiting behind the gather of a later block.
+// TMEM: O at columns 0..255, three S/P buffers at 256..447, Q_r slice 3 and
+// rope columns at 448..495.  Keeping that part of Q_r in TMEM frees the
+// shared memory for a fourth KV stage.
+// Shared memory: Q_r slices 0-2 48 KB, 4 KV stages of 36 KB, 2 float16 inbox
+// tiles of 16 KB (written by the partner), per-unit masks, barriers
+// (~226 KB).
 //
 // Decode (few query rows): each row's k indices are split over several CTA
 // pairs, which write unnormalised (O, m, l) partials; a small combine kernel
@@ -71,21 +76,20 @@ constexpr int KVW = 576;             // latent row width (K), first 512 = V
 constexpr int DV = 512;
 constexpr int NB = 64;               // keys per block
 constexpr int Q_ATOM = HQ * 128;     // one 64-column slice of Q (128-byte rows)
-constexpr int Q_ROPE = HQ * 64;      // the 32 rope columns of Q (64-byte rows)
 constexpr int KV_ATOM = NB * 128;    // one 64-column slice of a key block
 constexpr int KV_ROPE = NB * 64;     // the 32 rope columns of a key block
 constexpr int KV_STAGE = 4 * KV_ATOM + KV_ROPE;     // 36 KB
-constexpr int NSTAGE = 3;
+constexpr int NSTAGE = 4;
 constexpr int NSBUF = 3;                            // S/P buffers in TMEM
 constexpr int X_TILE = HQ * NB * 2;                 // 16 KB of float16 logits
 constexpr int X_QUAD = X_TILE / 4;                  // the 32 rows of one TMEM lane quadrant
-constexpr int ONES_BYTES = 16 * 128;                // 16 x 64 bf16 ones: the row-sum operand
-constexpr int MAX_UNIT_BLOCKS = 64;                 // at most 4096 indices per unit
+constexpr int MAX_UNIT_BLOCKS = 32;                 // at most 2048 indices per unit
+constexpr int Q_SMEM_ATOMS = 3;                     // value slices 0-2 of Q_r in shared memory;
+                                                    // slice 3 and the rope columns live in TMEM
 constexpr int OFF_Q = 0;
-constexpr int OFF_KV = 4 * Q_ATOM + Q_ROPE;         // 72 KB
+constexpr int OFF_KV = Q_SMEM_ATOMS * Q_ATOM;       // 48 KB
 constexpr int OFF_X = OFF_KV + NSTAGE * KV_STAGE;   // partner's float16 logits
-constexpr int OFF_ONES = OFF_X + 2 * X_TILE;
-constexpr int OFF_MASK = OFF_ONES + ONES_BYTES;
+constexpr int OFF_MASK = OFF_X + 2 * X_TILE;
 constexpr int OFF_BARS = OFF_MASK + 2 * MAX_UNIT_BLOCKS * 8;
 #ifndef IC_ATTN_GATHER_WARPS
 #define IC_ATTN_GATHER_WARPS 4
@@ -97,21 +101,20 @@ constexpr int GW = IC_ATTN_GATHER_WARPS;            // gather warps (2 or 4)
 constexpr bool GATHER_TMA = IC_ATTN_GATHER_TMA != 0;  // TMA four-row gathers, else coalesced cp.async
 static_assert(GW == 2 || GW == 4, "gather warps");
 constexpr int KPW = NB / GW;                        // key rows of a block per gather warp
-constexpr int W_X = GW, W_Y = GW + 4, W_S = GW + 8, W_PV = GW + 9;   // first warp of each role
+constexpr int W_Y = GW + 4, W_S = GW + 8, W_PV = GW + 9;   // first warp of each role (exchange: GW)
 constexpr int N_THREADS = 32 * (GW + 10);           // gather, 4 exchange, 4 softmax, 2 MMA warps
 constexpr int KV_FULL_ARRIVALS = GATHER_TMA ? GW : 32 * GW;
 static_assert(W_PV + 1 == N_THREADS / 32, "warp roles");
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t TM_O = 0;
 constexpr uint32_t TM_S = 256;                      // S/P buffer b at TM_S + 64 b
-constexpr uint32_t TM_L = TM_S + 64 * NSBUF;        // 16 columns, all equal to l
+constexpr uint32_t TM_QT = TM_S + 64 * NSBUF;       // Q_r slice 3 (32 cols) + rope (16 cols), bf16 pairs
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_THRESHOLD = 8.f;            // log2 units
-static_assert(OFF_ONES % 1024 == 0, "ones operand alignment");
-static_assert(TM_L + 16 <= TMEM_COLS, "tensor memory budget");
+static_assert(TM_QT + 48 <= TMEM_COLS, "tensor memory budget");
 
 struct __align__(8) AttnBars {
-    uint64_t q_full, q_empty;
+    uint64_t q_full, q_empty, q_tmem_full;
     uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
     uint64_t s_full[NSBUF], s_free[NSBUF];
     uint64_t own_full[NSBUF][4];    // exchange warp q -> softmax warp q: own float16 logits in TMEM
@@ -168,6 +171,7 @@ __device__ __forceinline__ void sum_pair(uint32_t own, uint32_t par, float& s0, 
 }
 
 struct AttnArgs {
+    const __nv_bfloat16* q;
     const __nv_bfloat16* kv;
     const int32_t* idx;
     __nv_bfloat16* out;
@@ -196,7 +200,7 @@ __device__ __forceinline__ Unit decode_unit(const AttnArgs& a, int seq) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(N_THREADS, 1)
-attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_qr,
+attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                const __grid_constant__ CUtensorMap map_kv, const __grid_constant__ CUtensorMap map_kvr,
                const AttnArgs args) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -216,6 +220,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
         mbar_init(&bars->q_empty, 1);
+        mbar_init(&bars->q_tmem_full, 4);
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(&bars->kv_full[s], KV_FULL_ARRIVALS);
             mbar_init(&bars->kv_empty[s], 1);
@@ -242,12 +247,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         mbar_init(&bars->drain[1], 1);
         bars->abort = 0;
         fence_mbar_init();
-    }
-    {
-        // the row-sum operand: bf16 ones, read by the tensor core
-        uint32_t* ones = reinterpret_cast<uint32_t*>(smem + OFF_ONES);
-        for (int i = threadIdx.x; i < ONES_BYTES / 4; i += N_THREADS) ones[i] = 0x3f803f80u;
-        fence_proxy_async_smem();
     }
     if (warp == W_S) tmem_alloc<TMEM_COLS>(&bars->tmem_base);
     tc_fence_before();
@@ -382,7 +381,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             if (!ok_all) break;
         }
         if constexpr (!GATHER_TMA) asm volatile("cp.async.wait_all;" ::: "memory");
-    } else if (warp < W_X + 4) {
+    } else if (warp < W_Y) {
         // ------------------------------------------------------------ exchange
         const int quad = warp & 3;                // TMEM lanes 32*quad .. +31
         const int h = quad * 32 + lane;           // head of this thread
@@ -397,6 +396,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             const int nb = bars->n_blocks[ip];
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->info_empty[ip]);
+            if (nb > 0) {
+                // Q_r columns the S MMA reads from TMEM (value slice 3 and the rope
+                // columns), row h, packed as bf16 pairs.  Every S MMA of the previous
+                // unit has finished: this warp has seen the S of its last block.
+                const Unit u = decode_unit(args, seq);
+                const __nv_bfloat16* qrow = args.q + ((int64_t)u.row * HQ + h) * KVW;
+                uint32_t qa[32], qb[16];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(qrow + (int)r * 256 + 192 + 8 * i);
+                    qa[4 * i] = v.x; qa[4 * i + 1] = v.y; qa[4 * i + 2] = v.z; qa[4 * i + 3] = v.w;
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(qrow + 512 + (int)r * 32 + 8 * i);
+                    qb[4 * i] = v.x; qb[4 * i + 1] = v.y; qb[4 * i + 2] = v.z; qb[4 * i + 3] = v.w;
+                }
+                tmem_st32(t_lane + TM_QT, qa);
+                tmem_st16(t_lane + TM_QT + 32, qb);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->q_tmem_full);
+            }
             for (int j = 0; j < nb; ++j, ++g) {
                 const int sb = g % NSBUF;
                 const int slot = g & 1;
@@ -455,6 +478,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             const int nb = bars->n_blocks[ip];
             float m_use = 0.f;      // running max (log2 units); meaningful once m_set
             bool m_set = false;
+            float l = 0.f;          // running sum of the bf16-rounded P
             for (int j = 0; j < nb; ++j, ++g) {
                 const int sb = g % NSBUF;
                 const int slot = g & 1;
@@ -515,9 +539,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                     m_set = true;
                 }
                 uint32_t pw[NB / 2];
+                float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int x = 0; x < NB / 2; ++x)
+                for (int x = 0; x < NB / 2; ++x) {
                     pw[x] = pack_bf16(ex2_approx(sv[2 * x] - m_use), ex2_approx(sv[2 * x + 1] - m_use));
+                    ps[x & 3] += __uint_as_float(pw[x] << 16) + __uint_as_float(pw[x] & 0xffff0000u);
+                }
+                l = (rescale ? l * alpha : l) + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
                 if (rescale) {
                     // O and l must hold P V of block g-1 before they are rescaled
                     if (!warp_wait(&bars->o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, status, abort)) {
@@ -534,12 +562,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                         for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
                         tmem_st32(t_lane + TM_O + 32 * c, o);
                     }
-                    uint32_t lr[16];
-                    tmem_ld16(t_lane + TM_L, lr);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) lr[x] = __float_as_uint(__uint_as_float(lr[x]) * alpha);
-                    tmem_st16(t_lane + TM_L, lr);
                 }
                 tmem_st32(t_lane + TM_S + 64 * sb, pw);
                 tmem_st_wait();
@@ -554,12 +576,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             if (nb > 0) {
                 if (!warp_wait(&bars->o_final, o_use & 1, status, abort)) { ok = false; break; }
                 tc_fence_after();
-                {
-                    uint32_t lr[16];
-                    tmem_ld16(t_lane + TM_L, lr);
-                    tmem_ld_wait();
-                    l_all = m_set ? __uint_as_float(lr[0]) : 0.f;
-                }
+                l_all = m_set ? l : 0.f;
                 const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
 #pragma unroll 1
                 for (int c = 0; c < 8; ++c) {
@@ -610,12 +627,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             bool q_loaded_next = false;
             auto load_q = [&](int seq) {
                 const Unit u = decode_unit(args, seq);
-                mbar_arrive_expect_tx(&bars->q_full, 4 * Q_ATOM + Q_ROPE);
-                for (int a = 0; a < 4; ++a)
+                mbar_arrive_expect_tx(&bars->q_full, Q_SMEM_ATOMS * Q_ATOM);
+                for (int a = 0; a < Q_SMEM_ATOMS; ++a)
                     tma_load_2d(smem + OFF_Q + a * Q_ATOM, &map_q, &bars->q_full, (int)r * 256 + a * 64,
                                 u.row * HQ);
-                tma_load_2d(smem + OFF_Q + 4 * Q_ATOM, &map_qr, &bars->q_full, 512 + (int)r * 32,
-                            u.row * HQ);
             };
             int n = 0;
             for (int seq = pair; seq < args.n_units && ok; seq += n_pairs, ++n) {
@@ -634,7 +649,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                     load_q(seq);
                 }
                 q_loaded_next = false;
-                if (!mbar_wait(&bars->q_full, o_use & 1, status, abort)) break;
+                if (!mbar_wait(&bars->q_full, o_use & 1, status, abort) ||
+                    !mbar_wait(&bars->q_tmem_full, o_use & 1, status, abort))
+                    break;
                 for (int j = 0; j < nb; ++j, ++g) {
                     const int sb = g % NSBUF;
                     const int ks = g % NSTAGE;
@@ -648,7 +665,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                     const uint32_t kv_addr = smem_base + OFF_KV + ks * KV_STAGE;
                     const uint32_t s_tm = tmem + TM_S + 64 * sb;
 #pragma unroll
-                    for (int a = 0; a < 4; ++a) {
+                    for (int a = 0; a < Q_SMEM_ATOMS; ++a) {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint64_t da = desc_sw128(q_addr + a * Q_ATOM + kk * 32, 16, 1024);
@@ -656,11 +673,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                             mma_bf16(s_tm, da, db, id_s, (a | kk) != 0);
                         }
                     }
+                    // value slice 3 and the rope columns: A (Q_r) from TMEM
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t db = desc_sw128(kv_addr + 3 * KV_ATOM + kk * 32, 16, 1024);
+                        mma_bf16_ts(s_tm, tmem + TM_QT + kk * 8, db, id_s, 1u);
+                    }
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk) {
-                        const uint64_t da = desc_sw64(q_addr + 4 * Q_ATOM + kk * 32);
                         const uint64_t db = desc_sw64(kv_addr + 4 * KV_ATOM + kk * 32);
-                        mma_bf16(s_tm, da, db, id_s, 1u);
+                        mma_bf16_ts(s_tm, tmem + TM_QT + 32 + kk * 8, db, id_s, 1u);
                     }
                     issued = true;
                     mma_commit(&bars->s_full[sb]);
@@ -690,8 +712,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         // ------------------------------------------------------------ O += P V, l += P 1 issuer
         if (lane == 0) {
             constexpr uint32_t id_pv = idesc_f32acc(1, 1, HQ, 256, 0, 1);    // O += P V (V MN-major)
-            constexpr uint32_t id_l = idesc_f32acc(1, 1, HQ, 16);            // l += P 1
-            const uint32_t ones_addr = smem_base + OFF_ONES;
             uint32_t g = 0, o_use = 0;
             bool issued = false, ok = true;
             int n = 0;
@@ -714,11 +734,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                     for (int kk = 0; kk < NB / 16; ++kk) {
                         const uint64_t db = desc_sw128(v_addr + kk * 16 * 128, 8192, 1024);
                         mma_bf16_ts(tmem + TM_O, p_tm + kk * 8, db, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < NB / 16; ++kk) {
-                        const uint64_t dl = desc_sw128(ones_addr + kk * 32, 16, 1024);
-                        mma_bf16_ts(tmem + TM_L, p_tm + kk * 8, dl, id_l, (j > 0 || kk > 0) ? 1u : 0u);
                     }
                     issued = true;
                     mma_commit(&bars->kv_empty[g % NSTAGE]);
@@ -853,18 +868,13 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
         return IC_ERR_INVALID_ARG;
     auto fn = encode_fn();
     if (fn == nullptr) return cuda_error("attn_tc");
-    CUtensorMap map_q, map_qr;
+    CUtensorMap map_q;
     cuuint64_t dims[2] = {(cuuint64_t)KVW, (cuuint64_t)r.B * r.Lq * HQ};
     cuuint64_t strides[1] = {(cuuint64_t)KVW * 2};
     cuuint32_t box[2] = {64, (cuuint32_t)HQ};
-    cuuint32_t box_r[2] = {32, (cuuint32_t)HQ};
     cuuint32_t estr[2] = {1, 1};
     if (fn(&map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box,
            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return cuda_error("attn_tc");
-    if (fn(&map_qr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box_r,
-           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cuda_error("attn_tc");
 
@@ -885,6 +895,7 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
         return cuda_error("attn_tc");
 
     AttnArgs a;
+    a.q = static_cast<const __nv_bfloat16*>(q);
     a.kv = static_cast<const __nv_bfloat16*>(kv);
     a.idx = idx;
     a.out = static_cast<__nv_bfloat16*>(out);
@@ -912,7 +923,7 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
                              (int)SMEM_BYTES) != cudaSuccess)
         return cuda_error("attn_tc");
     const int64_t pairs = std::min<int64_t>(units, std::max(1, sm_count() / 2));
-    attn_tc_kernel<<<(unsigned)(2 * pairs), N_THREADS, SMEM_BYTES, s>>>(map_q, map_qr, map_kv, map_kvr, a);
+    attn_tc_kernel<<<(unsigned)(2 * pairs), N_THREADS, SMEM_BYTES, s>>>(map_q, map_kv, map_kvr, a);
     count_launch(IC_LK_ATTN_TC);
     ic_status st = last_launch_status();
     if (st != IC_OK || a.splits <= 1) return st;
