@@ -36,16 +36,6 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
-__device__ __forceinline__ bool elect_one() {
-    uint32_t pred = 0;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "elect.sync _|p, 0xffffffff;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(pred));
-    return pred != 0;
-}
-
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
@@ -258,12 +248,6 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-}  // namespace sm100
-}  // namespace ic
-
-namespace ic {
-namespace sm100 {
-
 // D[tmem] (+)= A[tmem] * B[smem desc]: A (K-major, 16-bit pairs packed per
 // 32-bit column) read from tensor memory.
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
@@ -311,18 +295,6 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t ran
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
-}
-
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
-                 "f"(c), "f"(d)
-                 : "memory");
-}
-
-// Arrive (release at cluster scope) on an mbarrier of another CTA of the cluster.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-                 : "memory");
 }
 
 // Remote arrive without release semantics: for a consumer that hands a
@@ -399,12 +371,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-}  // namespace sm100
-}  // namespace ic
-
-namespace ic {
-namespace sm100 {
-
 // Shared-memory matrix descriptor for the 64-byte swizzled K-major layout:
 // rows of 64 B, 8-row core groups 512 B apart, layout type 4 (SWIZZLE_64B).
 __device__ __forceinline__ uint64_t desc_sw64(uint32_t smem_addr) {
@@ -416,19 +382,6 @@ __device__ __forceinline__ uint64_t desc_sw64(uint32_t smem_addr) {
     d |= (uint64_t)4u << 61;
     return d;
 }
-
-__device__ __forceinline__ void st_cluster_v4_b32(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                                  uint32_t d) {
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b),
-                 "r"(c), "r"(d)
-                 : "memory");
-}
-
-}  // namespace sm100
-}  // namespace ic
-
-namespace ic {
-namespace sm100 {
 
 // Asynchronous 16-byte store into another CTA's shared memory; when it lands
 // it counts 16 bytes of transaction on that CTA's mbarrier (no fence or
@@ -459,12 +412,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-}  // namespace sm100
-}  // namespace ic
-
-namespace ic {
-namespace sm100 {
-
 // Warp-uniform bounded waits: lane 0 waits, the outcome is broadcast, and
 // __syncwarp orders the other lanes' later reads after lane 0's acquire.
 // Every lane gets the same answer, so a timeout can never leave part of a
@@ -485,24 +432,6 @@ __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;
-}
-
-}  // namespace sm100
-}  // namespace ic
-
-namespace ic {
-namespace sm100 {
-
-// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into
-// another CTA's shared memory of the cluster; completion is counted in bytes
-// on that CTA's mbarrier.  No multicast.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
-                                                  uint32_t bar_cluster) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst_cluster),
-        "r"(src_cta), "r"(bytes), "r"(bar_cluster)
-        : "memory");
 }
 
 }  // namespace sm100
