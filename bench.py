@@ -501,6 +501,20 @@ def main():
     _finish(pg)
 
 
+def row_overlap(reused, own, T):
+    """Per row, |own & reused| / |reused| of two [rows, k] index sets whose
+    entries lie in [0, T) or are -1 padding (ignored): the top-k overlap the
+    chunked run reports for S layers.  Runs on the tensors' device."""
+    rows, k = reused.shape
+    off = (torch.arange(rows, device=reused.device, dtype=torch.int64) * (T + 1))[:, None]
+    a = reused.to(torch.int64)
+    b = own.to(torch.int64)
+    a = torch.where(a >= 0, a + off, torch.full_like(a, -1))
+    b = torch.where(b >= 0, b + off, torch.full_like(b, -2))
+    hit = torch.isin(b.flatten(), a.flatten()).view(rows, k).sum(1).to(torch.float64)
+    return hit / (reused >= 0).sum(1).clamp(min=1).to(torch.float64)
+
+
 def run_chunked(args, wl, pattern, dev, pg, rank, world):
     """Chunked prefill: the sequence's L query rows go through the layer stack
     in chunks of wl.chunk rows, chunk c against its causal prefix (q_start =
@@ -642,9 +656,6 @@ def run_chunked(args, wl, pattern, dev, pg, rank, world):
     acc = {}
     for c in range(nch):
         r = rows[c]
-        t_row = torch.arange(c * C, (c + 1) * C, device=dev)
-        m = torch.clamp(t_row + 1, max=wl.k).to(torch.float64)
-        off = (torch.arange(C, device=dev, dtype=torch.int64) * (wl.T + 1))[:, None]
         for l, kind in enumerate(pattern):
             kI = keys[l][0]
             ic.indexer_scores(qI[qkey(l, c)], wI[qkey(l, c)], kI, r, scores, ws,
@@ -652,12 +663,7 @@ def run_chunked(args, wl, pattern, dev, pg, rank, world):
             ic.topk(scores, r, wl.k, own if kind == "S" else idx_buf, ws)
             if kind == "F":
                 continue
-            a = idx_buf[0].to(torch.int64)
-            b = own[0].to(torch.int64)
-            a = torch.where(a >= 0, a + off, torch.full_like(a, -1))
-            b = torch.where(b >= 0, b + off, torch.full_like(b, -2))
-            hit = torch.isin(b.flatten(), a.flatten()).view(C, wl.k).sum(1).to(torch.float64)
-            frac = hit / m
+            frac = row_overlap(idx_buf[0], own[0], wl.T)
             s_, n_, mn = acc.get(l, (0.0, 0, 1.0))
             acc[l] = (s_ + float(frac.sum()), n_ + C, min(mn, float(frac.min())))
     overlap = {"layer_%d" % l: {"mean": v[0] / v[1], "min": v[2]} for l, v in sorted(acc.items())}

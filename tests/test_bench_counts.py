@@ -80,3 +80,24 @@ def test_roofline_line_uses_the_dominant_stage():
                                                            "attention": 0.6},
                                {"indexer": 2, "topk": 2, "attention": 8})
     assert dom == "attention" and roof["bound"] == "hbm" and roof["unit"] == "GB/s"
+
+
+def test_row_overlap_matches_the_oracle():
+    """The chunked run's S-layer overlap equals the oracle's definition,
+    |A & B| / |A| with A the reused set, on ragged (-1 padded) rows."""
+    import numpy as np
+    import torch
+    import oracle
+    rng = np.random.default_rng(7)
+    T, k, rows = 300, 40, 64
+    reused = np.full((rows, k), -1, dtype=np.int32)
+    own = np.full((rows, k), -1, dtype=np.int32)
+    for r in range(rows):
+        m = int(rng.integers(1, k + 1))           # t + 1 < k gives padded rows
+        pool = rng.choice(T, size=min(T, 2 * k), replace=False)
+        reused[r, :m] = np.sort(rng.choice(pool, m, replace=False))
+        own[r, :m] = np.sort(rng.choice(pool, m, replace=False))
+    got = bench.row_overlap(torch.from_numpy(reused), torch.from_numpy(own), T).numpy()
+    ref = oracle.topk_overlap(reused, own)
+    assert np.array_equal(got, ref)
+    assert np.all(bench.row_overlap(torch.from_numpy(reused), torch.from_numpy(reused), T).numpy() == 1.0)
