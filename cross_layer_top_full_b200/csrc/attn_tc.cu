@@ -91,19 +91,11 @@ constexpr int OFF_KV = Q_SMEM_ATOMS * Q_ATOM;       // 48 KB
 constexpr int OFF_X = OFF_KV + NSTAGE * KV_STAGE;   // partner's float16 logits
 constexpr int OFF_MASK = OFF_X + 2 * X_TILE;
 constexpr int OFF_BARS = OFF_MASK + 2 * MAX_UNIT_BLOCKS * 8;
-#ifndef IC_ATTN_GATHER_WARPS
-#define IC_ATTN_GATHER_WARPS 4
-#endif
-#ifndef IC_ATTN_GATHER_TMA
-#define IC_ATTN_GATHER_TMA 1
-#endif
-constexpr int GW = IC_ATTN_GATHER_WARPS;            // gather warps (2 or 4)
-constexpr bool GATHER_TMA = IC_ATTN_GATHER_TMA != 0;  // TMA four-row gathers, else coalesced cp.async
-static_assert(GW == 2 || GW == 4, "gather warps");
+constexpr int GW = 4;                               // gather warps
 constexpr int KPW = NB / GW;                        // key rows of a block per gather warp
 constexpr int W_Y = GW + 4, W_S = GW + 8, W_PV = GW + 9;   // first warp of each role (exchange: GW)
 constexpr int N_THREADS = 32 * (GW + 10);           // gather, 4 exchange, 4 softmax, 2 MMA warps
-constexpr int KV_FULL_ARRIVALS = GATHER_TMA ? GW : 32 * GW;
+constexpr int KV_FULL_ARRIVALS = GW;                // one expect-tx arrival per gather warp
 static_assert(W_PV + 1 == N_THREADS / 32, "warp roles");
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t TM_O = 0;
@@ -308,8 +300,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             // warp w fills key rows KPW*w .. KPW*w + KPW-1 of each block; lane
             // L < KPW holds the row of key KPW*w + L (the indices of block j+1
             // are loaded while block j is issued).  An invalid index becomes
-            // the out-of-range row B*T (zero-filled by TMA) or a zero-byte
-            // cp.async source (zero-filled as well).
+            // the out-of-range row B*T, which TMA fills with zeros.
             const int oob_row = args.B * args.T;
             bool ok_all = true;
             const int key = warp * KPW + lane;
@@ -327,60 +318,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     break;
                 }
                 const uint32_t stage = smem_base + OFF_KV + s * KV_STAGE;
-                if constexpr (GATHER_TMA) {
-                    // (KPW/4) groups of 4 rows x (four 64-column value slices + the 32
-                    // rope columns) tile::gather4 copies; copy c (group c / 5, slice
-                    // c % 5) is issued by lane c % 32
-                    constexpr int OPS = KPW / 4 * 5;
-                    if (lane == 0) mbar_arrive_expect_tx(&bars->kv_full[s], KPW / 4 * (4 * 512 + 256));
-                    __syncwarp();
+                // (KPW/4) groups of 4 rows x (four 64-column value slices + the 32
+                // rope columns) tile::gather4 copies; copy c (group c / 5, slice
+                // c % 5) is issued by lane c % 32
+                constexpr int OPS = KPW / 4 * 5;
+                if (lane == 0) mbar_arrive_expect_tx(&bars->kv_full[s], KPW / 4 * (4 * 512 + 256));
+                __syncwarp();
 #pragma unroll
-                    for (int c0 = 0; c0 < OPS; c0 += 32) {
-                        const int c = c0 + lane;
-                        const int grp = (c < OPS ? c : 0) / 5, sl = c % 5;
-                        const int r0 = __shfl_sync(0xffffffffu, row_lane, 4 * grp);
-                        const int r1 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 1);
-                        const int r2 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 2);
-                        const int r3 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 3);
-                        if (c < OPS) {
-                            const int krow = KPW * warp + 4 * grp;
-                            if (sl < 4)
-                                tma_gather4(stage + sl * KV_ATOM + krow * 128, &map_kv, &bars->kv_full[s],
-                                            (int)r * 256 + sl * 64, r0, r1, r2, r3);
-                            else
-                                tma_gather4(stage + 4 * KV_ATOM + krow * 64, &map_kvr, &bars->kv_full[s],
-                                            512 + (int)r * 32, r0, r1, r2, r3);
-                        }
+                for (int c0 = 0; c0 < OPS; c0 += 32) {
+                    const int c = c0 + lane;
+                    const int grp = (c < OPS ? c : 0) / 5, sl = c % 5;
+                    const int r0 = __shfl_sync(0xffffffffu, row_lane, 4 * grp);
+                    const int r1 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 1);
+                    const int r2 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 2);
+                    const int r3 = __shfl_sync(0xffffffffu, row_lane, 4 * grp + 3);
+                    if (c < OPS) {
+                        const int krow = KPW * warp + 4 * grp;
+                        if (sl < 4)
+                            tma_gather4(stage + sl * KV_ATOM + krow * 128, &map_kv, &bars->kv_full[s],
+                                        (int)r * 256 + sl * 64, r0, r1, r2, r3);
+                        else
+                            tma_gather4(stage + 4 * KV_ATOM + krow * 64, &map_kvr, &bars->kv_full[s],
+                                        512 + (int)r * 32, r0, r1, r2, r3);
                     }
-                } else {
-                    // one warp instruction per row for the 512 value bytes (lane =
-                    // 16-byte chunk), then 8 rows per instruction for the 64 rope bytes
-                    const int a_val = lane >> 3, ch_val = lane & 7;
-#pragma unroll 4
-                    for (int rr = 0; rr < KPW; ++rr) {
-                        const int krow = KPW * warp + rr;
-                        const int row = __shfl_sync(0xffffffffu, row_lane, rr);
-                        const bool valid = row != oob_row;
-                        cp_async16(stage + a_val * KV_ATOM + krow * 128 + ((ch_val ^ (krow & 7)) << 4),
-                                   args.kv + (int64_t)(valid ? row : 0) * KVW + r * 256 + lane * 8,
-                                   valid ? 16u : 0u);
-                    }
-#pragma unroll
-                    for (int i = 0; i < KPW / 8; ++i) {
-                        const int rr = 8 * i + (lane >> 2), chr = lane & 3;
-                        const int krow = KPW * warp + rr;
-                        const int row = __shfl_sync(0xffffffffu, row_lane, rr);
-                        const bool valid = row != oob_row;
-                        cp_async16(stage + 4 * KV_ATOM + krow * 64 + ((chr ^ ((krow >> 1) & 3)) << 4),
-                                   args.kv + (int64_t)(valid ? row : 0) * KVW + 512 + r * 32 + chr * 8,
-                                   valid ? 16u : 0u);
-                    }
-                    cp_async_arrive_noinc(&bars->kv_full[s]);
                 }
             }
             if (!ok_all) break;
         }
-        if constexpr (!GATHER_TMA) asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp < W_Y) {
         // ------------------------------------------------------------ exchange
         const int quad = warp & 3;                // TMEM lanes 32*quad .. +31
@@ -660,7 +624,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                         ok = false;
                         break;
                     }
-                    if constexpr (!GATHER_TMA) fence_proxy_async_smem();  // cp.async data -> tensor core
                     tc_fence_after();
                     const uint32_t kv_addr = smem_base + OFF_KV + ks * KV_STAGE;
                     const uint32_t s_tm = tmem + TM_S + 64 * sb;

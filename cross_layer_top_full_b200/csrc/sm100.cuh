@@ -351,26 +351,6 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     }
 }
 
-// ------------------------------------------------------------------ cp.async (16 B, L2 only)
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-
-// Arrive on `bar` once all prior cp.async of this thread have completed
-// (the arrival is counted against the barrier's expected count).
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-
-// Make generic-proxy shared-memory writes visible to the async proxy
-// (tensor-core operand reads).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // Shared-memory matrix descriptor for the 64-byte swizzled K-major layout:
 // rows of 64 B, 8-row core groups 512 B apart, layout type 4 (SWIZZLE_64B).
 __device__ __forceinline__ uint64_t desc_sw64(uint32_t smem_addr) {
