@@ -176,11 +176,10 @@ ic_status ic_topk(const float* scores, int64_t ld_scores, ic_rows r, int k, int3
  *   vmat value row (b,s) starts at vmat + (b*T + s) * v_row_stride elements
  *        (a latent KV cache passes the same pointer twice: K = the whole
  *        576-wide row, V = its first 512 columns)
- *   idx  [B, Lq, k] int32: positions in [0, t] or -1 (skipped).  The valid
- *        entries must form a prefix of the row when the tensor-core path is
- *        used (ic_topk's output always does).  An entry outside [0, t] is
- *        never dereferenced: the row is computed without it and the status
- *        bit IC_ERR_INDEX_RANGE is set.
+ *   idx  [B, Lq, k] int32: positions in [0, t] or -1 (skipped, anywhere in
+ *        the row).  An entry outside [0, t] and not -1 is never
+ *        dereferenced: the row is computed without it and the status bit
+ *        IC_ERR_INDEX_RANGE is set.
  *   out  [B, Lq, Hq, d_v] of dt.  A row with no valid index gets zeros.
  * Supported: Hq in [1,128], d_qk, d_v in [1,576].  The tensor-core path is
  * used for IC_BF16 with Hq == 128, d_qk == 576, d_v == 512 and kmat == vmat
