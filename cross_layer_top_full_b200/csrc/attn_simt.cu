@@ -125,7 +125,8 @@ ic_status launch_typed(const void* q, const void* kmat, int64_t ks, const void* 
                        float scale, void* out, uint32_t* status, cudaStream_t s) {
     const size_t smem = sizeof(float) * (size_t)KB * (d_qk + d_v);
     auto kern = attn_simt_kernel<T>;
-    if (smem > 48 * 1024) {
+    // opt in to more than 48 KB whenever dynamic + static (sel[KB]) pass it
+    if (smem + sizeof(int) * KB > 48 * 1024) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
             return cuda_error("attn_simt");
