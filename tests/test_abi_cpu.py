@@ -143,3 +143,13 @@ def test_workspace_sizes_grow_with_the_problem(lib):
     assert ic.topk_workspace_size((1, 4, 0, 4), 2) == ic.STATUS_BYTES
     latent = ic.sparse_attn_workspace_size((32, 1, 32767, 32768), 2048, 128, 576, 512, ic.BF16)
     assert latent >= ic.STATUS_BYTES
+
+
+def test_selftest_rejects_a_bad_workspace_before_launching(lib):
+    """The failure-path self-test validates its workspace on the host and
+    returns before any CUDA call (this host has no GPU to launch on)."""
+    ws = _FakeTensor(4096)
+    assert lib.ic_selftest_wait_timeout(ws.addr + 8, 4096, None) == -1    # misaligned
+    assert lib.ic_selftest_wait_timeout(ws.addr, 16, None) == -1          # < IC_STATUS_BYTES
+    assert lib.ic_selftest_wait_timeout(None, 4096, None) == -1           # no workspace
+    assert lib.ic_last_error() == b""                                     # no CUDA failure seen
