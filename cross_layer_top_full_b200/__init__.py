@@ -67,6 +67,7 @@ _P = ctypes.c_void_p
 _SIG = {
     "ic_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ic_last_error": (ctypes.c_char_p, []),
+    "ic_check_status": (ctypes.c_int, [_P, _P]),
     "ic_selftest_wait_timeout": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "ic_version": (ctypes.c_int, []),
     "ic_kernel_launches": (ctypes.c_uint64, [ctypes.c_int]),

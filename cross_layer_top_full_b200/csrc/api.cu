@@ -34,14 +34,14 @@ ic_status cuda_error(const char* where) {
     const cudaError_t e = cudaGetLastError();
     snprintf(tl_error, sizeof(tl_error), "%s: %s", where,
              e == cudaSuccess ? "CUDA driver call failed" : cudaGetErrorString(e));
-    return cuda_error("api");
+    return IC_ERR_CUDA;
 }
 
 ic_status last_launch_status() {
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) return IC_OK;
     snprintf(tl_error, sizeof(tl_error), "kernel launch: %s", cudaGetErrorString(e));
-    return cuda_error("api");
+    return IC_ERR_CUDA;
 }
 
 namespace {
@@ -165,6 +165,12 @@ ic_status ic_read_status(void* ws, void* stream, int32_t* device_status) {
     if (v & IC_DEV_INDEX_RANGE) return IC_ERR_INDEX_RANGE;
     if (v & IC_DEV_TIMEOUT) return IC_ERR_TIMEOUT;
     return IC_OK;
+}
+
+ic_status ic_check_status(void* ws, void* stream) {
+    if (ws == nullptr) return IC_ERR_INVALID_ARG;
+    int32_t bits = 0;
+    return ic_read_status(ws, stream, &bits);
 }
 
 size_t ic_indexer_workspace_size(ic_rows r, int H_I, int d_I, ic_dtype dt) {

@@ -96,6 +96,11 @@ ic_status ic_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * it.  Returns IC_OK when no bit was set, else the error of the lowest bit. */
 ic_status ic_read_status(void* ws, void* stream, int32_t* device_status);
 
+/* ic_read_status without the raw bits: synchronise `stream`, clear the
+ * status word of `ws` and return IC_OK, IC_ERR_INDEX_RANGE or IC_ERR_TIMEOUT
+ * (the error of the lowest set bit). */
+ic_status ic_check_status(void* ws, void* stream);
+
 /* Failure-path self-test: launches one CTA whose pipeline wait (the
  * library's bounded mbarrier wait) never completes.  After about 1 s the
  * wait gives up, bit 1 (wait timeout) of the status word of `ws` is set and

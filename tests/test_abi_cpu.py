@@ -152,4 +152,20 @@ def test_selftest_rejects_a_bad_workspace_before_launching(lib):
     assert lib.ic_selftest_wait_timeout(ws.addr + 8, 4096, None) == -1    # misaligned
     assert lib.ic_selftest_wait_timeout(ws.addr, 16, None) == -1          # < IC_STATUS_BYTES
     assert lib.ic_selftest_wait_timeout(None, 4096, None) == -1           # no workspace
-    assert lib.ic_last_error() == b""                                     # no CUDA failure seen
+    assert lib.ic_check_status(None, None) == -1                          # no workspace
+
+
+def test_cuda_failure_returns_an_error_with_its_text(lib):
+    """A failing launch returns IC_ERR_CUDA at once and ic_last_error names
+    the CUDA error; the binding puts the text into its exception.  On this
+    host (no usable GPU) every launch fails, which exercises the path."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present: the launch would run (the GPU tests cover it)")
+    ws = _FakeTensor(4096)
+    assert lib.ic_selftest_wait_timeout(ws.addr, 4096, None) == -5        # IC_ERR_CUDA
+    text = lib.ic_last_error().decode()
+    assert text.startswith("kernel launch: ") and len(text) > len("kernel launch: ")
+    with pytest.raises(ic.IcError) as e:
+        ic.selftest_wait_timeout(ws)
+    assert e.value.code == -5 and "kernel launch" in str(e.value)
