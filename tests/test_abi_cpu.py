@@ -169,3 +169,6 @@ def test_cuda_failure_returns_an_error_with_its_text(lib):
     with pytest.raises(ic.IcError) as e:
         ic.selftest_wait_timeout(ws)
     assert e.value.code == -5 and "kernel launch" in str(e.value)
+    # a failing runtime call (not a launch) goes through the same recorder
+    assert lib.ic_workspace_init(ws.addr, 4096, None) == -5
+    assert lib.ic_last_error().decode().startswith("api: ")
