@@ -19,7 +19,8 @@
  *     keeps no per-call state on the device.
  *   - Arrays are dense, row-major, with the layouts stated per argument.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
- *     default stream) and never synchronise, except ic_read_status.
+ *     default stream) and never synchronise, except ic_read_status and
+ *     ic_check_status.
  *   - Argument errors are returned before anything is launched.  A failed
  *     launch returns IC_ERR_CUDA.  Errors the kernels detect themselves (an
  *     index outside its row's causal range, a wait that ran out of time) are

@@ -101,7 +101,7 @@ def test_indexer_general_inputs_within_tolerance(dev, dtype):
                                     ((3, 1, 32767, 32768), 2048), # decode rows, cached
                                     ((2, 3, 40000, 40003), 2048), # few long rows of unequal length
                                     ((1, 2, 199998, 200000), 2048),
-                                    # row caches of 47.9 KB and exactly 48 KB of shared memory
+                                    # row caches of 46.9 KiB and exactly 48 KiB of shared memory
                                     # (plus the static select state: past the default limit)
                                     ((1, 300, 11700, 12000), 2048),
                                     ((1, 300, 11988, 12288), 2048),
