@@ -138,7 +138,12 @@ def test_topk_long_rows_of_equal_scores(dev):
 # ------------------------------------------------------------------------- attention
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("Hq,d_qk,d_v,latent", [(8, 64, 64, False), (128, 576, 512, True),
-                                                (3, 40, 24, False)])
+                                                (3, 40, 24, False),
+                                                # CUDA-core path: 16 staged K/V rows of
+                                                # 256 + 512 floats are exactly 48 KiB of dynamic
+                                                # shared memory, past the default limit with the
+                                                # kernel's static part
+                                                (4, 256, 512, False)])
 def test_sparse_attention_within_tolerance(dev, dtype, Hq, d_qk, d_v, latent):
     rows = (2, 37, 90, 127)        # q_start > 0, ragged
     B, Lq, q_start, T = rows
