@@ -282,6 +282,42 @@ def _blas_threads():
         return len(os.sched_getaffinity(0))
 
 
+def oracle_layers(wl, pattern):
+    """The layers the oracle sample runs: all of them, except for long decode
+    caches, where the first F group (4 layers) is timed and the rate scaled
+    by the share of layers it holds, so host memory stays bounded."""
+    if wl.L == 1 and wl.T * len(pattern) > 2_000_000:
+        return pattern[:4]
+    return pattern
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_baseline(wl, pattern, value, done, spent, how):
+    """The cpu_baseline object: the float64 oracle's rate on a bounded
+    sample (`how` says how the query rows were drawn)."""
+    lay = oracle_layers(wl, pattern)
+    if lay == pattern:
+        layers, note = "all %d layers of %s" % (len(pattern), pattern), ""
+    else:
+        layers = "the first %d of the %d layers of %s" % (len(lay), len(pattern), pattern)
+        note = "; rate scaled to all layers"
+    return {"value": value, "unit": "tok/s", "cores": _blas_threads(), "kind": "oracle",
+            "cpu_model": cpu_model(),
+            "sample": "%d %s of %s through %s (float64 NumPy, %.1f s of oracle time%s)"
+                      % (done, how, wl.name, layers, spent, note)}
+
+
 def oracle_sample(wl, pattern, budget_s):
     """Time the float64 oracle (as it stands) on a bounded sample of the
     workload: prefill -> blocks of consecutive query rows at random offsets of
@@ -294,11 +330,7 @@ def oracle_sample(wl, pattern, budget_s):
     import oracle
     rng = np.random.default_rng(0)
     done, spent, n = 0, 0.0, 1
-    # long decode caches: time the first F group of layers and scale by the
-    # share of layers it holds (host memory stays bounded)
-    sub_pattern = pattern
-    if wl.L == 1 and wl.T * len(pattern) > 2_000_000:
-        sub_pattern = pattern[:4]
+    sub_pattern = oracle_layers(wl, pattern)
     layer_share = len(sub_pattern) / len(pattern)
     dec_inputs = None
     while spent < budget_s:
@@ -469,11 +501,8 @@ def main():
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         rps, done, spent = oracle_sample(wl, pattern, args.cpu_budget)
-        lay = len(pattern) if (wl.L > 1 or wl.T * len(pattern) <= 2_000_000) else 4
-        cpu = {"value": rps, "unit": "tok/s", "cores": _blas_threads(), "kind": "oracle",
-               "sample": "%d query rows of %s through %d of the %d layers of %s (float64 NumPy, "
-                         "%.1f s; rate scaled to all layers)"
-                         % (done, wl.name, lay, len(pattern), pattern, spent)}
+        cpu = cpu_baseline(wl, pattern, rps, done, spent,
+                           "query rows" if wl.L > 1 else "single-sequence decode steps")
     line = {
         "metric": "prefill tok/s (IndexCache pattern) with all-F comparison; roofline of the "
                   "dominant kernel" if wl.L > 1 else "decode tok/s (IndexCache pattern)",
@@ -676,9 +705,7 @@ def run_chunked(args, wl, pattern, dev, pg, rank, world):
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         rps, done, spent = oracle_sample(wl, pattern, args.cpu_budget)
-        cpu = {"value": rps, "unit": "tok/s", "cores": _blas_threads(), "kind": "oracle",
-               "sample": "%d query rows of %s at random positions through all %d layers of %s "
-                         "(float64 NumPy, %.1f s)" % (done, wl.name, nl, pattern, spent)}
+        cpu = cpu_baseline(wl, pattern, rps, done, spent, "query rows at random positions")
     per_step_ms = ms / args.steps
     avg = {k: float(np.mean(v)) for k, v in stages.items()}
     line = {
@@ -789,7 +816,6 @@ def run_reference(args, wl, pattern, rank, world):
         done_all += done
         spent_all += spent
     value = done_all / spent_all
-    cores = _blas_threads()
     line = {
         "impl": "reference",
         "metric": "prefill tok/s (IndexCache pattern) with all-F comparison; roofline of the "
@@ -799,9 +825,8 @@ def run_reference(args, wl, pattern, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "pattern": pattern, "B": wl.B, "L": wl.L, "T": wl.T,
                    "k": wl.k},
-        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
-                         "sample": "%d sampled query rows of %s through all layers of %s per run "
-                                   "(float64 NumPy)" % (done_all, wl.name, pattern)},
+        "cpu_baseline": cpu_baseline(wl, pattern, value, done_all, spent_all,
+                                     "query rows" if wl.L > 1 else "single-sequence decode steps"),
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -101,3 +101,17 @@ def test_row_overlap_matches_the_oracle():
     ref = oracle.topk_overlap(reused, own)
     assert np.array_equal(got, ref)
     assert np.all(bench.row_overlap(torch.from_numpy(reused), torch.from_numpy(reused), T).numpy() == 1.0)
+
+
+@pytest.mark.parametrize("name,timed", [("prefill_8k_bf16", 4), ("decode_b32_t32k_bf16", 8),
+                                        ("decode_b8_t200k_fp8", 4)])
+def test_cpu_baseline_says_which_layers_the_oracle_timed(name, timed):
+    wl = synth.WORKLOADS[name]
+    assert len(bench.oracle_layers(wl, wl.pattern)) == timed
+    cb = bench.cpu_baseline(wl, wl.pattern, 1.5, 7, 12.0, "query rows")
+    assert cb["kind"] == "oracle" and cb["unit"] == "tok/s" and cb["value"] == 1.5
+    assert cb["cores"] >= 1 and cb["cpu_model"]
+    if timed < len(wl.pattern):
+        assert "first %d of the %d layers" % (timed, len(wl.pattern)) in cb["sample"]
+    else:
+        assert "all %d layers" % timed in cb["sample"]
