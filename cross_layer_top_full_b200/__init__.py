@@ -113,11 +113,22 @@ def lib() -> ctypes.CDLL:
 
 # --------------------------------------------------------------------------- helpers
 def _ptr(x) -> Optional[int]:
-    """Device/host address of a tensor, or an int address, or None."""
+    """Address of a tensor, or an int address passed through, or None.
+
+    The library reads every array argument as a dense row-major DEVICE array,
+    so a torch tensor in host memory (which a kernel would dereference as a
+    bad address) or a strided view (which it would misread) is refused here,
+    before the call."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
+    if getattr(x, "is_cuda", True) is False:
+        raise ValueError("expected a CUDA tensor, got one on %s" % x.device)
+    contiguous = getattr(x, "is_contiguous", None)
+    if contiguous is not None and not contiguous():
+        raise ValueError("expected a contiguous tensor, got shape %s with strides %s"
+                         % (tuple(x.shape), tuple(x.stride())))
     return x.data_ptr()
 
 

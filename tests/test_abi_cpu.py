@@ -172,3 +172,31 @@ def test_cuda_failure_returns_an_error_with_its_text(lib):
     # a failing runtime call (not a launch) goes through the same recorder
     assert lib.ic_workspace_init(ws.addr, 4096, None) == -5
     assert lib.ic_last_error().decode().startswith("api: ")
+
+
+def test_binding_refuses_host_tensors_and_strided_views(lib):
+    import torch
+    before = ic.kernel_launches(0)
+    rows = (1, 4, 0, 4)
+    host = torch.zeros(1, 4, 4)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        ic.topk(host, rows, 2, torch.zeros(1, 4, 2, dtype=torch.int32), _FakeTensor(4096))
+
+    class _StridedDevice:
+        """A device tensor's attributes, as a transposed view would report them."""
+        is_cuda = True
+        shape = (1, 4, 4)
+        device = "cuda:0"
+
+        def is_contiguous(self):
+            return False
+
+        def stride(self):
+            return (16, 1, 4)
+
+        def data_ptr(self):
+            return 1 << 40
+
+    with pytest.raises(ValueError, match="contiguous"):
+        ic.topk(_StridedDevice(), rows, 2, 1 << 40, _FakeTensor(4096))
+    assert ic.kernel_launches(0) == before
