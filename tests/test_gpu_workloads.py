@@ -2,26 +2,29 @@
 the benchmark times (the whole F/S stack through ic_layer_stack_forward).
 
 The oracle cannot redo a full workload in float64 within a test, so each
-check covers sampled outputs the oracle computes one by one: sampled query
-rows (prefill) or every sequence of a few layers (decode).  Per checked row:
-  * F layer: the kernel's indices obey the top-k band rule against the
-    oracle's float64 scores;
-  * S layer: its indices are the preceding F layer's, bit for bit (all rows);
-  * attention: where the kernel chose exactly the oracle's top-k set (all but
-    allowed near-tie swaps), the output is within the attention tolerance of
-    the oracle's, computed from the oracle's own indices.
-For decode the oracle reads only its own selected KV rows, which are gathered
-on the device by torch indexing with the oracle's indices (never with the
-kernel's) to keep host memory bounded.
+check covers outputs the oracle computes one by one (tests/stack_check.py):
+  * prefill 8K: the indices of all 8192 rows; attention on 512 seeded rows
+    (always rows 0, 1, k-1, k, k+1 and L-1) of all 4 layers;
+  * decode 32 x 32K: every sequence, indices and attention of all 8 layers;
+  * decode 8 x 200K (FP8 indexer): every sequence, all 48 layers;
+  * chunked prefill 64K: all 16 chunks, 16 rows each (always the chunk's
+    first and last row), indices and attention of all 12 layers.
+Per checked row: an F layer's indices obey the top-k band rule against the
+oracle's float64 scores; an S layer's indices are the F layer's bit for bit
+(all rows); attention, where the kernel chose exactly the oracle's top-k set
+(all but allowed near-tie swaps), is within the attention tolerance of the
+oracle's, computed from the oracle's own indices.  Each test also requires
+that the attention of most checked rows was compared: 80 % with the bf16
+indexer, 50 % with the FP8 one, whose tensor-core accumulation of 128 e4m3
+products is allowed more near-tie swaps (the band rule still holds on every
+row).
 """
-import numpy as np
 import pytest
 import torch
 
-import oracle
 import cross_layer_top_full_b200 as ic
 from cross_layer_top_full_b200 import synth
-from parity_util import check_attention, check_topk_band, host64
+from stack_check import check_stack, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -57,62 +60,19 @@ def run_stack(wl, pattern, inputs, rows, dev):
     return outs, copies, ic.kernel_launches(1) - n0
 
 
-def oracle_scores(wl, inp, q_start, rows, seqs):
-    """float64 indexer scores [len(seqs), len(rows), T] of query rows `rows`
-    (relative to the call's q_start) of sequences `seqs`, each row computed
-    on its own from the device inputs; -inf beyond the row's causal range."""
-    fp8 = wl.idx_dtype == "e4m3"
-    T = inp["k_I"].shape[1]
-    out = np.full((len(seqs), len(rows), T), -np.inf)
-    for bi, b in enumerate(seqs):
-        kI = host64(inp["k_I"][b:b + 1])
-        ks = host64(inp["k_scale"][b:b + 1]) if fp8 else None
-        for ri, i in enumerate(rows):
-            qs = host64(inp["q_scale"][b:b + 1, i:i + 1]) if fp8 else None
-            sc = oracle.indexer_scores(host64(inp["q_I"][b:b + 1, i:i + 1]),
-                                       host64(inp["w"][b:b + 1, i:i + 1]), kI, q_start + i, qs, ks,
-                                       fp8=fp8)
-            out[bi, ri] = sc[0, 0]
-    return out
-
-
-def oracle_attention_rows(wl, inp, ref_idx, b, i):
-    """Oracle output of row (b, i) over the oracle's indices ref_idx [k]."""
-    J = torch.as_tensor(ref_idx[ref_idx >= 0], dtype=torch.long, device=inp["kv"].device)
-    kvJ = host64(inp["kv"][b].index_select(0, J))          # only the selected rows
-    q = host64(inp["q"][b, i])[None, None]
-    pos = np.arange(kvJ.shape[0], dtype=np.int32)[None, None]
-    return oracle.sparse_attention(q, kvJ[None], kvJ[None, :, : wl.d_v], pos, wl.scale)[0, 0]
-
-
 # --------------------------------------------------------------------------- prefill 8k
 def test_prefill_8k_bf16_full_size(dev):
     wl = synth.WORKLOADS["prefill_8k_bf16"]
     inputs = [synth.layer_inputs(wl, l, dev) for l in range(wl.n_layers)]
     outs, copies, n_ix = run_stack(wl, wl.pattern, inputs, (wl.B, wl.L, 0, wl.T), dev)
     assert n_ix == wl.pattern.count("F")
-    rng = np.random.default_rng(1)
-    rows = sorted(set([0, 1, wl.k - 1, wl.k, wl.k + 1, wl.L - 1] +
-                      rng.choice(wl.L, 18, replace=False).tolist()))
-    n_same = 0
-    last_f, ref_idx = None, None
-    for l, kind in enumerate(wl.pattern):
-        gidx = host64(copies[l])
-        if kind == "F":
-            last_f = l
-            sc = oracle_scores(wl, inputs[l], 0, rows, [0])
-            check_topk_band(gidx[:, rows], sc, 0, wl.k, rows=rows)
-            ref_idx = oracle.topk_indices(sc, 0, wl.k, rows=rows)
-        else:
-            assert np.array_equal(gidx, host64(copies[last_f])), "S layer %d" % l
-        got = host64(outs[l][0, rows])
-        for r_i, i in enumerate(rows):
-            if not np.array_equal(gidx[0, i], ref_idx[0, r_i]):
-                continue                                    # allowed near-tie swap
-            n_same += 1
-            ref = oracle_attention_rows(wl, inputs[l], ref_idx[0, r_i], 0, i)
-            check_attention(got[r_i], ref, "prefill_8k layer %d row %d" % (l, i))
-    assert n_same >= 0.9 * len(rows) * wl.n_layers
+    attn_rows = sample_rows(wl.L, 512, seed=1,
+                            always=(0, 1, wl.k - 1, wl.k, wl.k + 1, wl.L - 1))
+    n_cmp, n_same = check_stack(wl, wl.pattern, inputs, copies, outs, 0, [0], range(wl.L),
+                                attn_rows, range(wl.n_layers), "prefill_8k")
+    assert n_same >= 0.8 * n_cmp
+    del inputs, outs, copies
+    torch.cuda.empty_cache()
 
 
 # --------------------------------------------------------------------------- decode 32 x 32k
@@ -121,91 +81,45 @@ def test_decode_b32_t32k_bf16_full_size(dev):
     inputs = [synth.layer_inputs(wl, l, dev) for l in range(wl.n_layers)]
     outs, copies, n_ix = run_stack(wl, wl.pattern, inputs, (wl.B, 1, wl.q_start, wl.T), dev)
     assert n_ix == wl.pattern.count("F")
-    check_layers = {0, 1, 4, 7}
-    n_same = 0
-    last_f, ref_idx = None, None
-    for l, kind in enumerate(wl.pattern):
-        gidx = host64(copies[l])
-        if kind == "F":
-            last_f = l
-            sc = oracle_scores(wl, inputs[l], wl.q_start, [0], range(wl.B))
-            check_topk_band(gidx, sc, wl.q_start, wl.k)
-            ref_idx = oracle.topk_indices(sc, wl.q_start, wl.k)
-        else:
-            assert np.array_equal(gidx, host64(copies[last_f]))
-        if l not in check_layers:
-            continue
-        got = host64(outs[l])
-        for b in range(wl.B):
-            if not np.array_equal(gidx[b, 0], ref_idx[b, 0]):
-                continue
-            n_same += 1
-            ref = oracle_attention_rows(wl, inputs[l], ref_idx[b, 0], b, 0)
-            check_attention(got[b, 0], ref, "decode_b32 layer %d seq %d" % (l, b))
-    assert n_same >= 0.9 * wl.B * len(check_layers)
+    n_cmp, n_same = check_stack(wl, wl.pattern, inputs, copies, outs, wl.q_start, range(wl.B),
+                                [0], [0], range(wl.n_layers), "decode_b32")
+    assert n_same >= 0.8 * n_cmp
+    del inputs, outs, copies
+    torch.cuda.empty_cache()
 
 
 # --------------------------------------------------------------------------- decode fp8 200k
-def test_decode_b8_t200k_fp8_first_8_layers(dev):
-    """Full B=8, T=200000 with the FP8 indexer; the first 8 of the 48 layers
-    (FSSSFSSS) to bound device memory in a test (the benchmark runs all 48)."""
+def test_decode_b8_t200k_fp8_full_size(dev):
+    """B = 8, T = 200000, all 48 layers ((FSSS) x 12) with the FP8 indexer:
+    about 98 GB of layer inputs on the device."""
     wl = synth.WORKLOADS["decode_b8_t200k_fp8"]
-    pattern = wl.pattern[:8]
-    inputs = [synth.layer_inputs(wl, l, dev) for l in range(len(pattern))]
-    outs, copies, n_ix = run_stack(wl, pattern, inputs, (wl.B, 1, wl.q_start, wl.T), dev)
-    assert n_ix == 2
-    n_same = 0
-    last_f, ref_idx = None, None
-    for l, kind in enumerate(pattern):
-        gidx = host64(copies[l])
-        if kind == "F":
-            last_f = l
-            sc = oracle_scores(wl, inputs[l], wl.q_start, [0], range(wl.B))
-            check_topk_band(gidx, sc, wl.q_start, wl.k)
-            ref_idx = oracle.topk_indices(sc, wl.q_start, wl.k)
-        else:
-            assert np.array_equal(gidx, host64(copies[last_f]))
-        if l not in (0, 1, 4, 7):
-            continue
-        got = host64(outs[l])
-        for b in range(wl.B):
-            if not np.array_equal(gidx[b, 0], ref_idx[b, 0]):
-                continue
-            n_same += 1
-            ref = oracle_attention_rows(wl, inputs[l], ref_idx[b, 0], b, 0)
-            check_attention(got[b, 0], ref, "decode_fp8 layer %d seq %d" % (l, b))
-    assert n_same >= 0.75 * wl.B * 4
+    inputs = [synth.layer_inputs(wl, l, dev) for l in range(wl.n_layers)]
+    outs, copies, n_ix = run_stack(wl, wl.pattern, inputs, (wl.B, 1, wl.q_start, wl.T), dev)
+    assert n_ix == wl.pattern.count("F") == 12
+    n_cmp, n_same = check_stack(wl, wl.pattern, inputs, copies, outs, wl.q_start, range(wl.B),
+                                [0], [0], range(wl.n_layers), "decode_fp8")
+    assert n_same >= 0.5 * n_cmp
+    del inputs, outs, copies
+    torch.cuda.empty_cache()
 
 
 # --------------------------------------------------------------------------- chunked 64k
-def test_chunked_prefill_64k_bf16_sampled_chunks(dev):
-    """All 12 layers, chunks 0, 7 and 15 of the 16 (keys up to 65536), each
-    run as in the chunked prefill: q_start = 4096 c, T = 4096 (c + 1)."""
+def test_chunked_prefill_64k_bf16_every_chunk(dev):
+    """All 12 layers and all 16 chunks, each run as in the chunked prefill:
+    q_start = 4096 c, T = 4096 (c + 1)."""
     wl = synth.WORKLOADS["chunked_prefill_64k_bf16"]
     C = wl.chunk
-    rng = np.random.default_rng(3)
-    for c in (0, 7, 15):
+    n_cmp = n_same = 0
+    for c in range(wl.L // C):
         inputs = [synth.layer_inputs(wl, l, dev, chunk=c) for l in range(wl.n_layers)]
         q_start, T = c * C, (c + 1) * C
         outs, copies, n_ix = run_stack(wl, wl.pattern, inputs, (1, C, q_start, T), dev)
         assert n_ix == wl.pattern.count("F")
-        rows = sorted(set([0, C - 1] + rng.choice(C, 3, replace=False).tolist()))
-        attn_rows = rows[:3]
-        last_f, ref_idx = None, None
-        for l, kind in enumerate(wl.pattern):
-            gidx = host64(copies[l])
-            if kind == "F":
-                last_f = l
-                sc = oracle_scores(wl, inputs[l], q_start, rows, [0])
-                check_topk_band(gidx[:, rows], sc, q_start, wl.k, rows=rows)
-                ref_idx = oracle.topk_indices(sc, q_start, wl.k, rows=rows)
-            else:
-                assert np.array_equal(gidx, host64(copies[last_f]))
-            got = host64(outs[l][0, attn_rows])
-            for r_i, i in enumerate(attn_rows):
-                if not np.array_equal(gidx[0, i], ref_idx[0, r_i]):
-                    continue
-                ref = oracle_attention_rows(wl, inputs[l], ref_idx[0, r_i], 0, i)
-                check_attention(got[r_i], ref, "chunk %d layer %d row %d" % (c, l, i))
+        rows = sample_rows(C, 14, seed=3 + c, always=(0, C - 1))
+        cmp_c, same_c = check_stack(wl, wl.pattern, inputs, copies, outs, q_start, [0], rows,
+                                    rows, range(wl.n_layers), "chunk %d" % c)
+        n_cmp += cmp_c
+        n_same += same_c
         del inputs, outs, copies
         torch.cuda.empty_cache()
+    assert n_same >= 0.8 * n_cmp
