@@ -131,9 +131,24 @@ def test_single_calls_validate_arguments(lib):
                               None) == -1                                # row stride < d_qk
     assert lib.ic_sparse_attn(1, 1, 64, 1, 64, 1, 4, ic.FP8_E4M3, r, 8, 64, 64, 0.1, 1, ws.addr,
                               4096, None) == -1                          # fp8 attention
-    # empty problems are valid no-ops
-    assert lib.ic_topk(1, 12, ic.Rows(0, 8, 2, 10), 4, 1, ws.addr, 4096, None) == 0
-    assert lib.ic_topk(1, 12, ic.Rows(1, 0, 2, 10), 4, 1, ws.addr, 4096, None) == 0
+    # empty problems (no sequence, or no query row) are valid no-ops that
+    # launch nothing, with NULL data pointers too
+    before = ic.kernel_launches(0)
+    for e in (ic.Rows(0, 8, 2, 10), ic.Rows(1, 0, 2, 10), ic.Rows(0, 0, 0, 0)):
+        assert lib.ic_topk(None, 12, e, 4, None, ws.addr, 4096, None) == 0
+        assert lib.ic_indexer_scores(None, None, None, None, None, ic.BF16, e, 64, 128, None, 12,
+                                     ws.addr, 4096, None) == 0
+        assert lib.ic_sparse_attn(None, None, 576, None, 576, None, 2048, ic.BF16, e, 128, 576,
+                                  512, 0.04, None, ws.addr, 4096, None) == 0
+        assert lib.ic_sparse_attn_noalloc(None, None, None, 2048, e, 0.04, None, None, None) == 0
+        sh = ic.StackShape(e, 64, 128, ic.BF16, 2048, 128, 576, 512, ic.BF16, 576, 576, 0.04)
+        big = _FakeTensor(ic.workspace_size(sh))
+        assert ic.lib().ic_layer_stack_forward(b"FS", 2, None, ctypes.byref(sh), None, None,
+                                               big.addr, big.nbytes, None) == -1   # no layers
+        layers = (ic.LayerIO * 2)()
+        assert ic.lib().ic_layer_stack_forward(b"FS", 2, layers, ctypes.byref(sh), None, None,
+                                               big.addr, big.nbytes, None) == 0
+    assert ic.kernel_launches(0) == before
 
 
 def test_workspace_sizes_grow_with_the_problem(lib):

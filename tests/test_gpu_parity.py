@@ -161,6 +161,7 @@ def test_sparse_attention_within_tolerance(dev, dtype, Hq, d_qk, d_v, latent):
         ks, vs = d_qk, d_v
     idx = synth.random_index_sets(B, Lq, q_start, k, dev, seed=3)
     idx[0, 0, 40:] = -1            # a row with fewer valid keys than k
+    idx[1, 2, :] = -1              # a row with no valid key: zero output
     out = torch.empty(B, Lq, Hq, d_v, device=dev, dtype=torch_dt)
     scale = d_qk ** -0.5
     ws = _ws(ic.sparse_attn_workspace_size(rows, k, Hq, d_qk, d_v, DT[dtype]), dev)
@@ -185,6 +186,7 @@ def test_latent_attention_tensor_core_path(dev, rows, k):
     idx = synth.random_index_sets(B, Lq, q_start, k, dev, seed=k)
     if Lq > 1:
         idx[0, 1, 5:9] = -1                      # holes inside a row are masked
+        idx[0, 2, :] = -1                        # no valid key: the row is zero
     out = torch.empty(B, Lq, 128, 512, device=dev, dtype=torch.bfloat16)
     ws = _ws(ic.sparse_attn_workspace_size(rows, k, 128, 576, 512, ic.BF16), dev)
     n0, tc0 = ic.kernel_launches(3), ic.kernel_launches(6)
@@ -314,7 +316,9 @@ def test_exact_mode_stack_is_bit_exact_in_indices(dev):
 
 
 def test_degenerate_rows(dev):
-    """Single candidate (t = 0), k larger than the context, empty batch."""
+    """Single candidate (t = 0) with k larger than the context: the one key
+    is selected and the output is its value row.  (Empty batches are no-ops
+    that return before any device work; the CPU ABI test covers them.)"""
     wl = synth.WORKLOADS["prefill_512_fp32"]
     inputs = [synth.layer_inputs(wl, 0, dev)]
     rows = (1, 1, 0, 1)
