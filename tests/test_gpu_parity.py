@@ -1,6 +1,8 @@
 """GPU parity of each call of the C ABI against the float64 oracle, at sizes
 the oracle finishes in seconds that still span several tiles and ragged
 tails.  Full-size workloads are in test_gpu_workloads.py."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -289,6 +291,32 @@ def test_prefill_512_fp32_stack_every_row(dev, pattern):
         check_attention(host64(outs[l])[same], ref[same], "layer %d" % l)
         assert same.mean() > 0.95, same.mean()
     del differ
+
+
+@pytest.mark.parametrize("latent", [False, True])
+def test_stack_is_dense_causal_attention_when_k_covers_the_context(dev, latent):
+    """With k >= t + 1 on every row, each F layer keeps every causal key, so
+    every layer's output is ordinary dense causal attention, computed by the
+    oracle's separate dense routine (fp32 CUDA-core path; bf16 tensor-core
+    path with the latent 576-wide KV, rows starting at q_start = 40)."""
+    if latent:
+        wl = synth.Workload("dense_latent", 1, 160, 200, 40, 64, 128, 256, 128, 576, 512, "bf16",
+                            "bf16", True, "FS", 13, 1 / 8, 128 ** -0.5, 128 ** -0.5, 1.0, 1.0)
+    else:
+        wl = dataclasses.replace(synth.WORKLOADS["prefill_512_fp32"], k=512)
+    inputs = _stack_inputs(wl, dev)
+    outs, idx_copies, n_ix = _run_stack(wl, wl.pattern, inputs, dev)
+    assert n_ix == wl.pattern.count("F")
+    ol = _oracle_layers(wl, inputs)
+    t = wl.q_start + np.arange(wl.L)
+    for l in range(wl.n_layers):
+        gidx = host64(idx_copies[l])[0]
+        for i in range(wl.L):
+            assert np.array_equal(gidx[i, : t[i] + 1], np.arange(t[i] + 1))
+            assert np.all(gidx[i, t[i] + 1:] == -1)
+        ref = oracle.dense_causal_attention(ol[l]["q"], ol[l]["K"], ol[l]["V"], wl.q_start,
+                                            wl.scale)
+        check_attention(host64(outs[l]), ref, "dense identity layer %d" % l)
 
 
 def test_exact_mode_stack_is_bit_exact_in_indices(dev):
