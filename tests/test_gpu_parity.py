@@ -201,6 +201,39 @@ def test_latent_attention_tensor_core_path(dev, rows, k):
     check_attention(host64(out), ref, "latent attention")
 
 
+@pytest.mark.parametrize("latent", [False, True])
+def test_equal_key_rows_give_that_value_row(dev, latent):
+    """Every key/value row equal: whatever the softmax weights, they sum to
+    one, so every head of every row outputs that value row (fp32 CUDA-core
+    path; bf16 tensor-core path, split-k decode rows included)."""
+    if latent:
+        rows, Hq, d_qk, d_v, dt, k = (3, 2, 1998, 2000), 128, 576, 512, torch.bfloat16, 1024
+    else:
+        rows, Hq, d_qk, d_v, dt, k = (2, 5, 195, 200), 8, 64, 48, torch.float32, 64
+    B, Lq, q_start, T = rows
+    g = torch.Generator(device=dev).manual_seed(17)
+    q = torch.randn(B, Lq, Hq, d_qk, device=dev, generator=g).to(dt)
+    one = torch.randn(1, 1, d_qk if latent else d_qk + d_v, device=dev, generator=g).to(dt)
+    if latent:
+        kmat = vmat = one.expand(B, T, d_qk).contiguous()
+        ks = vs = d_qk
+        v_row = host64(one)[0, 0, :d_v]
+    else:
+        kmat = one[..., :d_qk].expand(B, T, d_qk).contiguous()
+        vmat = one[..., d_qk:].expand(B, T, d_v).contiguous()
+        ks, vs = d_qk, d_v
+        v_row = host64(one)[0, 0, d_qk:]
+    idx = synth.random_index_sets(B, Lq, q_start, k, dev, seed=17)
+    out = torch.empty(B, Lq, Hq, d_v, device=dev, dtype=dt)
+    ws = _ws(ic.sparse_attn_workspace_size(rows, k, Hq, d_qk, d_v, DT["bf16" if latent else "f32"]),
+             dev)
+    ic.sparse_attn(q, kmat, ks, vmat, vs, idx, rows, d_v, d_qk ** -0.5, out, ws)
+    torch.cuda.synchronize()
+    assert ic.read_status(ws) == 0
+    ref = np.broadcast_to(v_row, (B, Lq, Hq, d_v))
+    check_attention(host64(out), ref, "equal key rows")
+
+
 def test_attention_flags_and_skips_out_of_range_indices(dev):
     rows = (1, 4, 10, 14)
     B, Lq, q_start, T = rows
