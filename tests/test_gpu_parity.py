@@ -69,6 +69,32 @@ def test_indexer_exact_mode_is_bit_exact(dev, dtype, H_I, d_I):
             assert np.array_equal(got[b, i, : t + 1], ref[b, i, : t + 1]), (dtype, b, i)
 
 
+@pytest.mark.parametrize("dtype,H_I", [("f32", 1), ("bf16", 1), ("bf16", 16), ("e4m3", 16)])
+def test_indexer_one_effective_head_is_relu_of_the_dot_product(dev, dtype, H_I):
+    """Closed form: with w = 1 on head 0 and 0 on every other head the score
+    is max(0, q_I[head 0] . k_I) (times the two FP8 scales), written here
+    with numpy directly.  H_I = 16 runs the tensor-core kernel, H_I = 1 the
+    CUDA-core one; integer operands make the expected values exact."""
+    rows = (1, 150, 70, 220)
+    B, Lq, q_start, T = rows
+    inp = synth.exact_indexer_inputs(B, Lq, T, H_I, 128, dtype, dev, seed=31 + H_I)
+    w = torch.zeros(B, Lq, H_I, device=dev)
+    w[..., 0] = 1.0
+    inp["w"] = w
+    got = host64(_gpu_scores(inp, rows, dtype, dev))
+    if dtype == "e4m3":
+        q0 = oracle.e4m3_decode(host64(inp["q_I"]))[0, :, 0]
+        k = oracle.e4m3_decode(host64(inp["k_I"]))[0]
+        sq, sk = host64(inp["q_scale"])[0], host64(inp["k_scale"])[0]
+    else:
+        q0, k = host64(inp["q_I"])[0, :, 0], host64(inp["k_I"])[0]
+        sq, sk = np.ones(Lq), np.ones(T)
+    expect = np.maximum(q0 @ k.T, 0.0) * sq[:, None] * sk[None, :]
+    for i in range(Lq):
+        t = q_start + i
+        assert np.array_equal(got[0, i, : t + 1], expect[i, : t + 1]), (dtype, H_I, i)
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "e4m3"])
 def test_indexer_general_inputs_within_tolerance(dev, dtype):
     rows = (3, 130, 5, 140)
