@@ -226,7 +226,7 @@ topk_cand_kernel(const float* __restrict__ scores, int64_t ld, int Lq, int q_sta
     if (n <= k || s0 >= n) return;
     const int s1 = min(n, s0 + CHUNK);
     const int nch = (n + CHUNK - 1) / CHUNK;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
 
     extern __shared__ uint32_t dyn[];          // resolve: cand keys + positions, chunk counts
     __shared__ uint32_t h[HBINS];
