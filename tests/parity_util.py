@@ -54,7 +54,7 @@ def check_scores(gpu: np.ndarray, ref: np.ndarray, absum: np.ndarray, q_start: i
             g = gpu[b, r, : t + 1]
             e = ref[b, r, : t + 1]
             tol = rel * absum[b, r, : t + 1]
-            bad = np.abs(g - e) > tol
+            bad = ~(np.abs(g - e) <= tol)        # a NaN (an unwritten entry) is bad too
             if bad.any():
                 s = int(np.argmax(bad))
                 raise AssertionError("score mismatch b=%d row=%d s=%d gpu=%r ref=%r tol=%r"
@@ -93,6 +93,9 @@ def check_topk_band(idx: np.ndarray, ref_scores: np.ndarray, q_start: int, k: in
 
 
 def check_attention(gpu: np.ndarray, ref: np.ndarray, what: str = "") -> None:
+    if not np.all(np.isfinite(gpu)):
+        at = np.unravel_index(int(np.argmin(np.isfinite(gpu))), gpu.shape)
+        raise AssertionError("%s non-finite output %r at %s" % (what, gpu[at], at))
     d = np.abs(gpu - ref)
     excess = d - (ATTN_ATOL + ATTN_RTOL * np.abs(ref))
     worst = float(excess.max()) if d.size else -1.0
