@@ -5,10 +5,11 @@ where they run attention (for example an engine whose memory pool owns the
 whole GPU, or a plugin that is handed only its input and output buffers).  It
 keeps the decode split-k partials in a fixed device array inside the library
 instead of a caller workspace.  Here it is called through the C ABI twice in a
-row, on different inputs, and each result must match ic_sparse_attn (the
-entry point with a workspace) within the attention tolerance of the other
-GPU tests.  This file sorts last so that a run stopping at the first failure
-has already run every other test; it also passes when run alone.
+row, on different inputs; each result must be within the attention tolerance
+of the float64 oracle, as must ic_sparse_attn's (the entry point with a
+workspace) on the same inputs, and the two must agree with each other.  This
+file sorts last so that a run stopping at the first failure has already run
+every other test; it also passes when run alone.
 """
 import ctypes
 
@@ -16,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import cross_layer_top_full_b200 as ic
 from cross_layer_top_full_b200 import synth
 from parity_util import check_attention, host64
@@ -77,7 +79,11 @@ def test_noalloc_matches_workspace_entry_point_twice(dev, rows, k):
         got, status = _noalloc(q, kv, idx, rows, scale, dev)
         torch.cuda.synchronize()
         assert int(status.item()) == 0, call
-        check_attention(host64(got), host64(ref), "no-alloc call %d" % call)
+        kvh = host64(kv)
+        want = oracle.sparse_attention(host64(q), kvh, kvh[..., :512], host64(idx), scale)
+        check_attention(host64(got), want, "no-alloc call %d vs oracle" % call)
+        check_attention(host64(ref), want, "workspace call %d vs oracle" % call)
+        check_attention(host64(got), host64(ref), "no-alloc call %d vs workspace" % call)
 
 
 def test_noalloc_rejects_problems_beyond_its_fixed_array(dev):
