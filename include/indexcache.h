@@ -53,7 +53,7 @@ typedef enum {
     IC_ERR_UNSUPPORTED = -3,  /* dtype / shape combination not implemented          */
     IC_ERR_WORKSPACE = -4,    /* ws too small or misaligned                         */
     IC_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed                */
-    IC_ERR_INDEX_RANGE = -6,  /* (device) an index was outside [0, t]; row skipped   */
+    IC_ERR_INDEX_RANGE = -6,  /* (device) an index was outside [0, t] and skipped   */
     IC_ERR_TIMEOUT = -7       /* (device) a pipeline wait ran out of time            */
 } ic_status;
 
