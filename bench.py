@@ -303,22 +303,65 @@ def cpu_model():
     return platform.processor() or "unknown"
 
 
-def cpu_baseline(wl, pattern, value, done, spent, how):
+def cpu_baseline(wl, pattern, value, done, spent, how, clock=None):
     """The cpu_baseline object: the float64 oracle's rate on a bounded
-    sample (`how` says how the query rows were drawn)."""
+    sample (`how` says how the query rows were drawn), and with `clock` its
+    time per query row in each stage (per F layer for the indexer and
+    top-k, per layer for attention) at the sampled rows' positions."""
     lay = oracle_layers(wl, pattern)
     if lay == pattern:
         layers, note = "all %d layers of %s" % (len(pattern), pattern), ""
     else:
         layers = "the first %d of the %d layers of %s" % (len(lay), len(pattern), pattern)
         note = "; rate scaled to all layers"
-    return {"value": value, "unit": "tok/s", "cores": _blas_threads(), "kind": "oracle",
-            "cpu_model": cpu_model(),
-            "sample": "%d %s of %s through %s (float64 NumPy, %.1f s of oracle time%s)"
-                      % (done, how, wl.name, layers, spent, note)}
+    res = {"value": value, "unit": "tok/s", "cores": _blas_threads(), "kind": "oracle",
+           "cpu_model": cpu_model(),
+           "sample": "%d %s of %s through %s (float64 NumPy, %.1f s of oracle time%s)"
+                     % (done, how, wl.name, layers, spent, note)}
+    if clock is not None:
+        res["per_row_ms"] = clock.per_row_ms()
+    return res
 
 
-def oracle_sample(wl, pattern, budget_s):
+class OracleStageClock:
+    """Adds up the time the oracle spends in each stage function while its
+    layer_stack runs, and the query rows each stage handled.  The module's
+    functions are wrapped for the duration of the `with` block and restored
+    afterwards; the oracle's arithmetic is untouched."""
+    STAGES = {"indexer": "indexer_scores", "topk": "topk_indices", "attention": "sparse_attention"}
+
+    def __init__(self):
+        import oracle.indexcache_oracle as om
+        self.mod = om
+        self.seconds = dict.fromkeys(self.STAGES, 0.0)
+        self.rows = dict.fromkeys(self.STAGES, 0)
+
+    def __enter__(self):
+        self.saved = {st: getattr(self.mod, fn) for st, fn in self.STAGES.items()}
+        for st, fn in self.STAGES.items():
+            setattr(self.mod, fn, self._timed(st, self.saved[st]))
+        return self
+
+    def __exit__(self, *exc):
+        for st, fn in self.STAGES.items():
+            setattr(self.mod, fn, self.saved[st])
+        return False
+
+    def _timed(self, stage, fn):
+        def run(*args, **kw):
+            t0 = time.perf_counter()
+            res = fn(*args, **kw)
+            self.seconds[stage] += time.perf_counter() - t0
+            self.rows[stage] += res.shape[0] * res.shape[1]      # [B, rows, ...]
+            return res
+        return run
+
+    def per_row_ms(self):
+        return {st: (1e3 * self.seconds[st] / self.rows[st] if self.rows[st] else None)
+                for st in self.STAGES}
+
+
+def oracle_sample(wl, pattern, budget_s, clock=None):
     """Time the float64 oracle (as it stands) on a bounded sample of the
     workload: prefill -> blocks of consecutive query rows at random offsets of
     one sequence; decode -> whole sequences, one at a time.  Inputs are drawn
@@ -350,8 +393,13 @@ def oracle_sample(wl, pattern, budget_s):
                 dec_inputs = _oracle_inputs(sub)
             inputs = dec_inputs
         t0 = time.perf_counter()
-        oracle.layer_stack(sub.pattern, inputs, sub.q_start, sub.k, sub.scale,
-                           fp8=sub.idx_dtype == "e4m3")
+        if clock is None:
+            oracle.layer_stack(sub.pattern, inputs, sub.q_start, sub.k, sub.scale,
+                               fp8=sub.idx_dtype == "e4m3")
+        else:
+            with clock:
+                oracle.layer_stack(sub.pattern, inputs, sub.q_start, sub.k, sub.scale,
+                                   fp8=sub.idx_dtype == "e4m3")
         dt = time.perf_counter() - t0
         done += sub.B * sub.L
         spent += dt
@@ -500,9 +548,10 @@ def main():
         return
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        rps, done, spent = oracle_sample(wl, pattern, args.cpu_budget)
+        clock = OracleStageClock()
+        rps, done, spent = oracle_sample(wl, pattern, args.cpu_budget, clock)
         cpu = cpu_baseline(wl, pattern, rps, done, spent,
-                           "query rows" if wl.L > 1 else "single-sequence decode steps")
+                           "query rows" if wl.L > 1 else "single-sequence decode steps", clock)
     line = {
         "metric": "prefill tok/s (IndexCache pattern) with all-F comparison; roofline of the "
                   "dominant kernel" if wl.L > 1 else "decode tok/s (IndexCache pattern)",
@@ -704,8 +753,10 @@ def run_chunked(args, wl, pattern, dev, pg, rank, world):
         return
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        rps, done, spent = oracle_sample(wl, pattern, args.cpu_budget)
-        cpu = cpu_baseline(wl, pattern, rps, done, spent, "query rows at random positions")
+        clock = OracleStageClock()
+        rps, done, spent = oracle_sample(wl, pattern, args.cpu_budget, clock)
+        cpu = cpu_baseline(wl, pattern, rps, done, spent, "query rows at random positions",
+                           clock)
     per_step_ms = ms / args.steps
     avg = {k: float(np.mean(v)) for k, v in stages.items()}
     line = {
@@ -810,8 +861,9 @@ def run_reference(args, wl, pattern, rank, world):
     for _ in range(args.warmup):
         oracle_sample(wl, pattern, budget / 4)
     rates, done_all, spent_all = [], 0, 0.0
+    clock = OracleStageClock()
     for _ in range(args.steps):
-        rps, done, spent = oracle_sample(wl, pattern, budget)
+        rps, done, spent = oracle_sample(wl, pattern, budget, clock)
         rates.append(rps)
         done_all += done
         spent_all += spent
@@ -826,7 +878,8 @@ def run_reference(args, wl, pattern, rank, world):
         "config": {"workload": wl.name, "pattern": pattern, "B": wl.B, "L": wl.L, "T": wl.T,
                    "k": wl.k},
         "cpu_baseline": cpu_baseline(wl, pattern, value, done_all, spent_all,
-                                     "query rows" if wl.L > 1 else "single-sequence decode steps"),
+                                     "query rows" if wl.L > 1 else "single-sequence decode steps",
+                                     clock),
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

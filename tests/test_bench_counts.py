@@ -115,3 +115,21 @@ def test_cpu_baseline_says_which_layers_the_oracle_timed(name, timed):
         assert "first %d of the %d layers" % (timed, len(wl.pattern)) in cb["sample"]
     else:
         assert "all %d layers" % timed in cb["sample"]
+
+
+def test_oracle_stage_clock_times_each_stage_and_restores_the_oracle():
+    import oracle.indexcache_oracle as om
+    before = (om.indexer_scores, om.topk_indices, om.sparse_attention)
+    wl = synth.WORKLOADS["prefill_512_fp32"]
+    clock = bench.OracleStageClock()
+    rate, done, spent = bench.oracle_sample(wl, wl.pattern, 0.3, clock)
+    assert (om.indexer_scores, om.topk_indices, om.sparse_attention) == before
+    assert rate > 0 and done > 0
+    # FSSS: one indexer and top-k pass per row, four attention passes
+    assert clock.rows["indexer"] == clock.rows["topk"] == done
+    assert clock.rows["attention"] == 4 * done
+    per_row = clock.per_row_ms()
+    assert all(per_row[s] > 0 for s in ("indexer", "topk", "attention"))
+    assert sum(clock.seconds.values()) <= spent
+    cb = bench.cpu_baseline(wl, wl.pattern, rate, done, spent, "query rows", clock)
+    assert cb["per_row_ms"] == per_row
