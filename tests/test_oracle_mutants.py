@@ -14,8 +14,6 @@ import shutil
 import subprocess
 import sys
 
-import pytest
-
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "indexcache_oracle.py")
 PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")

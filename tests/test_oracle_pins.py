@@ -6,7 +6,6 @@ library routine, so that a plausible slip in the oracle (a dropped ReLU, a
 wrong sign, an off-by-one causal bound, a reversed tie-break, a transposed
 operand, a missing scale) fails at least one of them.
 """
-import itertools
 import json
 import math
 import os

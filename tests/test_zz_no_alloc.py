@@ -13,7 +13,6 @@ every other test; it also passes when run alone.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
