@@ -15,6 +15,8 @@ reading notes in each entry):
 * ``prefill_8k_bf16``      1 sequence, L=8192, FSSS, H_I=64, d_I=128, k=2048;
   MQA with 128 heads over one latent KV row of width 576 (V = its first 512
   columns); bf16 activations.
+* ``prefill_8k_fp8``       the same with the indexer operands as E4M3 codes
+  and one float32 scale per token (the FP8 prefill indexer).
 * ``decode_b32_t32k_bf16`` 32 sequences x 32768 cached keys, one new query
   each, pattern FSSSFSSS; caches N(0,1)/sqrt(d) with 16 heavy-hitter
   positions per sequence scaled x4.
@@ -85,6 +87,14 @@ WORKLOADS: Dict[str, Workload] = {
     "prefill_8k_bf16": Workload(
         "prefill_8k_bf16", B=1, L=8192, T=8192, q_start=0, H_I=64, d_I=128, k=2048,
         Hq=128, d_qk=576, d_v=512, idx_dtype="bf16", attn_dtype="bf16", latent=True,
+        pattern="FSSS", seed=1, w_std=1 / 8, qI_std=1 / math.sqrt(128),
+        kI_std=1 / math.sqrt(128), q_std=1.0, kv_std=1.0),
+    # the prefill workload with the indexer operands in E4M3 (one float32
+    # scale per token), the FP8 prefill indexer; same seed, so its q_I / k_I
+    # are the bf16 workload's values before quantisation
+    "prefill_8k_fp8": Workload(
+        "prefill_8k_fp8", B=1, L=8192, T=8192, q_start=0, H_I=64, d_I=128, k=2048,
+        Hq=128, d_qk=576, d_v=512, idx_dtype="e4m3", attn_dtype="bf16", latent=True,
         pattern="FSSS", seed=1, w_std=1 / 8, qI_std=1 / math.sqrt(128),
         kI_std=1 / math.sqrt(128), q_std=1.0, kv_std=1.0),
     # decode q / q_I / w follow the prefill workload (only the caches are
