@@ -124,23 +124,3 @@ def test_chunked_prefill_64k_bf16_every_chunk(dev):
         torch.cuda.empty_cache()
     assert n_same >= 0.8 * n_cmp
 
-
-# --------------------------------------------------------------------------- prefill 8k, FP8 indexer
-def test_prefill_8k_fp8_indexer_full_size(dev):
-    """The 8K prefill with the indexer operands in E4M3 (one scale per token):
-    the prefill-shaped FP8 tensor-core indexer at full size.  Indices of 512
-    seeded rows (always 0, 1, k-1, k, k+1, L-1); attention on 128 of them,
-    all 4 layers."""
-    wl = synth.WORKLOADS["prefill_8k_fp8"]
-    inputs = [synth.layer_inputs(wl, l, dev) for l in range(wl.n_layers)]
-    outs, copies, n_ix = run_stack(wl, wl.pattern, inputs, (wl.B, wl.L, 0, wl.T), dev)
-    assert n_ix == wl.pattern.count("F")
-    always = (0, 1, wl.k - 1, wl.k, wl.k + 1, wl.L - 1)
-    idx_rows = sample_rows(wl.L, 512, seed=7, always=always)
-    attn_rows = sample_rows(len(idx_rows), 122, seed=8)
-    attn_rows = sorted(set([idx_rows[j] for j in attn_rows]) | set(always))
-    n_cmp, n_same = check_stack(wl, wl.pattern, inputs, copies, outs, 0, [0], idx_rows,
-                                attn_rows, range(wl.n_layers), "prefill_8k_fp8")
-    assert n_same >= 0.5 * n_cmp
-    del inputs, outs, copies
-    torch.cuda.empty_cache()
