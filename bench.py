@@ -185,36 +185,58 @@ def algorithmic(wl):
     return d
 
 
-def roofline(wl, work, total_ms, launches, per_pass=1):
+def stage_bound(wl, work, stage):
+    """(tensor-bound?, algorithmic work of one pass) of a stage: flops for the
+    prefill indexer and the bf16 prefill attention (tensor cores), bytes
+    otherwise (HBM)."""
+    if stage == "attention":
+        tensor = wl.attn_dtype == "bf16" and wl.L > 1
+        return tensor, work["attn_flop"] if tensor else work["attn_bytes"]
+    if stage == "indexer":
+        tensor = wl.L > 1
+        return tensor, work["indexer_flop"] if tensor else work["indexer_bytes"]
+    return False, work["topk_bytes"]
+
+
+def _roof(num, per_pass_ms, tensor, fp8, peak):
+    hbm, tf_burst, tf_sus, peak_src = _peaks()
+    if tensor:
+        p = tf_sus if peak == "sustained" else tf_burst
+        if fp8:
+            p *= 2.0                               # e4m3 dense peak: 2x the bf16 figure
+        roof = {"bound": "tensor", "achieved": num / (per_pass_ms * 1e-3) / 1e12, "peak": p,
+                "unit": "TFLOP/s"}
+        roof["peak_source"] = "%s (%s %s)" % (peak_src, peak, "bf16 x2 for e4m3" if fp8 else "bf16")
+    else:
+        roof = {"bound": "hbm", "achieved": num / (per_pass_ms * 1e-3) / 1e9, "peak": hbm,
+                "unit": "GB/s", "peak_source": "%s (copy bandwidth)" % peak_src}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    return roof
+
+
+def stage_roofline(wl, work, stage, per_launch_ms, peak="burst", per_pass=1):
+    """Roofline of one stage from its mean time per launch."""
+    tensor, num = stage_bound(wl, work, stage)
+    fp8 = stage == "indexer" and wl.idx_dtype == "e4m3"
+    roof = _roof(num, per_launch_ms * per_pass, tensor, fp8, peak)
+    roof["ms_per_launch"] = per_launch_ms
+    return roof
+
+
+def roofline(wl, work, total_ms, launches, per_pass=1, peak="sustained"):
     """Roofline line of the dominant stage.  total_ms / launches: summed
     event time and launch count per stage over the measured passes; work:
     algorithmic work of one pass of a stage over all rows (``algorithmic``;
     summed over the chunks of a chunked run), which takes ``per_pass``
-    launches."""
-    hbm, tf_burst, tf_sus, peak_src = _peaks()
+    launches.  ``peak``: "burst" or "sustained" bf16 figure."""
     dom = max(total_ms, key=lambda k: total_ms[k])
     passes = launches[dom] / per_pass
     per_pass_ms = total_ms[dom] / passes
-    if dom == "attention":
-        tensor = wl.attn_dtype == "bf16" and wl.L > 1
-        num = work["attn_flop"] if tensor else work["attn_bytes"]
-    elif dom == "indexer":
-        tensor = wl.L > 1
-        num = work["indexer_flop"] if tensor else work["indexer_bytes"]
-    else:
-        tensor = False
-        num = work["topk_bytes"]
-    if tensor:
-        roof = {"bound": "tensor", "achieved": num / (per_pass_ms * 1e-3) / 1e12, "peak": tf_sus,
-                "unit": "TFLOP/s"}
-    else:
-        roof = {"bound": "hbm", "achieved": num / (per_pass_ms * 1e-3) / 1e9, "peak": hbm,
-                "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
+    tensor, num = stage_bound(wl, work, dom)
+    fp8 = dom == "indexer" and wl.idx_dtype == "e4m3"
+    roof = _roof(num, per_pass_ms, tensor, fp8, peak)
     roof["kernel"] = dom
     roof["ms_per_launch"] = total_ms[dom] / launches[dom]
-    roof["peak_source"] = "%s (%s)" % (peak_src, "sustained bf16" if roof["unit"] == "TFLOP/s"
-                                       else "copy bandwidth")
     return roof, dom
 
 
@@ -430,6 +452,9 @@ def _oracle_inputs(wl):
 
 
 # ----------------------------------------------------------------------------- main
+DEFAULT_DECODE = (("decode_b32_t32k_bf16", 500), ("decode_b8_t200k_fp8", 150))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -440,6 +465,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="time only --workload (the default run also times the decode workloads)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--graph", action="store_true",
                     help="replay each step as a captured CUDA graph (decode: removes launch gaps)")
@@ -450,7 +477,6 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     wl = synth.WORKLOADS[args.workload]
     pattern = args.pattern or wl.pattern
-    tokens_per_step = wl.B * wl.L
 
     if args.impl == "reference":
         return run_reference(args, wl, pattern, rank, world)
@@ -467,28 +493,94 @@ def main():
 
     if wl.chunk:
         return run_chunked(args, wl, pattern, dev, pg, rank, world)
+    line = measure_stack(wl, pattern, dev, pg, rank, world, steps=args.steps,
+                         warmup=args.warmup, graph=args.graph or wl.L == 1,
+                         e2e=not args.no_e2e,
+                         cpu_budget=None if args.no_cpu_baseline else args.cpu_budget)
+    # the default run: the decode half of the metric (decode step us, IndexCache
+    # pattern vs all-F) on the two decode workloads, CUDA-graph replay
+    if args.workload == "prefill_8k_bf16" and args.pattern is None and not args.no_decode:
+        line["decode"] = {}
+        for name, dsteps in DEFAULT_DECODE:
+            dwl = synth.WORKLOADS[name]
+            entry = measure_stack(dwl, dwl.pattern, dev, pg, rank, world,
+                                  steps=max(args.steps, dsteps), warmup=args.warmup, graph=True,
+                                  e2e=not args.no_e2e,
+                                  cpu_budget=None if args.no_cpu_baseline else args.cpu_budget / 2)
+            line["decode"][name] = decode_entry(entry)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    _finish(pg)
+
+
+def decode_entry(line):
+    """The decode workload's measurement as an entry of the default line:
+    step time in microseconds for the IndexCache pattern and for all-F."""
+    return {
+        "metric": "decode step us (IndexCache pattern) vs all-F",
+        "step_us": line["ms_per_step"] * 1e3,
+        "all_f_step_us": line["all_f"]["ms_per_step"] * 1e3,
+        "speedup_of_pattern": line["all_f"]["speedup_of_pattern"],
+        "value": line["value"], "unit": line["unit"], "steps": line["steps"],
+        "config": line["config"], "stages_us": {
+            k: {"per_launch": v["per_launch"] * 1e3, "launches_per_step": v["launches_per_step"]}
+            for k, v in line["stages_ms"].items()},
+        "roofline_by_stage": line["roofline_by_stage"],
+        "indexer_share_of_step": line["indexer_share_of_step"],
+        "cpu_baseline": line["cpu_baseline"], "e2e": line["e2e"],
+        "gpu_launches": line["gpu_launches"], "cuda_graph": line["cuda_graph"],
+        "clocks": line["clocks"], "device_status": line["device_status"],
+    }
+
+
+def require_clean(ws, what):
+    """Read (and clear) the device status word of a workspace after a timed
+    region; a kernel that flagged an index error or gave up a bounded wait
+    voids the measurement."""
+    bits = ic.read_status(ws)
+    if bits:
+        raise SystemExit("%s: device status bits %d set (1 = index out of range, "
+                         "2 = wait timeout); the measurement is void" % (what, bits))
+    return bits
+
+
+def peak_kind(clk):
+    """The bf16 peak to divide by: the sustained (power-capped) figure when
+    the run itself was power-capped or ran well below its maximum clock,
+    else the burst figure."""
+    if clk and ("sw_power_cap" in clk["reasons"] or clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"]):
+        return "sustained"
+    return "burst"
+
+
+def measure_stack(wl, pattern, dev, pg, rank, world, *, steps, warmup, graph, e2e, cpu_budget):
+    """Time one workload's layer stack (IndexCache pattern and all-F) and
+    return its JSON line (as a dict)."""
+    import gc
+    tokens_per_step = wl.B * wl.L
     st = Stack(wl, dev, rank)
     all_f = "F" * len(pattern)
 
-    def timed(fn, steps):
+    def timed(fn, n):
         if pg:
             pg.barrier()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        for _ in range(steps):
+        for _ in range(n):
             fn()
         b.record()
         torch.cuda.synchronize()
         return max_over_ranks(a.elapsed_time(b), pg, dev)
 
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         st.step(pattern)
         st.step(all_f)
     torch.cuda.synchronize()
+    require_clean(st.ws, "%s warm-up" % wl.name)
     step_fn, step_all_f = (lambda: st.step(pattern)), (lambda: st.step(all_f))
     graphs = []
-    if args.graph:
+    if graph:
         for pat in (pattern, all_f):
             g = torch.cuda.CUDAGraph()
             s_cap = torch.cuda.Stream()
@@ -507,75 +599,87 @@ def main():
         torch.cuda.synchronize()
 
     # main timed region: the IndexCache pattern through the C ABI
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev.index or 0)
     clocks.start()
     n0 = ic.kernel_launches(0)
-    ms = timed(step_fn, args.steps)
+    ms = timed(step_fn, steps)
     launches = ic.kernel_launches(0) - n0
-    if args.graph:   # replays launch the captured kernels: count them per step
+    if graph:   # replays launch the captured kernels: count them per step
+        torch.cuda.synchronize()
         n1 = ic.kernel_launches(0)
         st.step(pattern)
-        launches = (ic.kernel_launches(0) - n1) * args.steps
+        launches = (ic.kernel_launches(0) - n1) * steps
         torch.cuda.synchronize()
-    ms_all_f = timed(step_all_f, args.steps)
+    status = require_clean(st.ws, "%s IndexCache steps" % wl.name)
+    ms_all_f = timed(step_all_f, steps)
     clk = clocks.stop()
+    require_clean(st.ws, "%s all-F steps" % wl.name)
+    del graphs, step_fn, step_all_f
 
     # stage breakdown (same kernels as separate calls, events on the launch stream)
     ev = Events()
-    for _ in range(args.steps):
+    stage_passes = min(steps, 20)
+    for _ in range(stage_passes):
         st.stage_step(pattern, ev)
     stages = ev.collect()
+    require_clean(st.ws, "%s stage pass" % wl.name)
 
     # end to end from pinned host buffers through the public API
-    e2e = None
-    if not args.no_e2e:
-        e2e = run_e2e(st, pattern, args.steps, dev, pg)
+    e2e_line = None
+    if e2e:
+        e2e_line = run_e2e(st, pattern, min(steps, 50 if wl.L == 1 else steps), dev, pg)
+        require_clean(st.ws, "%s e2e" % wl.name)
 
-    per_step_ms = ms / args.steps
+    per_step_ms = ms / steps
     value = whole_job_rate(tokens_per_step, world, per_step_ms)
     work = algorithmic(wl)
     avg = {k: float(np.mean(v)) for k, v in stages.items()}
-    roof, dom = roofline(wl, work, {k: sum(v) for k, v in stages.items()},
-                         {k: len(v) for k, v in stages.items()})
-    roof["traffic"] = _traffic(dom, args.workload)
-    # decode: share of the step spent choosing keys (indexer + top-k)
-    total_stage = sum(sum(v) for v in stages.values())
-    sel_share = (sum(stages.get("indexer", [])) + sum(stages.get("topk", []))) / total_stage
+    kind = peak_kind(clk)
+    totals = {k: sum(v) for k, v in stages.items()}
+    counts = {k: len(v) for k, v in stages.items()}
+    roof, dom = roofline(wl, work, totals, counts, peak=kind)
+    roof["traffic"] = _traffic(dom, wl.name)
+    by_stage = {k: stage_roofline(wl, work, k, avg[k], kind) for k in stages}
+    # share of the step spent choosing keys (indexer + top-k)
+    total_stage = sum(totals.values())
+    sel_share = (totals.get("indexer", 0.0) + totals.get("topk", 0.0)) / total_stage
+    bytes_in = st.bytes_per_step(pattern)
+    del st
+    gc.collect()
+    torch.cuda.empty_cache()
 
-    if rank != 0:
-        _finish(pg)
-        return
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and cpu_budget:
         clock = OracleStageClock()
-        rps, done, spent = oracle_sample(wl, pattern, args.cpu_budget, clock)
+        rps, done, spent = oracle_sample(wl, pattern, cpu_budget, clock)
         cpu = cpu_baseline(wl, pattern, rps, done, spent,
                            "query rows" if wl.L > 1 else "single-sequence decode steps", clock)
-    line = {
+    return {
         "metric": "prefill tok/s (IndexCache pattern) with all-F comparison; roofline of the "
                   "dominant kernel" if wl.L > 1 else "decode tok/s (IndexCache pattern)",
-        "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": per_step_ms, "higher_is_better": True,
+        "value": value, "unit": "tok/s", "n_gpus": world, "steps": steps,
+        "warmup": max(3, warmup), "ms_per_step": per_step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.attn_dtype, "data": "synthetic",
         "config": {"workload": wl.name, "pattern": pattern, "B": wl.B, "L": wl.L, "T": wl.T,
                    "H_I": wl.H_I, "d_I": wl.d_I, "k": wl.k, "Hq": wl.Hq, "d_qk": wl.d_qk,
-                   "d_v": wl.d_v, "indexer_dtype": wl.idx_dtype, "parallelism": "replicas x%d" % world,
-                   "l2": "inputs larger than L2 (%.2f GB read per step)" % (st.bytes_per_step(pattern) / 1e9)},
-        "all_f": {"pattern": all_f, "ms_per_step": ms_all_f / args.steps,
-                  "value": tokens_per_step * world / (ms_all_f / args.steps / 1e3),
+                   "d_v": wl.d_v, "indexer_dtype": wl.idx_dtype,
+                   "parallelism": "replicas x%d" % world,
+                   "l2": "inputs larger than L2 (%.2f GB read per step)" % (bytes_in / 1e9)},
+        "all_f": {"pattern": all_f, "ms_per_step": ms_all_f / steps,
+                  "value": tokens_per_step * world / (ms_all_f / steps / 1e3),
                   "speedup_of_pattern": ms_all_f / ms},
-        "stages_ms": {k: {"per_launch": avg[k], "launches_per_step": len(v) / args.steps}
+        "stages_ms": {k: {"per_launch": avg[k], "launches_per_step": len(v) / stage_passes}
                       for k, v in stages.items()},
         "indexer_share_of_step": sel_share,
         "roofline": roof,
+        "roofline_by_stage": by_stage,
         "cpu_baseline": cpu,
-        "e2e": e2e,
+        "e2e": e2e_line,
         "gpu_launches": launches,
-        "cuda_graph": bool(args.graph),
+        "cuda_graph": bool(graph),
         "clocks": clk,
+        "device_status": status,
     }
-    print(json.dumps(line), flush=True)
-    _finish(pg)
 
 
 def row_overlap(reused, own, T):
@@ -804,10 +908,14 @@ CACHE_KEYS = ("kv", "k", "v", "k_I", "k_scale")
 
 def run_e2e(st, pattern, steps, dev, pg):
     """Same metric through the public API from pinned host buffers: every step
-    copies that step's inputs host->device, runs the stack and reads the last
-    layer's output back.  Prefill copies every input of the step.  Decode keeps
-    the KV / K_I caches resident on the device (serving state) and copies the
-    new token's queries, weights and its own cache rows (position T-1)."""
+    copies that step's inputs host->device, runs the stack through
+    ic_layer_stack_forward and copies EVERY layer's output back to pinned
+    host memory (each layer is an independent synthetic layer, so all of
+    them are the step's result).  Prefill copies every input of the step.
+    Decode keeps the KV / K_I caches resident on the device (serving state)
+    and copies the new token's queries, weights and its own cache rows
+    (position T-1).  The copies are torch copy_ calls on the launch stream
+    around the C-ABI call."""
     wl = st.wl
     decode = wl.L == 1
     host = []
@@ -822,8 +930,8 @@ def run_e2e(st, pattern, steps, dev, pg):
             d[key].copy_(src)
             h2d += src.numel() * src.element_size()
         host.append(d)
-    out_host = torch.empty(st.outs[-1].shape, dtype=st.outs[-1].dtype, pin_memory=True)
-    d2h = out_host.numel() * out_host.element_size()
+    outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in st.outs]
+    d2h = sum(o.numel() * o.element_size() for o in outs_host)
 
     def step():
         for l, d in enumerate(host):
@@ -833,7 +941,8 @@ def run_e2e(st, pattern, steps, dev, pg):
                 else:
                     st.inputs[l][key].copy_(t, non_blocking=True)
         st.step(pattern)
-        out_host.copy_(st.outs[-1], non_blocking=True)
+        for o_h, o in zip(outs_host, st.outs):
+            o_h.copy_(o, non_blocking=True)
 
     step()
     torch.cuda.synchronize()
@@ -847,10 +956,11 @@ def run_e2e(st, pattern, steps, dev, pg):
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b), pg, dev)
     world = pg.get_world_size() if pg else 1
-    wl = st.wl
-    del host
+    del host, outs_host
     return {"value": wl.B * wl.L * world / (ms / steps / 1e3), "unit": "tok/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "copies": "torch copy_ from/to pinned host memory on the launch stream, around "
+                      "ic_layer_stack_forward; every layer's output is read back"}
 
 
 def run_reference(args, wl, pattern, rank, world):
@@ -872,7 +982,13 @@ def run_reference(args, wl, pattern, rank, world):
         "metric": "prefill tok/s (IndexCache pattern) with all-F comparison; roofline of the "
                   "dominant kernel" if wl.L > 1 else "decode tok/s (IndexCache pattern)",
         "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1e3 * wl.B * wl.L / value, "higher_is_better": True,
+        # a reference step is one bounded sample of the workload (its rows are
+        # timed, not the whole step's); ms_per_step is that sample's wall time
+        "warmup": args.warmup, "ms_per_step": 1e3 * spent_all / max(1, args.steps),
+        "ms_per_full_step_extrapolated": 1e3 * wl.B * wl.L / value,
+        "step_definition": "one bounded oracle sample of the workload per step; the full "
+                           "step's time is extrapolated from the sampled rows' rate",
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "pattern": pattern, "B": wl.B, "L": wl.L, "T": wl.T,
                    "k": wl.k},

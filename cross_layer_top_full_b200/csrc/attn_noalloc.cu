@@ -16,6 +16,8 @@
 // at its start is cleared at the beginning of every call, and the partials
 // are always written before they are read.  Two calls whose kernels overlap on
 // the GPU (different streams, or different host threads) race on the array.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -24,26 +26,58 @@ namespace ic {
 namespace {
 
 constexpr size_t kStatusBytes = 256;
+// split-k units (query rows x splits) whose partials fit in the array
+constexpr int64_t kMaxUnits = 64;
 
 // status word (first 256 bytes) followed by the split-k partials
 static __device__ __align__(256) unsigned char g_noalloc_scratch[IC_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
-void* g_scratch_addr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+struct ScratchAddr {
+    void* ctx;    // the CUDA context the address was looked up in
+    void* addr;   // device address of g_noalloc_scratch in that context
+};
+ScratchAddr g_scratch_addr[kMaxDevices];
 
-// Device address of the scratch array on the current device (looked up once
-// per device, with that device current).  Returns nullptr on failure.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
+// Device address of the scratch array in the current device's current
+// context.  Looked up with cudaGetSymbolAddress on the first call on each
+// device, with that device current, and again whenever that device's
+// context has changed since (for example after a cudaDeviceReset, which
+// frees the old address).  Returns nullptr on failure.
 void* scratch_address() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    CtxGetCurrentFn get = ctx_get_current();
+    if (get == nullptr) return nullptr;
+    CUcontext ctx = nullptr;
+    if (get(&ctx) != CUDA_SUCCESS) return nullptr;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (g_scratch_addr[dev] == nullptr) {
+    ScratchAddr& e = g_scratch_addr[dev];
+    if (ctx == nullptr || e.addr == nullptr || e.ctx != (void*)ctx) {
+        // binds the device's primary context first when none is current yet
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-        g_scratch_addr[dev] = p;
+        if (get(&ctx) != CUDA_SUCCESS || ctx == nullptr) return nullptr;
+        e.ctx = (void*)ctx;
+        e.addr = p;
     }
-    return g_scratch_addr[dev];
+    return e.addr;
 }
 
 }  // namespace
@@ -59,7 +93,11 @@ extern "C" ic_status ic_sparse_attn_noalloc(const void* q, const void* kv, const
     if (k < 1 || k > 16384) return IC_ERR_INVALID_ARG;
     if (r.B == 0 || r.Lq == 0) return IC_OK;
     if (!q || !kv || !idx || !out) return IC_ERR_INVALID_ARG;
-    const size_t need = attn_tc_scratch_bytes(r, k);
+    // rows that split their keys need partials in the array: plan at most
+    // kMaxUnits units (rows x splits); only when even the fewest splits a row
+    // can have (ceil(k / 2048)) leave more units is the call refused
+    const size_t need = attn_tc_scratch_bytes(r, k, kMaxUnits);
+    if (need > 0 && attn_tc_units(r, k, kMaxUnits) > kMaxUnits) return IC_ERR_WORKSPACE;
     if (need > IC_NOALLOC_SCRATCH_BYTES - kStatusBytes) return IC_ERR_WORKSPACE;
     char* base = static_cast<char*>(scratch_address());
     if (base == nullptr) return cuda_error("attn_noalloc");
@@ -67,7 +105,7 @@ extern "C" ic_status ic_sparse_attn_noalloc(const void* q, const void* kv, const
     uint32_t* status = reinterpret_cast<uint32_t*>(base);
     if (cudaMemsetAsync(status, 0, sizeof(uint32_t), s) != cudaSuccess) return cuda_error("attn_noalloc");
     ic_status st = launch_attn_tc(q, kv, 576, idx, k, r, scale, out, status, base + kStatusBytes,
-                                  IC_NOALLOC_SCRATCH_BYTES - kStatusBytes, s);
+                                  IC_NOALLOC_SCRATCH_BYTES - kStatusBytes, s, kMaxUnits);
     if (st != IC_OK) return st;
     if (device_status != nullptr &&
         cudaMemcpyAsync(device_status, status, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) !=

@@ -786,7 +786,11 @@ int sm_count() {
 
 // Split-k plan: number of splits of the k indices per query row.  A unit
 // (one split of one row) holds at most MAX_UNIT_BLOCKS blocks of indices.
-void plan_splits(const ic_rows& r, int k, int& splits, int& keys_per_split) {
+// The split count minimises (waves of CTA pairs) x (blocks per split + a
+// fixed cost per unit) among the counts whose units (rows x splits) do not
+// pass max_units; the smallest admissible count is always kept, so the
+// caller checks rows x splits against its own limit.
+void plan_splits(const ic_rows& r, int k, int& splits, int& keys_per_split, int64_t max_units) {
     const int64_t rows = (int64_t)r.B * r.Lq;
     const int pairs = std::max(1, sm_count() / 2);
     const int nblk = ceil_div(k, NB);
@@ -795,6 +799,7 @@ void plan_splits(const ic_rows& r, int k, int& splits, int& keys_per_split) {
     if (rows < pairs) {
         double best = 1e30;
         for (int s = min_splits; s <= std::max(min_splits, std::min(nblk, 32)); ++s) {
+            if (s > min_splits && rows * s > max_units) break;
             const double waves = (double)ceil_div64(rows * s, pairs);
             const double cost = waves * (ceil_div(nblk, s) + 1.5);
             if (cost < best - 1e-9) {
@@ -815,9 +820,15 @@ bool attn_tc_supported(const void* kmat, const void* vmat, int64_t ks, int64_t v
            vs == KVW;
 }
 
-size_t attn_tc_scratch_bytes(ic_rows r, int k) {
+int64_t attn_tc_units(ic_rows r, int k, int64_t max_units) {
     int splits, kps;
-    plan_splits(r, k, splits, kps);
+    plan_splits(r, k, splits, kps, max_units);
+    return (int64_t)r.B * r.Lq * splits;
+}
+
+size_t attn_tc_scratch_bytes(ic_rows r, int k, int64_t max_units) {
+    int splits, kps;
+    plan_splits(r, k, splits, kps, max_units);
     if (splits <= 1) return 0;
     const size_t units = (size_t)r.B * r.Lq * splits;
     return units * HQ * DV * sizeof(float) + 256 + units * HQ * sizeof(float2);
@@ -825,7 +836,7 @@ size_t attn_tc_scratch_bytes(ic_rows r, int k) {
 
 ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_t* idx, int k,
                          ic_rows r, float scale, void* out, uint32_t* status, void* scratch,
-                         size_t scratch_bytes, cudaStream_t s) {
+                         size_t scratch_bytes, cudaStream_t s, int64_t max_units) {
     (void)ks;
     if (((uintptr_t)q & 15) || ((uintptr_t)kv & 15) || ((uintptr_t)out & 15))
         return IC_ERR_INVALID_ARG;
@@ -869,14 +880,15 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
     a.q_start = r.q_start;
     a.T = r.T;
     a.scale_log2 = scale * LOG2E;
-    plan_splits(r, k, a.splits, a.keys_per_split);
+    plan_splits(r, k, a.splits, a.keys_per_split, max_units);
     const int64_t units = (int64_t)r.B * r.Lq * a.splits;
     if (2 * units > 0x7fffffff) return IC_ERR_UNSUPPORTED;
     a.n_units = (int)units;
     a.part_o = nullptr;
     a.part_ml = nullptr;
     if (a.splits > 1) {
-        if (scratch_bytes < attn_tc_scratch_bytes(r, k) || scratch == nullptr) return IC_ERR_WORKSPACE;
+        if (scratch_bytes < attn_tc_scratch_bytes(r, k, max_units) || scratch == nullptr)
+            return IC_ERR_WORKSPACE;
         a.part_o = static_cast<float*>(scratch);
         a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(scratch) +
                                               (size_t)units * HQ * DV * sizeof(float) + 256 -

@@ -75,9 +75,14 @@ ic_status launch_attn_simt(const void* q, const void* kmat, int64_t ks, const vo
 
 bool attn_tc_supported(const void* kmat, const void* vmat, int64_t ks, int64_t vs, ic_dtype dt,
                        int Hq, int d_qk, int d_v);
-size_t attn_tc_scratch_bytes(ic_rows r, int k);
+// max_units caps the split-k plan's units (rows x splits); the smallest
+// split count is kept even above it, so callers with a fixed limit check
+// attn_tc_units against it first.
+constexpr int64_t kNoUnitLimit = INT64_MAX;
+int64_t attn_tc_units(ic_rows r, int k, int64_t max_units = kNoUnitLimit);
+size_t attn_tc_scratch_bytes(ic_rows r, int k, int64_t max_units = kNoUnitLimit);
 ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_t* idx, int k,
                          ic_rows r, float scale, void* out, uint32_t* status, void* scratch,
-                         size_t scratch_bytes, cudaStream_t s);
+                         size_t scratch_bytes, cudaStream_t s, int64_t max_units = kNoUnitLimit);
 
 }  // namespace ic

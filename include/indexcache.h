@@ -212,17 +212,23 @@ ic_status ic_sparse_attn(const void* q, const void* kmat, int64_t k_row_stride,
  * kmat = vmat = kv and row strides 576, except that the split-k partials of
  * decode live in a fixed device array inside the library of
  * IC_NOALLOC_SCRATCH_BYTES bytes (about 16 MiB; every GPU that loads the
- * library holds it until the process exits), enough for
- * B*Lq*splits <= 64 partial rows.  A call that would need more returns
- * IC_ERR_WORKSPACE before launching anything; use ic_sparse_attn with a
+ * library holds it until the process exits), room for 64 partial rows
+ * (query rows x splits).  Among its split counts this call only considers
+ * those that keep B*Lq*splits <= 64, so it may split less finely than
+ * ic_sparse_attn (same results within the attention tolerance, maybe
+ * slower).  A row needs at least ceil(k / 2048) splits, so the call is
+ * refused with IC_ERR_WORKSPACE, before launching anything, exactly when
+ * k > 2048 and B*Lq*ceil(k / 2048) > 64; use ic_sparse_attn with a
  * workspace instead.  This function allocates nothing.
  *   device_status  NULL, or a DEVICE int32 that receives the call's status
  *                  bits (as ic_read_status reports them) when it completes.
- * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  All calls share the array and it keeps the last call's contents
- * (the status word is cleared at the start of each call): calls whose kernels
- * overlap on the GPU race on it, so serialise them (one stream, one thread).
+ * The array's device address is looked up on the first call on a device
+ * (with that device current) and again when the device's CUDA context has
+ * changed since (after a cudaDeviceReset); make the first call on each
+ * device, and the first after a reset, before any stream capture.  All calls
+ * share the array and it keeps the last call's contents (the status word is
+ * cleared at the start of each call): calls whose kernels overlap on the GPU
+ * race on it, so serialise them (one stream, one thread).
  */
 #define IC_NOALLOC_SCRATCH_BYTES ((16u << 20) + (64u << 10) + 512u)
 ic_status ic_sparse_attn_noalloc(const void* q, const void* kv, const int32_t* idx, int k,

@@ -1,7 +1,7 @@
 """Run one stage of the hot path on a small slice of a workload, for profilers.
 
-    python -m cross_layer_top_full_b200.profile_case --stage attention \
-        --workload prefill_8k_bf16 --rows 512 --launches 3
+    python profile_case.py --stage attention --workload prefill_8k_bf16 \
+        --rows 512 --launches 3
 
 Builds the inputs of layer 0 of the workload on cuda:0, keeps the last
 ``--rows`` query rows of each sequence (the heaviest rows of a prefill), runs
@@ -14,11 +14,15 @@ from __future__ import annotations
 import argparse
 import dataclasses
 import json
+import os
+import sys
 
 import torch
 
-import cross_layer_top_full_b200 as ic
-from cross_layer_top_full_b200 import synth
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+import cross_layer_top_full_b200 as ic  # noqa: E402
+from cross_layer_top_full_b200 import synth  # noqa: E402
 
 DT = {"f32": ic.F32, "bf16": ic.BF16, "e4m3": ic.FP8_E4M3}
 

@@ -11,10 +11,11 @@
   position scores at least tau - 1e-3|tau|; no duplicates, all in [0, t],
   ascending, -1 padded, exactly min(k, t+1) kept.
 * attention: "within 1e-2 max abs and 1e-2 relative" read elementwise as
-  |gpu - oracle| <= 1e-2 + 1e-2 |oracle| (the allclose form), plus the
+  |gpu - oracle| <= max(1e-2, 1e-2 |oracle|): 1e-2 absolute where the
+  output is below 1 in magnitude, 1e-2 relative above it; plus the
   aggregate ||gpu - oracle||_2 <= 1e-2 ||oracle||_2.  A pure 1e-2 absolute
   bound cannot hold for bf16 outputs of magnitude >= 2, whose rounding step
-  alone is 2^-7 or more.
+  alone is 2^-7 or more (a relative 2^-8 half-step, inside 1e-2).
 """
 import numpy as np
 import torch
@@ -92,16 +93,21 @@ def check_topk_band(idx: np.ndarray, ref_scores: np.ndarray, q_start: int, k: in
     return differ
 
 
+def attn_bound(ref: np.ndarray) -> np.ndarray:
+    """Elementwise attention bound max(1e-2, 1e-2 |ref|)."""
+    return np.maximum(ATTN_ATOL, ATTN_RTOL * np.abs(ref))
+
+
 def check_attention(gpu: np.ndarray, ref: np.ndarray, what: str = "") -> None:
     if not np.all(np.isfinite(gpu)):
         at = np.unravel_index(int(np.argmin(np.isfinite(gpu))), gpu.shape)
         raise AssertionError("%s non-finite output %r at %s" % (what, gpu[at], at))
     d = np.abs(gpu - ref)
-    excess = d - (ATTN_ATOL + ATTN_RTOL * np.abs(ref))
+    excess = d - attn_bound(ref)
     worst = float(excess.max()) if d.size else -1.0
     rel = float(np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-30))
     if worst > 0:
         at = np.unravel_index(int(np.argmax(excess)), d.shape)
-        raise AssertionError("%s |diff| %g > %g + %g*|ref| at %s (ref %g)"
+        raise AssertionError("%s |diff| %g > max(%g, %g*|ref|) at %s (ref %g)"
                              % (what, d[at], ATTN_ATOL, ATTN_RTOL, at, ref[at]))
     assert rel <= ATTN_REL_L2, "%s rel L2 = %g" % (what, rel)

@@ -9,15 +9,16 @@ check covers outputs the oracle computes one by one (tests/stack_check.py):
   * decode 8 x 200K (FP8 indexer): every sequence, all 48 layers;
   * chunked prefill 64K: all 16 chunks, 16 rows each (always the chunk's
     first and last row), indices and attention of all 12 layers.
+  * prefill 8K with the FP8 indexer: indices of 512 seeded rows, attention
+    on 128 of them, all 4 layers.
 Per checked row: an F layer's indices obey the top-k band rule against the
 oracle's float64 scores; an S layer's indices are the F layer's bit for bit
-(all rows); attention, where the kernel chose exactly the oracle's top-k set
-(all but allowed near-tie swaps), is within the attention tolerance of the
-oracle's, computed from the oracle's own indices.  Each test also requires
-that the attention of most checked rows was compared: 80 % with the bf16
-indexer, 50 % with the FP8 one, whose tensor-core accumulation of 128 e4m3
-products is allowed more near-tie swaps (the band rule still holds on every
-row).
+(all rows); attention of EVERY sampled row is within the attention
+tolerance of the oracle's float64 attention over the index set the kernel
+used (band-valid, so a valid top-k; where it differs from the oracle's own
+exact top-k by allowed near-tie swaps, the comparison still runs).  The
+number of rows whose set equals the oracle's exact top-k is printed, not
+asserted: it measures near ties, not correctness.
 """
 import pytest
 import torch
@@ -37,6 +38,14 @@ def dev():
         pytest.skip("no CUDA device")
     ic.lib()
     return torch.device("cuda:0")
+
+
+def report(what, n_cmp, n_same):
+    """Every sampled attention row was compared; say how many of them used
+    exactly the oracle's top-k set (the rest differ by allowed near ties)."""
+    assert n_cmp > 0
+    print("%s: %d attention rows compared, %d with the oracle's exact index set"
+          % (what, n_cmp, n_same))
 
 
 def run_stack(wl, pattern, inputs, rows, dev):
@@ -70,7 +79,7 @@ def test_prefill_8k_bf16_full_size(dev):
                             always=(0, 1, wl.k - 1, wl.k, wl.k + 1, wl.L - 1))
     n_cmp, n_same = check_stack(wl, wl.pattern, inputs, copies, outs, 0, [0], range(wl.L),
                                 attn_rows, range(wl.n_layers), "prefill_8k")
-    assert n_same >= 0.8 * n_cmp
+    report("prefill_8k", n_cmp, n_same)
     del inputs, outs, copies
     torch.cuda.empty_cache()
 
@@ -83,7 +92,7 @@ def test_decode_b32_t32k_bf16_full_size(dev):
     assert n_ix == wl.pattern.count("F")
     n_cmp, n_same = check_stack(wl, wl.pattern, inputs, copies, outs, wl.q_start, range(wl.B),
                                 [0], [0], range(wl.n_layers), "decode_b32")
-    assert n_same >= 0.8 * n_cmp
+    report("decode_b32", n_cmp, n_same)
     del inputs, outs, copies
     torch.cuda.empty_cache()
 
@@ -98,7 +107,7 @@ def test_decode_b8_t200k_fp8_full_size(dev):
     assert n_ix == wl.pattern.count("F") == 12
     n_cmp, n_same = check_stack(wl, wl.pattern, inputs, copies, outs, wl.q_start, range(wl.B),
                                 [0], [0], range(wl.n_layers), "decode_fp8")
-    assert n_same >= 0.5 * n_cmp
+    report("decode_fp8", n_cmp, n_same)
     del inputs, outs, copies
     torch.cuda.empty_cache()
 
@@ -122,5 +131,26 @@ def test_chunked_prefill_64k_bf16_every_chunk(dev):
         n_same += same_c
         del inputs, outs, copies
         torch.cuda.empty_cache()
-    assert n_same >= 0.8 * n_cmp
+    report("chunked_64k", n_cmp, n_same)
+
+
+# --------------------------------------------------------------------------- prefill 8k, FP8 indexer
+def test_prefill_8k_fp8_indexer_full_size(dev):
+    """The 8K prefill with the indexer operands in E4M3 (one scale per token):
+    the prefill-shaped FP8 tensor-core indexer at full size.  Indices of 512
+    seeded rows (always 0, 1, k-1, k, k+1, L-1); attention on 128 of them,
+    all 4 layers."""
+    wl = synth.WORKLOADS["prefill_8k_fp8"]
+    inputs = [synth.layer_inputs(wl, l, dev) for l in range(wl.n_layers)]
+    outs, copies, n_ix = run_stack(wl, wl.pattern, inputs, (wl.B, wl.L, 0, wl.T), dev)
+    assert n_ix == wl.pattern.count("F")
+    always = (0, 1, wl.k - 1, wl.k, wl.k + 1, wl.L - 1)
+    idx_rows = sample_rows(wl.L, 512, seed=7, always=always)
+    attn_rows = sample_rows(len(idx_rows), 122, seed=8)
+    attn_rows = sorted(set([idx_rows[j] for j in attn_rows]) | set(always))
+    n_cmp, n_same = check_stack(wl, wl.pattern, inputs, copies, outs, 0, [0], idx_rows,
+                                attn_rows, range(wl.n_layers), "prefill_8k_fp8")
+    report("prefill_8k_fp8", n_cmp, n_same)
+    del inputs, outs, copies
+    torch.cuda.empty_cache()
 

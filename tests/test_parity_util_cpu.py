@@ -6,7 +6,8 @@ import numpy as np
 import pytest
 
 import oracle
-from parity_util import ATTN_ATOL, ATTN_RTOL, check_attention, check_scores, check_topk_band
+from parity_util import (ATTN_ATOL, attn_bound, check_attention, check_scores,
+                         check_topk_band)
 
 
 def _scores():
@@ -61,12 +62,19 @@ def test_check_attention():
     rng = np.random.default_rng(5)
     ref = rng.standard_normal((2, 3, 4, 16)) * 3
     check_attention(ref.copy(), ref)
-    near = ref + 0.9 * (ATTN_ATOL + ATTN_RTOL * np.abs(ref)) * rng.choice([-1, 1], ref.shape) * 0.01
+    near = ref + 0.9 * attn_bound(ref) * rng.choice([-1, 1], ref.shape) * 0.01
     check_attention(near, ref)
     bad = ref.copy()
-    bad[1, 2, 3, 4] += 2 * (ATTN_ATOL + ATTN_RTOL * abs(ref[1, 2, 3, 4]))
+    bad[1, 2, 3, 4] += 2 * attn_bound(ref[1, 2, 3, 4])
     with pytest.raises(AssertionError, match="diff"):
         check_attention(bad, ref, "planted")
+    # the bound is the larger of the two terms, not their sum: an error of
+    # 1.5e-2 on an output of 1.0 fails (the sum form would allow 2e-2)
+    one = np.ones((4, 8))
+    bad = one.copy()
+    bad[2, 3] += 1.5e-2
+    with pytest.raises(AssertionError, match="diff"):
+        check_attention(bad, one, "planted")
     bad = ref.copy()
     bad[0, 0, 0, 0] = np.nan
     with pytest.raises(AssertionError, match="non-finite"):

@@ -65,15 +65,18 @@ def _noalloc(q, kv, idx, rows, scale, dev):
 
 
 @pytest.mark.parametrize("rows,k", [((8, 1, 4999, 5000), 2048),     # decode, split-k partials
+                                    ((6, 1, 4999, 5000), 2048),     # split count capped by the array
+                                    ((12, 1, 4999, 5000), 2048),
+                                    ((16, 1, 8999, 9000), 4096),    # 2+ splits per row, 64 units
                                     ((3, 2, 700, 702), 512)])
 def test_noalloc_matches_workspace_entry_point_twice(dev, rows, k):
     scale = 576 ** -0.5
-    # the decode case must actually use the fixed array (split-k partials)
+    # the decode cases must actually use the fixed array (split-k partials)
     need = ic.sparse_attn_workspace_size(rows, k, 128, 576, 512, ic.BF16) - ic.STATUS_BYTES
-    if rows[0] == 8:
+    if rows[1] == 1:
         assert need > 0
     for call, seed in enumerate((1, 2)):            # two calls in a row, different inputs
-        q, kv, idx = _inputs(rows, k, dev, seed + 10 * k)
+        q, kv, idx = _inputs(rows, k, dev, seed + 10 * k + rows[0])
         ref = _with_workspace(q, kv, idx, rows, scale, dev)
         got, status = _noalloc(q, kv, idx, rows, scale, dev)
         torch.cuda.synchronize()
@@ -86,17 +89,26 @@ def test_noalloc_matches_workspace_entry_point_twice(dev, rows, k):
 
 
 def test_noalloc_rejects_problems_beyond_its_fixed_array(dev):
-    rows, k = (33, 1, 2999, 3000), 2048
-    need = ic.sparse_attn_workspace_size(rows, k, 128, 576, 512, ic.BF16) - ic.STATUS_BYTES
+    """k = 4096 needs at least two splits of 2048 keys per row, so 33 decode
+    rows need at least 66 partial rows, more than the array's 64, on any GPU:
+    the call is refused before anything is launched and leaves the output
+    untouched."""
+    rows, k = (33, 1, 4999, 5000), 4096
     q, kv, idx = _inputs(rows, k, dev, 5)
     out = torch.zeros(33, 1, 128, 512, dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
     code = ic.lib().ic_sparse_attn_noalloc(q.data_ptr(), kv.data_ptr(), idx.data_ptr(), k,
                                            ic.Rows(*rows), ctypes.c_float(0.04), out.data_ptr(),
                                            None, torch.cuda.current_stream().cuda_stream)
-    limit = (16 << 20) + (64 << 10) + 512 - 256
-    if need > limit:
-        assert code == -4                          # IC_ERR_WORKSPACE, nothing launched
-        torch.cuda.synchronize()
-        assert not out.float().abs().sum().item()
-    else:
-        assert code == 0
+    assert code == -4                              # IC_ERR_WORKSPACE, nothing launched
+    torch.cuda.synchronize()
+    assert not out.float().abs().sum().item()
+    # one row fewer than the limit allows (32 rows x 2 splits = 64) runs
+    rows, k = (32, 1, 4999, 5000), 4096
+    q, kv, idx = q[:32].contiguous(), kv[:32].contiguous(), idx[:32].contiguous()
+    got, status = _noalloc(q, kv, idx, rows, 0.04, dev)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    kvh = host64(kv)
+    want = oracle.sparse_attention(host64(q), kvh, kvh[..., :512], host64(idx), 0.04)
+    check_attention(host64(got), want, "no-alloc at its limit vs oracle")
