@@ -527,6 +527,7 @@ def decode_entry(line):
             for k, v in line["stages_ms"].items()},
         "roofline_by_stage": line["roofline_by_stage"],
         "indexer_share_of_step": line["indexer_share_of_step"],
+        "topk_overlap_matrix": line["topk_overlap_matrix"],
         "cpu_baseline": line["cpu_baseline"], "e2e": line["e2e"],
         "gpu_launches": line["gpu_launches"], "cuda_graph": line["cuda_graph"],
         "clocks": line["clocks"], "device_status": line["device_status"],
@@ -630,6 +631,21 @@ def measure_stack(wl, pattern, dev, pg, rank, world, *, steps, warmup, graph, e2
         e2e_line = run_e2e(st, pattern, min(steps, 50 if wl.L == 1 else steps), dev, pg)
         require_clean(st.ws, "%s e2e" % wl.name)
 
+    # untimed: every layer's own top-k (each running its own indexer) and the
+    # all-pairs layer overlap matrix a pattern search would consume
+    own = []
+    for l in range(len(pattern)):
+        L_ = st.layers[l]
+        ic.indexer_scores(L_["q_idx"], L_["w"], L_["k_idx"], st.rows, st.scores, st.ws,
+                          q_scale=L_["q_scale"], k_scale=L_["k_scale"], dtype=DT[wl.idx_dtype])
+        ic.topk(st.scores, st.rows, wl.k, st.idx, st.ws)
+        own.append(st.idx.view(-1, wl.k).clone())
+    s_sum, s_min, n_rows = overlap_matrix(own, wl.T)
+    overlap = overlap_json(s_sum, s_min, n_rows, "%s, all %d layers, %d query rows"
+                           % (wl.name, len(pattern), n_rows))
+    del own
+    require_clean(st.ws, "%s overlap pass" % wl.name)
+
     per_step_ms = ms / steps
     value = whole_job_rate(tokens_per_step, world, per_step_ms)
     work = algorithmic(wl)
@@ -673,6 +689,7 @@ def measure_stack(wl, pattern, dev, pg, rank, world, *, steps, warmup, graph, e2
         "indexer_share_of_step": sel_share,
         "roofline": roof,
         "roofline_by_stage": by_stage,
+        "topk_overlap_matrix": overlap,
         "cpu_baseline": cpu,
         "e2e": e2e_line,
         "gpu_launches": launches,
@@ -694,6 +711,45 @@ def row_overlap(reused, own, T):
     b = torch.where(b >= 0, b + off, torch.full_like(b, -2))
     hit = torch.isin(b.flatten(), a.flatten()).view(rows, k).sum(1).to(torch.float64)
     return hit / (reused >= 0).sum(1).clamp(min=1).to(torch.float64)
+
+
+def overlap_matrix(sets, T):
+    """All-pairs top-k overlap of per-layer index sets: sets[l] is an [rows,
+    k] tensor of layer l's own top-k (ascending positions in [0, T), -1
+    padding last).  Entry (l, m) is, per row, |A_l & A_m| / |A_l| (the
+    oracle's topk_overlap), returned as (sum over rows, min over rows, rows)
+    so that calls over several chunks can be merged.  Runs on the sets'
+    device: each row of A_m is searched for the entries of A_l."""
+    L = len(sets)
+    rows = sets[0].shape[0]
+    big = torch.iinfo(torch.int32).max
+    sorted_sets = []
+    sizes = []
+    for a in sets:
+        a = a.to(torch.int64)
+        sizes.append((a >= 0).sum(1).clamp(min=1).to(torch.float64))
+        sorted_sets.append(torch.where(a >= 0, a, torch.full_like(a, big)))   # padding sorts last
+    s_sum = torch.zeros(L, L, dtype=torch.float64)
+    s_min = torch.ones(L, L, dtype=torch.float64)
+    for l in range(L):
+        a = sets[l].to(torch.int64)
+        for m in range(L):
+            b = sorted_sets[m]
+            pos = torch.searchsorted(b, a.contiguous()).clamp(max=b.shape[1] - 1)
+            hit = ((b.gather(1, pos) == a) & (a >= 0)).sum(1).to(torch.float64)
+            frac = hit / sizes[l]
+            s_sum[l, m] = float(frac.sum())
+            s_min[l, m] = float(frac.min())
+    return s_sum, s_min, rows
+
+
+def overlap_json(s_sum, s_min, rows, what):
+    L = s_sum.shape[0]
+    return {"layers": L, "rows": rows, "of": what,
+            "definition": "per row |A_l & A_m| / |A_l| of layer l's and layer m's own top-k "
+                          "(each layer running its own indexer), mean and minimum over rows",
+            "mean": [[round(float(s_sum[l, m]) / rows, 4) for m in range(L)] for l in range(L)],
+            "min": [[round(float(s_min[l, m]), 4) for m in range(L)] for l in range(L)]}
 
 
 def run_chunked(args, wl, pattern, dev, pg, rank, world):
@@ -832,22 +888,34 @@ def run_chunked(args, wl, pattern, dev, pg, rank, world):
                          {k: len(v) for k, v in stages.items()}, per_pass=nch)
     roof["traffic"] = _traffic(dom, args.workload)
 
-    # untimed: top-k overlap of each S layer's own selection with the reused one
-    own = torch.empty_like(idx_buf)
+    # untimed: every layer's own top-k per chunk; the top-k overlap of each S
+    # layer's own selection with the reused one, and the all-pairs layer
+    # overlap matrix over every row of every chunk
+    own = [torch.empty(C, wl.k, dtype=torch.int32, device=dev) for _ in range(nl)]
     acc = {}
+    m_sum = torch.zeros(nl, nl, dtype=torch.float64)
+    m_min = torch.ones(nl, nl, dtype=torch.float64)
     for c in range(nch):
         r = rows[c]
+        reused = None
         for l, kind in enumerate(pattern):
             kI = keys[l][0]
             ic.indexer_scores(qI[qkey(l, c)], wI[qkey(l, c)], kI, r, scores, ws,
                               dtype=DT[wl.idx_dtype])
-            ic.topk(scores, r, wl.k, own if kind == "S" else idx_buf, ws)
+            ic.topk(scores, r, wl.k, own[l].view(1, C, wl.k), ws)
             if kind == "F":
+                reused = own[l]
                 continue
-            frac = row_overlap(idx_buf[0], own[0], wl.T)
+            frac = row_overlap(reused, own[l], wl.T)
             s_, n_, mn = acc.get(l, (0.0, 0, 1.0))
             acc[l] = (s_ + float(frac.sum()), n_ + C, min(mn, float(frac.min())))
+        s_sum, s_min, _ = overlap_matrix(own, wl.T)
+        m_sum += s_sum
+        m_min = torch.minimum(m_min, s_min)
     overlap = {"layer_%d" % l: {"mean": v[0] / v[1], "min": v[2]} for l, v in sorted(acc.items())}
+    overlap_all = overlap_json(m_sum, m_min, nch * C, "%s, all %d layers, every row of the %d "
+                               "chunks" % (wl.name, nl, nch))
+    del own
     torch.cuda.synchronize()
     progress("overlap pass done")
 
@@ -881,6 +949,7 @@ def run_chunked(args, wl, pattern, dev, pg, rank, world):
         "stages_ms": {k: {"per_launch": avg[k], "launches_per_step": len(v)}
                       for k, v in stages.items()},
         "topk_overlap_s_layers": overlap,
+        "topk_overlap_matrix": overlap_all,
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": None,

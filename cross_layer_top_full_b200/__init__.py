@@ -16,12 +16,14 @@ import os
 from typing import Dict, List, Optional, Sequence
 
 __all__ = [
-    "IcError", "lib", "library_path", "Rows", "StackShape", "LayerIO",
+    "IcError", "lib", "library_path", "Rows", "StackShape", "LayerIO", "PagedRows", "paged_rows",
     "F32", "BF16", "FP8_E4M3", "STATUS_BYTES",
     "status_string", "version", "kernel_launches", "workspace_init", "read_status",
     "indexer_workspace_size", "indexer_scores", "topk_workspace_size", "topk",
     "sparse_attn_workspace_size", "sparse_attn", "sparse_attn_noalloc", "workspace_size",
-    "layer_stack_forward",
+    "layer_stack_forward", "indexer_scores_paged", "topk_varlen_workspace_size", "topk_varlen",
+    "sparse_attn_paged_workspace_size", "sparse_attn_paged", "paged_workspace_size",
+    "layer_stack_forward_paged",
 ]
 
 F32, BF16, FP8_E4M3 = 0, 1, 2
@@ -63,6 +65,14 @@ class LayerIO(ctypes.Structure):
                 ("q_idx", "q_scale", "w", "k_idx", "k_scale", "q", "kmat", "vmat", "out")]
 
 
+class PagedRows(ctypes.Structure):
+    """ic_paged_rows: a variable-length batch over paged caches."""
+    _fields_ = [("B", ctypes.c_int), ("Lq", ctypes.c_int), ("T_max", ctypes.c_int),
+                ("seq_lens", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+                ("max_pages", ctypes.c_int), ("page_size", ctypes.c_int),
+                ("num_pages", ctypes.c_int)]
+
+
 _P = ctypes.c_void_p
 _SIG = {
     "ic_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -89,6 +99,24 @@ _SIG = {
     "ic_layer_stack_forward": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_int,
                                               ctypes.POINTER(LayerIO), ctypes.POINTER(StackShape),
                                               _P, ctypes.POINTER(_P), _P, ctypes.c_size_t, _P]),
+    "ic_indexer_scores_paged": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int,
+                                               ctypes.POINTER(PagedRows), ctypes.c_int,
+                                               ctypes.c_int, _P, ctypes.c_int64, _P,
+                                               ctypes.c_size_t, _P]),
+    "ic_topk_varlen_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(PagedRows), ctypes.c_int]),
+    "ic_topk_varlen": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.POINTER(PagedRows), ctypes.c_int,
+                                      _P, _P, ctypes.c_size_t, _P]),
+    "ic_sparse_attn_paged_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(PagedRows),
+                                                              ctypes.c_int]),
+    "ic_sparse_attn_paged": (ctypes.c_int, [_P, _P, _P, ctypes.c_int, ctypes.POINTER(PagedRows),
+                                            ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+    "ic_paged_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(StackShape),
+                                                  ctypes.POINTER(PagedRows)]),
+    "ic_layer_stack_forward_paged": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_int,
+                                                    ctypes.POINTER(LayerIO),
+                                                    ctypes.POINTER(StackShape),
+                                                    ctypes.POINTER(PagedRows), _P,
+                                                    ctypes.POINTER(_P), _P, ctypes.c_size_t, _P]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -273,3 +301,72 @@ def layer_stack_forward(pattern: str, layers: Sequence[Dict], shape: StackShape,
     _check(lib().ic_layer_stack_forward(pattern.encode(), n, arr, ctypes.byref(shape),
                                         _ptr(idx_buf), outs, _ptr(ws), _nbytes(ws),
                                         _stream(stream)), "ic_layer_stack_forward")
+
+
+# --------------------------------------------------------------------------- paged / varlen
+def paged_rows(seq_lens, block_table, T_max: int, page_size: int, num_pages: int,
+               Lq: int = 1) -> PagedRows:
+    """ic_paged_rows for seq_lens [B] int32 and block_table [B, max_pages]
+    int32 (device tensors, kept alive by the caller)."""
+    B = int(seq_lens.shape[0])
+    max_pages = int(block_table.shape[1]) if block_table is not None else 0
+    return PagedRows(B, int(Lq), int(T_max), _ptr(seq_lens), _ptr(block_table), max_pages,
+                     int(page_size), int(num_pages))
+
+
+def indexer_scores_paged(q_idx, w, k_pages, pr: PagedRows, scores, ws, *, q_scale=None,
+                         k_scale_pages=None, dtype: Optional[int] = None,
+                         ld_scores: Optional[int] = None, stream=None) -> None:
+    dt = _dtype_of(q_idx) if dtype is None else dtype
+    H_I, d_I = q_idx.shape[-2], q_idx.shape[-1]
+    ld = scores.shape[-1] if ld_scores is None else ld_scores
+    _check(lib().ic_indexer_scores_paged(_ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(k_pages),
+                                         _ptr(k_scale_pages), dt, ctypes.byref(pr), H_I, d_I,
+                                         _ptr(scores), ld, _ptr(ws), _nbytes(ws), _stream(stream)),
+           "ic_indexer_scores_paged")
+
+
+def topk_varlen_workspace_size(pr: PagedRows, k: int) -> int:
+    return int(lib().ic_topk_varlen_workspace_size(ctypes.byref(pr), k))
+
+
+def topk_varlen(scores, pr: PagedRows, k: int, idx, ws, *, ld_scores: Optional[int] = None,
+                stream=None) -> None:
+    ld = scores.shape[-1] if ld_scores is None else ld_scores
+    _check(lib().ic_topk_varlen(_ptr(scores), ld, ctypes.byref(pr), k, _ptr(idx), _ptr(ws),
+                                _nbytes(ws), _stream(stream)), "ic_topk_varlen")
+
+
+def sparse_attn_paged_workspace_size(pr: PagedRows, k: int) -> int:
+    return int(lib().ic_sparse_attn_paged_workspace_size(ctypes.byref(pr), k))
+
+
+def sparse_attn_paged(q, kv_pages, idx, pr: PagedRows, scale: float, out, ws, *,
+                      stream=None) -> None:
+    _check(lib().ic_sparse_attn_paged(_ptr(q), _ptr(kv_pages), _ptr(idx), idx.shape[-1],
+                                      ctypes.byref(pr), float(scale), _ptr(out), _ptr(ws),
+                                      _nbytes(ws), _stream(stream)), "ic_sparse_attn_paged")
+
+
+def paged_workspace_size(shape: StackShape, pr: PagedRows) -> int:
+    return int(lib().ic_paged_workspace_size(ctypes.byref(shape), ctypes.byref(pr)))
+
+
+def layer_stack_forward_paged(pattern: str, layers: Sequence[Dict], shape: StackShape,
+                              pr: PagedRows, idx_buf, ws, *, idx_out: Optional[List] = None,
+                              stream=None) -> None:
+    """The F/S layer stack over paged caches: each layer dict holds q_idx,
+    q_scale, w, k_idx (= that layer's paged k_I), k_scale (its paged scales),
+    q, kmat (= its paged KV rows) and out."""
+    n = len(layers)
+    arr = (LayerIO * max(1, n))()
+    for l, L in enumerate(layers):
+        for name, _ in LayerIO._fields_:
+            setattr(arr[l], name, _ptr(L.get(name)))
+    outs = None
+    if idx_out is not None:
+        outs = (_P * max(1, n))(*[_ptr(x) for x in idx_out])
+    _check(lib().ic_layer_stack_forward_paged(pattern.encode(), n, arr, ctypes.byref(shape),
+                                              ctypes.byref(pr), _ptr(idx_buf), outs, _ptr(ws),
+                                              _nbytes(ws), _stream(stream)),
+           "ic_layer_stack_forward_paged")

@@ -84,6 +84,35 @@ size_t attn_scratch(const ic_rows& r, int k, int Hq, int d_qk, int d_v, ic_dtype
     return 0;
 }
 
+// A paged batch: sizes consistent, device arrays present, every sequence's
+// logical pages addressable by its block-table row.
+bool paged_ok(const ic_paged_rows* pr, bool need_pages) {
+    if (pr == nullptr || pr->B < 0 || pr->Lq < 1 || pr->T_max < pr->Lq) return false;
+    if (pr->B > 0 && pr->seq_lens == nullptr) return false;
+    if (!need_pages) return true;
+    if (pr->page_size < 128 || pr->page_size % 128 != 0 || pr->num_pages < 1) return false;
+    if ((int64_t)pr->num_pages * pr->page_size >= 0x7fffffffLL) return false;
+    if ((int64_t)pr->max_pages * pr->page_size < pr->T_max) return false;
+    return pr->B == 0 || pr->block_table != nullptr;
+}
+
+// Planning rows of a paged batch: every sequence as long as T_max.
+ic_rows plan_rows(const ic_paged_rows* pr) { return ic_rows{pr->B, pr->Lq, pr->T_max - pr->Lq, pr->T_max}; }
+
+ic_status run_topk_varlen(const float* scores, int64_t ld, const ic_paged_rows* pr, int k,
+                          int32_t* idx, cudaStream_t s) {
+    const ic_rows r = plan_rows(pr);
+    if (topk_cluster_applies(r, k) && ((uintptr_t)scores & 15) == 0)
+        return launch_topk_cluster(scores, ld, r, k, idx, s, pr->seq_lens);
+    return launch_topk_rows(scores, ld, r, k, idx, s, pr->seq_lens);
+}
+
+bool latent_tc_shape(const ic_stack_shape* sh) {
+    return indexer_tc_supported(sh->idx_dtype, sh->H_I, sh->d_I) && sh->attn_dtype == IC_BF16 &&
+           sh->Hq == 128 && sh->d_qk == 576 && sh->d_v == 512 && sh->k_row_stride == 576 &&
+           sh->v_row_stride == 576;
+}
+
 ic_status run_indexer(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                       const float* k_scale, ic_dtype dt, ic_rows r, int H_I, int d_I,
                       float* scores, int64_t ld, uint32_t* status, cudaStream_t s) {
@@ -95,7 +124,11 @@ ic_status run_indexer(const void* q_idx, const float* q_scale, const float* w, c
 
 ic_status run_topk(const float* scores, int64_t ld, ic_rows r, int k, int32_t* idx, void* scratch,
                    size_t scratch_bytes, cudaStream_t s) {
-    // the multi-CTA path reads 16-byte vectors: it needs 16-byte aligned rows
+    // the cluster and multi-CTA paths read 16-byte vectors: they need 16-byte
+    // aligned rows.  Few long rows (decode): one cluster per row, one launch;
+    // rows too long for the cluster's shared memory: three launches.
+    if (topk_cluster_applies(r, k) && ((uintptr_t)scores & 15) == 0)
+        return launch_topk_cluster(scores, ld, r, k, idx, s);
     if (topk_multi_applies(r, k) && scratch != nullptr && ((uintptr_t)scores & 15) == 0 &&
         scratch_bytes >= topk_multi_scratch_bytes(r, k))
         return launch_topk_multi(scores, ld, r, k, idx, scratch, s);
@@ -285,6 +318,115 @@ ic_status ic_layer_stack_forward(const char* pattern, int n_layers, const ic_lay
         ic_status st = run_attn(L.q, L.kmat, sh->k_row_stride, L.vmat, sh->v_row_stride, idx_buf,
                                 sh->k, sh->attn_dtype, r, sh->Hq, sh->d_qk, sh->d_v, sh->scale,
                                 L.out, status, attn_ws, attn_ws_bytes, s);
+        if (st != IC_OK) return st;
+        if (idx_out != nullptr && idx_out[l] != nullptr) {
+            if (cudaMemcpyAsync(idx_out[l], idx_buf, idx_bytes, cudaMemcpyDeviceToDevice, s) !=
+                cudaSuccess)
+                return cuda_error("api");
+        }
+    }
+    return IC_OK;
+}
+
+// ------------------------------------------------------------------ paged / varlen
+ic_status ic_indexer_scores_paged(const void* q_idx, const float* q_scale, const float* w,
+                                  const void* k_pages, const float* k_scale_pages, ic_dtype dt,
+                                  const ic_paged_rows* pr, int H_I, int d_I, float* scores,
+                                  int64_t ld_scores, void* ws, size_t ws_bytes, void* stream) {
+    if (!paged_ok(pr, true) || !indexer_args_ok(dt, H_I, d_I)) return IC_ERR_INVALID_ARG;
+    if (!indexer_tc_supported(dt, H_I, d_I)) return IC_ERR_UNSUPPORTED;
+    if (ld_scores < pr->T_max || ld_scores % 4 != 0) return IC_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, IC_STATUS_BYTES)) return IC_ERR_WORKSPACE;
+    if (pr->B == 0) return IC_OK;
+    if (!q_idx || !w || !k_pages || !scores) return IC_ERR_INVALID_ARG;
+    if (dt == IC_FP8_E4M3 && (!q_scale || !k_scale_pages)) return IC_ERR_INVALID_ARG;
+    if (dt != IC_FP8_E4M3 && (q_scale || k_scale_pages)) return IC_ERR_INVALID_ARG;
+    return launch_indexer_tc_paged(q_idx, q_scale, w, k_pages, k_scale_pages, dt, *pr, H_I, d_I,
+                                   scores, ld_scores, status_of(ws), (cudaStream_t)stream);
+}
+
+size_t ic_topk_varlen_workspace_size(const ic_paged_rows* pr, int k) {
+    (void)pr; (void)k;
+    return IC_STATUS_BYTES;
+}
+
+ic_status ic_topk_varlen(const float* scores, int64_t ld_scores, const ic_paged_rows* pr, int k,
+                         int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+    if (!paged_ok(pr, false) || k < 1 || k > 16384) return IC_ERR_INVALID_ARG;
+    if (ld_scores < pr->T_max || ld_scores % 4 != 0) return IC_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, ic_topk_varlen_workspace_size(pr, k))) return IC_ERR_WORKSPACE;
+    if (pr->B == 0) return IC_OK;
+    if (!scores || !idx) return IC_ERR_INVALID_ARG;
+    return run_topk_varlen(scores, ld_scores, pr, k, idx, (cudaStream_t)stream);
+}
+
+size_t ic_sparse_attn_paged_workspace_size(const ic_paged_rows* pr, int k) {
+    if (pr == nullptr || k < 1) return IC_STATUS_BYTES;
+    return IC_STATUS_BYTES + align_up(attn_tc_scratch_bytes(plan_rows(pr), k));
+}
+
+ic_status ic_sparse_attn_paged(const void* q, const void* kv_pages, const int32_t* idx, int k,
+                               const ic_paged_rows* pr, float scale, void* out, void* ws,
+                               size_t ws_bytes, void* stream) {
+    if (!paged_ok(pr, true) || k < 1 || k > 16384) return IC_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, ic_sparse_attn_paged_workspace_size(pr, k))) return IC_ERR_WORKSPACE;
+    if (pr->B == 0) return IC_OK;
+    if (!q || !kv_pages || !idx || !out) return IC_ERR_INVALID_ARG;
+    return launch_attn_tc_paged(q, kv_pages, idx, k, *pr, scale, out, status_of(ws),
+                                scratch_of(ws), ws_bytes - IC_STATUS_BYTES, (cudaStream_t)stream);
+}
+
+size_t ic_paged_workspace_size(const ic_stack_shape* sh, const ic_paged_rows* pr) {
+    if (sh == nullptr || pr == nullptr) return 0;
+    const ic_rows r = plan_rows(pr);
+    return IC_STATUS_BYTES + align_up(scores_bytes(r)) + align_up(attn_tc_scratch_bytes(r, sh->k));
+}
+
+ic_status ic_layer_stack_forward_paged(const char* pattern, int n_layers, const ic_layer_io* layers,
+                                       const ic_stack_shape* sh, const ic_paged_rows* pr,
+                                       int32_t* idx_buf, int32_t* const* idx_out, void* ws,
+                                       size_t ws_bytes, void* stream) {
+    if (pattern == nullptr || n_layers < 0) return IC_ERR_PATTERN;
+    if (strlen(pattern) != (size_t)n_layers) return IC_ERR_PATTERN;
+    for (int l = 0; l < n_layers; ++l)
+        if (pattern[l] != 'F' && pattern[l] != 'S') return IC_ERR_PATTERN;
+    if (n_layers > 0 && pattern[0] != 'F') return IC_ERR_PATTERN;
+    if (sh == nullptr || (n_layers > 0 && layers == nullptr)) return IC_ERR_INVALID_ARG;
+    if (!paged_ok(pr, true) || sh->k < 1 || sh->k > 16384) return IC_ERR_INVALID_ARG;
+    if (!latent_tc_shape(sh)) return IC_ERR_UNSUPPORTED;
+    if (!ws_ok(ws, ws_bytes, ic_paged_workspace_size(sh, pr))) return IC_ERR_WORKSPACE;
+    if (pr->B == 0 || n_layers == 0) return IC_OK;
+    if (idx_buf == nullptr) return IC_ERR_INVALID_ARG;
+    for (int l = 0; l < n_layers; ++l) {
+        const ic_layer_io& L = layers[l];
+        if (!L.q || !L.kmat || !L.out || (L.vmat && L.vmat != L.kmat)) return IC_ERR_INVALID_ARG;
+        if (pattern[l] == 'F') {
+            if (!L.q_idx || !L.w || !L.k_idx) return IC_ERR_INVALID_ARG;
+            const bool fp8 = sh->idx_dtype == IC_FP8_E4M3;
+            if (fp8 != (L.q_scale != nullptr) || fp8 != (L.k_scale != nullptr))
+                return IC_ERR_INVALID_ARG;
+        }
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t* status = status_of(ws);
+    const ic_rows r = plan_rows(pr);
+    float* scores = reinterpret_cast<float*>(scratch_of(ws));
+    const int64_t ld = ((int64_t)r.T + 3) / 4 * 4;
+    char* attn_ws = scratch_of(ws) + align_up(scores_bytes(r));
+    const size_t attn_ws_bytes = ws_bytes - IC_STATUS_BYTES - align_up(scores_bytes(r));
+    const size_t idx_bytes = (size_t)pr->B * pr->Lq * sh->k * sizeof(int32_t);
+    for (int l = 0; l < n_layers; ++l) {
+        const ic_layer_io& L = layers[l];
+        if (pattern[l] == 'F') {  // the one conditional branch of IndexCache
+            ic_status st = launch_indexer_tc_paged(L.q_idx, L.q_scale, L.w, L.k_idx, L.k_scale,
+                                                   sh->idx_dtype, *pr, sh->H_I, sh->d_I, scores,
+                                                   ld, status, s);
+            if (st != IC_OK) return st;
+            st = run_topk_varlen(scores, ld, pr, sh->k, idx_buf, s);
+            if (st != IC_OK) return st;
+        }
+        ic_status st = launch_attn_tc_paged(L.q, L.kmat, idx_buf, sh->k, *pr, sh->scale, L.out,
+                                            status, attn_ws, attn_ws_bytes, s);
         if (st != IC_OK) return st;
         if (idx_out != nullptr && idx_out[l] != nullptr) {
             if (cudaMemcpyAsync(idx_out[l], idx_buf, idx_bytes, cudaMemcpyDeviceToDevice, s) !=

@@ -13,12 +13,17 @@
 // splits the latent dimension evenly: CTA r gathers only its 288 columns of
 // every selected row (value columns 256r..256r+255 and rope columns
 // 512+32r..512+32r+31), computes the partial logits S_r = Q_r K_r^T on the
-// tensor core, scales them to base-2 units and swaps them with its partner
-// through distributed shared memory as float16.  Both CTAs add the two
-// halves in float32 (a commutative single rounding, so both get the very
-// same logits) and run the same online softmax.  Each then accumulates its
-// own 256 value columns, O_r += P V_r, in TMEM.  No key byte is gathered
-// twice and no flop is done twice.
+// tensor core, scales them to base-2 units and sends them to its partner
+// through distributed shared memory: per head, the block's largest valid
+// partial logit m as float16 and every partial logit's difference from m as
+// float16.  Near the row maximum, where the softmax weights are decided, the
+// differences are small, so the float16 rounding (2^-11 of the difference)
+// stays far inside the attention tolerance even for sharp logits of tens of
+// base-2 units.  Each CTA adds its own half in float32, straight from TMEM,
+// to the partner's reconstructed half and runs the online softmax; each then
+// accumulates its own 256 value columns, O_r += P V_r, in TMEM, normalised by
+// its own softmax sum.  No key byte is gathered twice and no flop is done
+// twice.
 //
 // Per CTA (448 threads), persistent over work units (one unit = one query
 // row, or one split of a row's indices in decode):
@@ -31,12 +36,12 @@
 //   warps 4-7  exchange (thread = head = TMEM lane): at the start of a unit,
 //              the unit's Q_r columns that the S MMA reads from TMEM (value
 //              slice 3 and the 32 rope columns); per 64-key block, partial S
-//              from TMEM -> base-2 float16, sent straight into the partner's
-//              inbox with st.async (counted in bytes on the partner's
-//              mbarrier) and stored back into TMEM for the softmax warps;
-//              they run ahead of the softmax warps, so the exchange latency
-//              of block j+1 hides behind the softmax of block j;
-//   warps 8-11 softmax (thread = head): own + partner logits, row max,
+//              from TMEM -> base 2 -> (block maximum, float16 differences),
+//              sent straight into the partner's inbox with st.async (counted
+//              in bytes on the partner's mbarrier); they run ahead of the
+//              softmax warps, so the exchange latency of block j+1 hides
+//              behind the softmax of block j;
+//   warps 8-11 softmax (thread = head): own (float32) + partner logits, row max,
 //              online softmax in base 2 with lazy rescaling (O is rescaled
 //              only when the running max grows by more than 2^8), P as bf16
 //              into TMEM over the S columns, the row sum l of the same
@@ -53,12 +58,12 @@
 // rope columns at 448..495.  Keeping that part of Q_r in TMEM frees the
 // shared memory for a fourth KV stage.
 // Shared memory: Q_r slices 0-2 48 KB, 4 KV stages of 36 KB, 2 float16 inbox
-// tiles of 16 KB (written by the partner), per-unit masks, barriers
-// (~226 KB).
+// tiles of 16 KB + 256 B of per-head offsets (written by the partner),
+// per-unit masks, barriers (~227 KB).
 //
 // Decode (few query rows): each row's k indices are split over several CTA
-// pairs, which write unnormalised (O, m, l) partials; a small combine kernel
-// merges them by log-sum-exp.
+// pairs, which write unnormalised (O, m, l) partials, (m, l) per CTA half;
+// a small combine kernel merges them by log-sum-exp.
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 
@@ -81,15 +86,18 @@ constexpr int KV_ROPE = NB * 64;     // the 32 rope columns of a key block
 constexpr int KV_STAGE = 4 * KV_ATOM + KV_ROPE;     // 36 KB
 constexpr int NSTAGE = 4;
 constexpr int NSBUF = 3;                            // S/P buffers in TMEM
-constexpr int X_TILE = HQ * NB * 2;                 // 16 KB of float16 logits
+constexpr int X_TILE = HQ * NB * 2;                 // 16 KB of float16 logit differences
 constexpr int X_QUAD = X_TILE / 4;                  // the 32 rows of one TMEM lane quadrant
+constexpr int X_OFF = HQ * 2;                       // per-head float16 offsets of one inbox slot
+constexpr int X_OFF_QUAD = X_OFF / 4;
 constexpr int MAX_UNIT_BLOCKS = 32;                 // at most 2048 indices per unit
 constexpr int Q_SMEM_ATOMS = 3;                     // value slices 0-2 of Q_r in shared memory;
                                                     // slice 3 and the rope columns live in TMEM
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = Q_SMEM_ATOMS * Q_ATOM;       // 48 KB
-constexpr int OFF_X = OFF_KV + NSTAGE * KV_STAGE;   // partner's float16 logits
-constexpr int OFF_MASK = OFF_X + 2 * X_TILE;
+constexpr int OFF_X = OFF_KV + NSTAGE * KV_STAGE;   // partner's float16 logit differences
+constexpr int OFF_XOFF = OFF_X + 2 * X_TILE;        // partner's float16 per-head offsets
+constexpr int OFF_MASK = OFF_XOFF + 2 * X_OFF;
 constexpr int OFF_BARS = OFF_MASK + 2 * MAX_UNIT_BLOCKS * 8;
 constexpr int GW = 4;                               // gather warps
 constexpr int KPW = NB / GW;                        // key rows of a block per gather warp
@@ -109,7 +117,7 @@ struct __align__(8) AttnBars {
     uint64_t q_full, q_empty, q_tmem_full;
     uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
     uint64_t s_full[NSBUF], s_free[NSBUF];
-    uint64_t own_full[NSBUF][4];    // exchange warp q -> softmax warp q: own float16 logits in TMEM
+    uint64_t own_full[NSBUF][4];    // exchange warp q has read S of the buffer: P may overwrite it
     uint64_t p_full[NSBUF];         // softmax warps -> MMA: P in TMEM
     uint64_t x_full[2][4];          // [inbox slot][quad]: the partner's 32 rows (counted in bytes)
     uint64_t peer_free[2][4];       // the partner's softmax warp q has read its inbox slot
@@ -154,12 +162,19 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     return d;
 }
 
-// both logits of a key pair: own (float16 pair) + partner (float16 pair)
-__device__ __forceinline__ void sum_pair(uint32_t own, uint32_t par, float& s0, float& s1) {
-    const float o0 = __half2float(__ushort_as_half((unsigned short)(own & 0xffffu)));
-    const float o1 = __half2float(__ushort_as_half((unsigned short)(own >> 16)));
-    s0 = add_f16_f32((unsigned short)(par & 0xffffu), o0);
-    s1 = add_f16_f32((unsigned short)(par >> 16), o1);
+// float16 -> float32 of the low / high half of a packed pair
+__device__ __forceinline__ float f16_lo(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v & 0xffffu))); }
+__device__ __forceinline__ float f16_hi(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
+
+// largest of 64 values
+__device__ __forceinline__ float max64(const float (&v)[NB]) {
+    float mx[21];
+#pragma unroll
+    for (int x = 0; x < 21; ++x) mx[x] = max3(v[3 * x], v[3 * x + 1], v[3 * x + 2]);
+    float m = max3(mx[0], mx[1], v[63]);
+#pragma unroll
+    for (int x = 2; x + 1 < 21; x += 2) m = max3(m, mx[x], mx[x + 1]);
+    return fmaxf(m, mx[20]);
 }
 
 struct AttnArgs {
@@ -167,12 +182,19 @@ struct AttnArgs {
     const __nv_bfloat16* kv;
     const int32_t* idx;
     __nv_bfloat16* out;
-    float* part_o;      // [units][128][512] (split-k only)
-    float2* part_ml;    // [units][128]      (split-k only)
+    float* part_o;      // [units][128][512]   (split-k only)
+    float2* part_ml;    // [units][2][128]     (split-k only; (m, l) of each CTA half)
     uint32_t* status;
     int k, B, Lq, q_start, T;
     int splits, keys_per_split, n_units;
     float scale_log2;
+    // KV rows: dense (seq_lens == nullptr) at b*T + s; paged at
+    // block_table[b*max_pages + s/page_size]*page_size + s%page_size, with
+    // per-sequence lengths (queries at seq_lens[b] - Lq + i, T = the upper bound)
+    const int32_t* seq_lens;
+    const int32_t* block_table;
+    int max_pages, page_size, num_pages;
+    int kv_rows;        // rows of the KV tensor map; row kv_rows is the zero-filled stand-in
 };
 
 struct Unit {
@@ -185,10 +207,30 @@ __device__ __forceinline__ Unit decode_unit(const AttnArgs& a, int seq) {
     u.row = u.unit / a.splits;
     const int split = u.unit - u.row * a.splits;
     u.b = u.row / a.Lq;
-    u.t = a.q_start + (u.row - u.b * a.Lq);
+    const int i = u.row - u.b * a.Lq;
+    if (a.seq_lens == nullptr) {
+        u.t = a.q_start + i;
+    } else {
+        // a length outside [Lq, T] leaves the row without a valid index
+        const int Tb = __ldg(a.seq_lens + u.b);
+        u.t = (Tb >= a.Lq && Tb <= a.T) ? Tb - a.Lq + i : -1;
+    }
     u.e0 = split * a.keys_per_split;
     u.e1 = min(a.k, u.e0 + a.keys_per_split);
     return u;
+}
+
+// KV tensor-map row of key position v of sequence b (v already checked to
+// lie in [0, t]); a page outside [0, num_pages) gives the zero-filled row and
+// the index-range status bit.
+__device__ __forceinline__ int kv_row(const AttnArgs& a, int b, int v) {
+    if (a.seq_lens == nullptr) return b * a.T + v;
+    const int page = __ldg(a.block_table + (int64_t)b * a.max_pages + v / a.page_size);
+    if (page < 0 || page >= a.num_pages) {
+        flag_status(a.status, IC_DEV_INDEX_RANGE);
+        return a.kv_rows;
+    }
+    return page * a.page_size + v % a.page_size;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(N_THREADS, 1)
@@ -301,7 +343,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             // L < KPW holds the row of key KPW*w + L (the indices of block j+1
             // are loaded while block j is issued).  An invalid index becomes
             // the out-of-range row B*T, which TMA fills with zeros.
-            const int oob_row = args.B * args.T;
+            const int oob_row = args.kv_rows;
             bool ok_all = true;
             const int key = warp * KPW + lane;
             int v_next = (lane < KPW && u.e0 + key < u.e1) ? idx_row[u.e0 + key] : -1;
@@ -312,7 +354,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     const int e1 = u.e0 + (j + 1) * NB + key;
                     v_next = (lane < KPW && e1 < u.e1) ? idx_row[e1] : -1;
                 }
-                const int row_lane = idx_valid(v_lane, u.t, args.T) ? u.b * args.T + v_lane : oob_row;
+                const int row_lane = idx_valid(v_lane, u.t, args.T) ? kv_row(args, u.b, v_lane) : oob_row;
                 if (!warp_wait(&bars->kv_empty[s], ((g / NSTAGE) & 1) ^ 1, status, abort)) {
                     ok_all = false;
                     break;
@@ -351,6 +393,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         const int h = quad * 32 + lane;           // head of this thread
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t x_remote = map_to_rank(smem_base + OFF_X + h * 128, peer);
+        const uint32_t xoff_remote = map_to_rank(smem_base + OFF_XOFF + (h >> 1) * 4, peer);
+        const float sl2 = args.scale_log2;
         uint32_t g = 0;
         int n = 0;
         bool ok = true;
@@ -359,7 +403,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             if (!warp_wait(&bars->info_full[ip], (n >> 1) & 1, status, abort)) break;
             const int nb = bars->n_blocks[ip];
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->info_empty[ip]);
             if (nb > 0) {
                 // Q_r columns the S MMA reads from TMEM (value slice 3 and the rope
                 // columns), row h, packed as bf16 pairs.  Every S MMA of the previous
@@ -389,41 +432,65 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 const int slot = g & 1;
                 if (!warp_wait(&bars->s_full[sb], (g / NSBUF) & 1, status, abort)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t own[NB / 2];
+                float x[NB];
                 {
                     uint32_t r0[32], r1[32];
                     tmem_ld32(t_lane + TM_S + 64 * sb, r0);
                     tmem_ld32(t_lane + TM_S + 64 * sb + 32, r1);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        own[x] = half2_sat(__uint_as_float(r0[2 * x]) * args.scale_log2,
-                                           __uint_as_float(r0[2 * x + 1]) * args.scale_log2);
-                        own[16 + x] = half2_sat(__uint_as_float(r1[2 * x]) * args.scale_log2,
-                                                __uint_as_float(r1[2 * x + 1]) * args.scale_log2);
+                    for (int c = 0; c < 32; ++c) {
+                        x[c] = __uint_as_float(r0[c]) * sl2;
+                        x[32 + c] = __uint_as_float(r1[c]) * sl2;
                     }
                 }
-                // own float16 logits for the softmax warp of this quadrant (the
-                // store completes while the partner's copy is sent)
-                tmem_st32(t_lane + TM_S + 64 * sb + 32, own);
-                // the partner's softmax warp must have read this inbox slot (block g-2)
+                // S(g) is in registers: the softmax warp of this quadrant may now
+                // read it and overwrite it with P
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
+                // the offset is the largest VALID partial logit of the block (keys
+                // of invalid indices are zero rows whose logits would pull it off)
+                const uint32_t m_lo = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j];
+                const uint32_t m_hi = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j + 1];
+                float mb;
+                if ((m_lo & m_hi) != 0xffffffffu) {
+                    float xm[NB];
+#pragma unroll
+                    for (int c = 0; c < NB; ++c)
+                        xm[c] = (((c < 32 ? m_lo : m_hi) >> (c & 31)) & 1u) ? x[c] : -INFINITY;
+                    mb = max64(xm);
+                } else {
+                    mb = max64(x);
+                }
+                // offset as float16 (saturated); the differences are taken from
+                // the rounded offset, so offset + difference rebuilds the value
+                const uint32_t m16 = half2_sat(mb, 0.f) & 0xffffu;
+                const float mf = f16_lo(m16);
+                uint32_t d[NB / 2];
+#pragma unroll
+                for (int c = 0; c < NB / 2; ++c) d[c] = half2_sat(x[2 * c] - mf, x[2 * c + 1] - mf);
+                // two heads' offsets per 32-bit word: lane 2i sends heads 2i, 2i+1
+                const uint32_t m16_odd = __shfl_down_sync(0xffffffffu, m16, 1);
+                // the partner's softmax warp q must have read this inbox slot (block g-2)
                 if (!warp_wait_cluster(&bars->peer_free[slot][quad], ((g >> 1) & 1) ^ 1, status, abort)) {
                     ok = false;
                     break;
                 }
-                // row h of the partner's inbox; each 16-byte st.async counts its
-                // bytes on the partner's x_full (no fence or arrive on this side)
+                // row h of the partner's inbox; each st.async counts its bytes on
+                // the partner's x_full (no fence or arrive on this side)
                 const uint32_t xr = x_remote + slot * X_TILE;
                 const uint32_t br = map_to_rank(smem_u32(&bars->x_full[slot][quad]), peer);
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
-                    st_async_v4(xr + ((c ^ (h & 7)) << 4), own[4 * c], own[4 * c + 1], own[4 * c + 2],
-                                own[4 * c + 3], br);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
+                    st_async_v4(xr + ((c ^ (h & 7)) << 4), d[4 * c], d[4 * c + 1], d[4 * c + 2],
+                                d[4 * c + 3], br);
+                if ((lane & 1) == 0)
+                    st_async_b32(xoff_remote + slot * X_OFF, m16 | (m16_odd << 16), br);
             }
+            // the unit's masks have been read: the gather warps may refill them
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->info_empty[ip]);
         }
     } else if (warp < W_S) {
         // ------------------------------------------------------------ softmax
@@ -446,20 +513,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             for (int j = 0; j < nb; ++j, ++g) {
                 const int sb = g % NSBUF;
                 const int slot = g & 1;
-                if (lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD);
+                if (lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD + X_OFF_QUAD);
                 const uint32_t m_lo = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j];
                 const uint32_t m_hi = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j + 1];
+                // S(g) is final in TMEM and the exchange warp has read it
                 if (!warp_wait(&bars->own_full[sb][quad], (g / NSBUF) & 1, status, abort)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                uint32_t own[NB / 2], par[NB / 2];
-                tmem_ld32(t_lane + TM_S + 64 * sb + 32, own);
+                uint32_t s0[32], s1[32], par[NB / 2];
+                tmem_ld32(t_lane + TM_S + 64 * sb, s0);
+                tmem_ld32(t_lane + TM_S + 64 * sb + 32, s1);
                 if (!warp_wait_cluster(&bars->x_full[slot][quad], (g >> 1) & 1, status, abort)) {
                     ok = false;
                     break;
                 }
+                float pf;
                 {
                     const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + slot * X_TILE + h * 128);
 #pragma unroll
@@ -470,12 +540,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                         par[4 * c + 2] = w4.z;
                         par[4 * c + 3] = w4.w;
                     }
+                    const uint32_t ow = reinterpret_cast<const uint32_t*>(smem + OFF_XOFF + slot * X_OFF)[h >> 1];
+                    pf = (h & 1) ? f16_hi(ow) : f16_lo(ow);
                 }
                 tmem_ld_wait();
-                // full logits of the 64 keys (log2 units), masked keys -> -inf
+                // full logits of the 64 keys (log2 units): own half in float32 plus
+                // the partner's (offset + float16 difference); masked keys -> -inf
                 float sv[NB];
 #pragma unroll
-                for (int x = 0; x < NB / 2; ++x) sum_pair(own[x], par[x], sv[2 * x], sv[2 * x + 1]);
+                for (int c = 0; c < NB / 2; ++c) {
+                    sv[c] = fmaf(__uint_as_float(s0[c]), args.scale_log2,
+                                 add_f16_f32((unsigned short)((c & 1) ? (par[c >> 1] >> 16) : (par[c >> 1] & 0xffffu)), pf));
+                    sv[32 + c] = fmaf(__uint_as_float(s1[c]), args.scale_log2,
+                                      add_f16_f32((unsigned short)((c & 1) ? (par[16 + (c >> 1)] >> 16)
+                                                                           : (par[16 + (c >> 1)] & 0xffffu)), pf));
+                }
                 if ((m_lo & m_hi) != 0xffffffffu) {
 #pragma unroll
                     for (int kk = 0; kk < NB; ++kk) {
@@ -483,13 +562,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                         if (!((mw >> (kk & 31)) & 1u)) sv[kk] = -INFINITY;
                     }
                 }
-                float mx[21];
-#pragma unroll
-                for (int x = 0; x < 21; ++x) mx[x] = max3(sv[3 * x], sv[3 * x + 1], sv[3 * x + 2]);
-                float mloc = max3(mx[0], mx[1], sv[63]);
-#pragma unroll
-                for (int x = 2; x + 1 < 21; x += 2) mloc = max3(mloc, mx[x], mx[x + 1]);
-                mloc = fmaxf(mloc, mx[20]);
+                const float mloc = max64(sv);
                 // every inbox value of this slot has been consumed (mloc depends on
                 // all of them): hand the slot back to the partner's exchange warp
                 __syncwarp();
@@ -576,7 +649,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 uint4* dst = reinterpret_cast<uint4*>(args.out + ((int64_t)u.row * HQ + h) * DV + r * 256);
                 for (int v = 0; v < 32; ++v) dst[v] = make_uint4(0, 0, 0, 0);
             }
-            if (split && r == 0) args.part_ml[(int64_t)u.unit * HQ + h] = make_float2(m_use, l_all);
+            // each CTA half keeps its own (m, l): the two CTAs' logits differ by
+            // rounding, so their running maxima and sums may differ slightly
+            if (split) args.part_ml[((int64_t)u.unit * 2 + r) * HQ + h] = make_float2(m_use, l_all);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->info_empty[ip]);
         }
@@ -723,16 +798,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
     }
 }
 
-// Merge split-k partials: out = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c.
+// Merge split-k partials: out = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c,
+// with (m_c, l_c) of the CTA half that produced the columns.
 __global__ void __launch_bounds__(128)
 attn_combine_kernel(const float* __restrict__ part_o, const float2* __restrict__ part_ml,
                     int splits, __nv_bfloat16* __restrict__ out) {
     const int64_t row = blockIdx.x;
     const int h = blockIdx.y;
     const int d = threadIdx.x * 4;
+    const int half = d / 256;
     float M = -INFINITY;
     for (int c = 0; c < splits; ++c) {
-        const float2 ml = part_ml[(row * splits + c) * HQ + h];
+        const float2 ml = part_ml[((row * splits + c) * 2 + half) * HQ + h];
         if (ml.y > 0.f) M = fmaxf(M, ml.x);
     }
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -740,7 +817,7 @@ attn_combine_kernel(const float* __restrict__ part_o, const float2* __restrict__
     if (M > -INFINITY) {
         for (int c = 0; c < splits; ++c) {
             const int64_t u = row * splits + c;
-            const float2 ml = part_ml[u * HQ + h];
+            const float2 ml = part_ml[(u * 2 + half) * HQ + h];
             if (!(ml.y > 0.f)) continue;
             const float wgt = exp2f(ml.x - M);
             den += wgt * ml.y;
@@ -831,13 +908,16 @@ size_t attn_tc_scratch_bytes(ic_rows r, int k, int64_t max_units) {
     plan_splits(r, k, splits, kps, max_units);
     if (splits <= 1) return 0;
     const size_t units = (size_t)r.B * r.Lq * splits;
-    return units * HQ * DV * sizeof(float) + 256 + units * HQ * sizeof(float2);
+    return units * HQ * DV * sizeof(float) + 256 + units * 2 * HQ * sizeof(float2);
 }
 
-ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_t* idx, int k,
-                         ic_rows r, float scale, void* out, uint32_t* status, void* scratch,
-                         size_t scratch_bytes, cudaStream_t s, int64_t max_units) {
-    (void)ks;
+namespace {
+
+// r: planning rows (dense: the call's rows; paged: every sequence T_max long).
+ic_status attn_tc_core(const void* q, const void* kv, const int32_t* idx, int k, ic_rows r,
+                       float scale, void* out, uint32_t* status, void* scratch,
+                       size_t scratch_bytes, cudaStream_t s, int64_t max_units,
+                       const ic_paged_rows* pr) {
     if (((uintptr_t)q & 15) || ((uintptr_t)kv & 15) || ((uintptr_t)out & 15))
         return IC_ERR_INVALID_ARG;
     auto fn = encode_fn();
@@ -854,11 +934,12 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
 
     // KV rows for the gathers: one box row of 64 value columns (128-byte
     // swizzle) or of the 32 rope columns (64-byte swizzle)
+    const int64_t kv_rows = pr ? (int64_t)pr->num_pages * pr->page_size : (int64_t)r.B * r.T;
+    if (kv_rows >= 0x7fffffff) return IC_ERR_UNSUPPORTED;
     CUtensorMap map_kv, map_kvr;
-    cuuint64_t kdims[2] = {(cuuint64_t)KVW, (cuuint64_t)r.B * r.T};
+    cuuint64_t kdims[2] = {(cuuint64_t)KVW, (cuuint64_t)kv_rows};
     cuuint32_t kbox[2] = {64, 1};
     cuuint32_t kbox_r[2] = {32, 1};
-    if ((int64_t)r.B * r.T >= 0x7fffffff) return IC_ERR_UNSUPPORTED;
     if (fn(&map_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv), kdims, strides, kbox,
            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -880,6 +961,12 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
     a.q_start = r.q_start;
     a.T = r.T;
     a.scale_log2 = scale * LOG2E;
+    a.seq_lens = pr ? pr->seq_lens : nullptr;
+    a.block_table = pr ? pr->block_table : nullptr;
+    a.max_pages = pr ? pr->max_pages : 0;
+    a.page_size = pr ? pr->page_size : 1;
+    a.num_pages = pr ? pr->num_pages : 0;
+    a.kv_rows = (int)kv_rows;
     plan_splits(r, k, a.splits, a.keys_per_split, max_units);
     const int64_t units = (int64_t)r.B * r.Lq * a.splits;
     if (2 * units > 0x7fffffff) return IC_ERR_UNSUPPORTED;
@@ -907,6 +994,24 @@ ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_
                                              static_cast<__nv_bfloat16*>(out));
     count_launch(IC_LK_COMBINE);
     return last_launch_status();
+}
+
+}  // namespace
+
+ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_t* idx, int k,
+                         ic_rows r, float scale, void* out, uint32_t* status, void* scratch,
+                         size_t scratch_bytes, cudaStream_t s, int64_t max_units) {
+    (void)ks;
+    return attn_tc_core(q, kv, idx, k, r, scale, out, status, scratch, scratch_bytes, s, max_units,
+                        nullptr);
+}
+
+ic_status launch_attn_tc_paged(const void* q, const void* kv_pages, const int32_t* idx, int k,
+                               const ic_paged_rows& pr, float scale, void* out, uint32_t* status,
+                               void* scratch, size_t scratch_bytes, cudaStream_t s) {
+    const ic_rows r = {pr.B, pr.Lq, pr.T_max - pr.Lq, pr.T_max};
+    return attn_tc_core(q, kv_pages, idx, k, r, scale, out, status, scratch, scratch_bytes, s,
+                        kNoUnitLimit, &pr);
 }
 
 }  // namespace ic

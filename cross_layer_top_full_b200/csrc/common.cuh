@@ -61,8 +61,14 @@ ic_status launch_indexer_tc(const void* q_idx, const float* q_scale, const float
                             int H_I, int d_I, float* scores, int64_t ld, uint32_t* status,
                             cudaStream_t s);
 
+// seq_lens: nullptr (every row of sequence b has q_start + i + 1 candidates)
+// or [B] per-sequence key counts (row i: seq_lens[b] - Lq + i + 1; r.T is
+// then the upper bound T_max and r.q_start = T_max - Lq).
 ic_status launch_topk_rows(const float* scores, int64_t ld, ic_rows r, int k, int32_t* idx,
-                           cudaStream_t s);
+                           cudaStream_t s, const int32_t* seq_lens = nullptr);
+bool topk_cluster_applies(ic_rows r, int k);
+ic_status launch_topk_cluster(const float* scores, int64_t ld, ic_rows r, int k, int32_t* idx,
+                              cudaStream_t s, const int32_t* seq_lens = nullptr);
 bool topk_multi_applies(ic_rows r, int k);
 size_t topk_multi_scratch_bytes(ic_rows r, int k);
 ic_status launch_topk_multi(const float* scores, int64_t ld, ic_rows r, int k, int32_t* idx,
@@ -84,5 +90,15 @@ size_t attn_tc_scratch_bytes(ic_rows r, int k, int64_t max_units = kNoUnitLimit)
 ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_t* idx, int k,
                          ic_rows r, float scale, void* out, uint32_t* status, void* scratch,
                          size_t scratch_bytes, cudaStream_t s, int64_t max_units = kNoUnitLimit);
+
+// Paged / variable-length variants (ic_paged_rows: per-sequence lengths and a
+// block table; see include/indexcache.h).
+ic_status launch_indexer_tc_paged(const void* q_idx, const float* q_scale, const float* w,
+                                  const void* k_pages, const float* k_scale_pages, ic_dtype dt,
+                                  const ic_paged_rows& pr, int H_I, int d_I, float* scores,
+                                  int64_t ld, uint32_t* status, cudaStream_t s);
+ic_status launch_attn_tc_paged(const void* q, const void* kv_pages, const int32_t* idx, int k,
+                               const ic_paged_rows& pr, float scale, void* out, uint32_t* status,
+                               void* scratch, size_t scratch_bytes, cudaStream_t s);
 
 }  // namespace ic

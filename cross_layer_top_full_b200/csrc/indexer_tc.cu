@@ -66,6 +66,43 @@ struct Work {
     int n_groups, n_chunks, chunk_tiles, n_items;
 };
 
+// Where the keys of sequence b live.  Dense: rows b*T .. b*T + T-1 of k_I,
+// every sequence T keys, queries from q_start.  Paged: sequence b has
+// seq_lens[b] keys, its queries start at seq_lens[b] - Lq, and key position
+// s is row block_table[b*max_pages + s/page_size]*page_size + s%page_size
+// (page_size a multiple of the 128-key tile, so a tile never straddles pages).
+struct Paging {
+    const int32_t* seq_lens;      // nullptr: dense
+    const int32_t* block_table;
+    int max_pages, page_size, T_max;
+    int64_t key_rows;             // rows of k_I (and of k_scale)
+};
+
+// This sequence's first query position and key count; false (and the
+// index-range status bit) for a length outside [Lq, T_max].
+__device__ __forceinline__ bool seq_extent(const Paging& pg, int b, int Lq, int q_start, int T,
+                                           int& qs, int& Tb) {
+    if (pg.seq_lens == nullptr) {
+        qs = q_start;
+        Tb = T;
+        return true;
+    }
+    Tb = __ldg(pg.seq_lens + b);
+    qs = Tb - Lq;
+    return Tb >= Lq && Tb <= pg.T_max;
+}
+
+// First k_I row of the 128-key tile starting at logical key position s0.  A
+// block-table entry outside the cache gives key_rows: the tile then lies
+// past the end of the tensor map, which TMA fills with zeros, and its keys
+// are dropped from the score row.
+__device__ __forceinline__ int64_t key_row(const Paging& pg, int b, int T, int s0) {
+    if (pg.seq_lens == nullptr) return (int64_t)b * T + s0;
+    const int page = __ldg(pg.block_table + (int64_t)b * pg.max_pages + s0 / pg.page_size);
+    if (page < 0 || (int64_t)page * pg.page_size >= pg.key_rows) return pg.key_rows;
+    return (int64_t)page * pg.page_size + s0 % pg.page_size;
+}
+
 struct __align__(8) Bars {
     uint64_t a_full[8], a_empty[8];
     uint64_t b_full, b_empty;
@@ -76,15 +113,17 @@ struct __align__(8) Bars {
 };
 
 __device__ __forceinline__ bool decode_item(int id, const Work& wk, int B, int Lq, int q_start,
-                                            int ntok, int& b, int& i0, int& kt0, int& kt1) {
+                                            int T, const Paging& pg, int ntok, int& b, int& i0,
+                                            int& kt0, int& kt1, int& qs, int& Tb) {
     const int per_group = B * wk.n_chunks;
     const int g = wk.n_groups - 1 - id / per_group;   // heaviest (latest) group first
     const int rem = id - (wk.n_groups - 1 - g) * per_group;
     b = rem / wk.n_chunks;
     const int c = rem - b * wk.n_chunks;
     i0 = g * ntok;
+    if (!seq_extent(pg, b, Lq, q_start, T, qs, Tb)) return false;
     const int i_last = min(i0 + ntok, Lq) - 1;
-    const int tiles = (q_start + i_last + 1 + BM - 1) / BM;
+    const int tiles = (qs + i_last + 1 + BM - 1) / BM;
     kt0 = c * wk.chunk_tiles;
     kt1 = min(kt0 + wk.chunk_tiles, tiles);
     return kt0 < kt1;
@@ -95,7 +134,7 @@ __global__ void __launch_bounds__(N_THREADS, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                   const float* __restrict__ w, const float* __restrict__ q_scale,
                   const float* __restrict__ k_scale, float* __restrict__ scores, int64_t ld, int B,
-                  int Lq, int q_start, int T, Work wk, uint32_t* status) {
+                  int Lq, int q_start, int T, Work wk, Paging pg, uint32_t* status) {
     using C = Cfg<H, NTOK, FP8>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
@@ -153,8 +192,13 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
                 return true;
             };
             for (int id = blockIdx.x; id < wk.n_items; id += gridDim.x) {
-                int b, i0, kt0, kt1;
-                if (!decode_item(id, wk, B, Lq, q_start, NTOK, b, i0, kt0, kt1)) continue;
+                int b, i0, kt0, kt1, qs, Tb;
+                if (!decode_item(id, wk, B, Lq, q_start, T, pg, NTOK, b, i0, kt0, kt1, qs, Tb)) {
+                    // a paged sequence whose length is out of range has no keys
+                    if (pg.seq_lens != nullptr && !(Tb >= Lq && Tb <= pg.T_max))
+                        flag_status(status, IC_DEV_INDEX_RANGE);
+                    continue;
+                }
                 // The first key tiles of the item go out before the query block:
                 // they only need free ring slots, which the previous item's MMAs
                 // release, so they overlap its tail.
@@ -169,7 +213,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
                     if (!mbar_wait(&bars->a_empty[s], ph ^ 1, status, abort)) { ok = false; break; }
                     mbar_arrive_expect_tx(&bars->a_full[s], C::A_BYTES);
                     uint8_t* dst = a_smem + s * C::A_BYTES;
-                    const int krow = b * T + kt * BM;
+                    const int krow = (int)key_row(pg, b, T, kt * BM);
                     for (int a = 0; a < C::ATOMS; ++a)
                         tma_load_2d(dst + a * (BM * 128), &map_k, &bars->a_full[s],
                                     a * (128 / C::ESZ), krow);
@@ -190,8 +234,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
             const uint32_t a_base = smem_u32(a_smem), b_base = smem_u32(b_smem);
             bool issued = false;
             for (int id = blockIdx.x; id < wk.n_items; id += gridDim.x) {
-                int b, i0, kt0, kt1;
-                if (!decode_item(id, wk, B, Lq, q_start, NTOK, b, i0, kt0, kt1)) continue;
+                int b, i0, kt0, kt1, qs, Tb;
+                if (!decode_item(id, wk, B, Lq, q_start, T, pg, NTOK, b, i0, kt0, kt1, qs, Tb)) continue;
                 if (!mbar_wait(&bars->b_full, b_it & 1, status, abort)) break;
                 bool ok = true;
                 for (int kt = kt0; kt < kt1; ++kt, ++a_it, ++acc_it) {
@@ -236,8 +280,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
         if (group < C::EPI_GROUPS) {
             uint32_t acc_it = 0;
             for (int id = blockIdx.x; id < wk.n_items; id += gridDim.x) {
-                int b, i0, kt0, kt1;
-                if (!decode_item(id, wk, B, Lq, q_start, NTOK, b, i0, kt0, kt1)) continue;
+                int b, i0, kt0, kt1, qs, Tb;
+                if (!decode_item(id, wk, B, Lq, q_start, T, pg, NTOK, b, i0, kt0, kt1, qs, Tb)) continue;
                 // stage this item's head weights (and query scales) of my tokens
                 // in this warp's own buffer: only the warp itself reads it
                 float* w_w = w_smem + ew * C::TOK_PER_GROUP * H;
@@ -288,8 +332,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
                     if (lane == 0) mbar_arrive(&bars->acc_empty[acc]);   // TMEM free again
 
                     const int s = kt * BM + quad * 32 + lane;
+                    const int64_t krow0 = key_row(pg, b, T, kt * BM);
+                    const bool key_ok = krow0 < pg.key_rows;
+                    if (!key_ok && lane == 0 && quad == 0) flag_status(status, IC_DEV_INDEX_RANGE);
                     float ks = 1.f;
-                    if (FP8 && s < T) ks = k_scale[(int64_t)b * T + s];
+                    if (FP8 && s < Tb && key_ok) ks = k_scale[krow0 + quad * 32 + lane];
 #pragma unroll
                     for (int jj = 0; jj < C::TOK_PER_GROUP; ++jj) {
                         const int j = tok0 + jj;
@@ -306,8 +353,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
                         }
                         float sc = acc0 + acc1;
                         if (FP8) sc *= qs_w[jj] * ks;
-                        if (i < Lq && s <= q_start + i)
-                            scores[((int64_t)b * Lq + i) * ld + s] = sc;
+                        if (i < Lq && s <= qs + i)
+                            scores[((int64_t)b * Lq + i) * ld + s] = key_ok ? sc : -INFINITY;
                     }
                 }
                 if (!ok) break;
@@ -368,13 +415,14 @@ int num_sms() {
 template <int H, int NTOK, bool FP8>
 ic_status launch_cfg(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                      const float* k_scale, ic_rows r, float* scores, int64_t ld, uint32_t* status,
-                     cudaStream_t s) {
+                     cudaStream_t s, const Paging& pg, int64_t key_rows) {
     using C = Cfg<H, NTOK, FP8>;
     CUtensorMap map_k, map_q;
-    if (!make_map(&map_k, k_idx, (int64_t)r.B * r.T, FP8, BM)) return cuda_error("indexer_tc");
+    if (!make_map(&map_k, k_idx, key_rows, FP8, BM)) return cuda_error("indexer_tc");
     if (!make_map(&map_q, q_idx, (int64_t)r.B * r.Lq * H, FP8, C::N)) return cuda_error("indexer_tc");
     Work wk;
     wk.n_groups = ceil_div(r.Lq, NTOK);
+    // dense: the last row's candidates; paged: the longest possible sequence
     const int max_tiles = ceil_div(r.q_start + r.Lq, BM);
     const int base_items = r.B * wk.n_groups;
     const int sms = num_sms();
@@ -393,7 +441,7 @@ ic_status launch_cfg(const void* q_idx, const float* q_scale, const float* w, co
         return cuda_error("indexer_tc");
     const int grid = (int)std::min<int64_t>(items, sms);
     kern<<<grid, N_THREADS, smem, s>>>(map_k, map_q, w, q_scale, k_scale, scores, ld, r.B, r.Lq,
-                                       r.q_start, r.T, wk, status);
+                                       r.q_start, r.T, wk, pg, status);
     count_launch(IC_LK_INDEXER_TC);
     return last_launch_status();
 }
@@ -401,11 +449,34 @@ ic_status launch_cfg(const void* q_idx, const float* q_scale, const float* w, co
 template <int H, bool FP8>
 ic_status launch_h(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                    const float* k_scale, ic_rows r, float* scores, int64_t ld, uint32_t* status,
-                   cudaStream_t s) {
+                   cudaStream_t s, const Paging& pg, int64_t key_rows) {
     constexpr int NT_WIDE = 256 / H;
     if (r.Lq <= 2)  // decode: one token per accumulator, the scan is HBM-bound
-        return launch_cfg<H, 1, FP8>(q_idx, q_scale, w, k_idx, k_scale, r, scores, ld, status, s);
-    return launch_cfg<H, NT_WIDE, FP8>(q_idx, q_scale, w, k_idx, k_scale, r, scores, ld, status, s);
+        return launch_cfg<H, 1, FP8>(q_idx, q_scale, w, k_idx, k_scale, r, scores, ld, status, s,
+                                     pg, key_rows);
+    return launch_cfg<H, NT_WIDE, FP8>(q_idx, q_scale, w, k_idx, k_scale, r, scores, ld, status,
+                                       s, pg, key_rows);
+}
+
+ic_status launch_any(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
+                     const float* k_scale, ic_dtype dt, ic_rows r, int H_I, float* scores,
+                     int64_t ld, uint32_t* status, cudaStream_t s, const Paging& pg,
+                     int64_t key_rows) {
+    const bool fp8 = dt == IC_FP8_E4M3;
+#define IC_IDX_CASE(HH)                                                                         \
+    case HH:                                                                                    \
+        return fp8 ? launch_h<HH, true>(q_idx, q_scale, w, k_idx, k_scale, r, scores, ld,      \
+                                        status, s, pg, key_rows)                                \
+                   : launch_h<HH, false>(q_idx, q_scale, w, k_idx, k_scale, r, scores, ld,     \
+                                         status, s, pg, key_rows);
+    switch (H_I) {
+        IC_IDX_CASE(16)
+        IC_IDX_CASE(32)
+        IC_IDX_CASE(64)
+        IC_IDX_CASE(128)
+    }
+#undef IC_IDX_CASE
+    return IC_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -421,21 +492,23 @@ ic_status launch_indexer_tc(const void* q_idx, const float* q_scale, const float
                             cudaStream_t s) {
     if (!indexer_tc_supported(dt, H_I, d_I)) return IC_ERR_UNSUPPORTED;
     if (((uintptr_t)q_idx & 15) || ((uintptr_t)k_idx & 15)) return IC_ERR_INVALID_ARG;
-    const bool fp8 = dt == IC_FP8_E4M3;
-#define IC_IDX_CASE(HH)                                                                         \
-    case HH:                                                                                    \
-        return fp8 ? launch_h<HH, true>(q_idx, q_scale, w, k_idx, k_scale, r, scores, ld,      \
-                                        status, s)                                              \
-                   : launch_h<HH, false>(q_idx, q_scale, w, k_idx, k_scale, r, scores, ld,     \
-                                         status, s);
-    switch (H_I) {
-        IC_IDX_CASE(16)
-        IC_IDX_CASE(32)
-        IC_IDX_CASE(64)
-        IC_IDX_CASE(128)
-    }
-#undef IC_IDX_CASE
-    return IC_ERR_UNSUPPORTED;
+    const Paging dense = {nullptr, nullptr, 0, 0, 0, (int64_t)r.B * r.T};
+    return launch_any(q_idx, q_scale, w, k_idx, k_scale, dt, r, H_I, scores, ld, status, s, dense,
+                      (int64_t)r.B * r.T);
+}
+
+ic_status launch_indexer_tc_paged(const void* q_idx, const float* q_scale, const float* w,
+                                  const void* k_pages, const float* k_scale_pages, ic_dtype dt,
+                                  const ic_paged_rows& pr, int H_I, int d_I, float* scores,
+                                  int64_t ld, uint32_t* status, cudaStream_t s) {
+    if (!indexer_tc_supported(dt, H_I, d_I)) return IC_ERR_UNSUPPORTED;
+    if (((uintptr_t)q_idx & 15) || ((uintptr_t)k_pages & 15)) return IC_ERR_INVALID_ARG;
+    const Paging pg = {pr.seq_lens, pr.block_table, pr.max_pages, pr.page_size, pr.T_max,
+                       (int64_t)pr.num_pages * pr.page_size};
+    // planning rows: every sequence as long as T_max
+    const ic_rows r = {pr.B, pr.Lq, pr.T_max - pr.Lq, pr.T_max};
+    return launch_any(q_idx, q_scale, w, k_pages, k_scale_pages, dt, r, H_I, scores, ld, status, s,
+                      pg, (int64_t)pr.num_pages * pr.page_size);
 }
 
 }  // namespace ic

@@ -375,6 +375,15 @@ __device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t a, u
         : "memory");
 }
 
+// Asynchronous 4-byte store into another CTA's shared memory, counted in
+// bytes on that CTA's mbarrier like st_async_v4.
+__device__ __forceinline__ void st_async_b32(uint32_t cluster_addr, uint32_t v, uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+                     cluster_addr),
+                 "r"(v), "r"(cluster_bar)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "

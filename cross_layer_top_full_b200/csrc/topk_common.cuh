@@ -11,6 +11,17 @@
 
 namespace ic {
 
+// Candidates of score row `row` (= b*Lq + i): t + 1 with t = q_start + i,
+// or with per-sequence lengths (seq_lens != nullptr) t = seq_lens[b] - Lq + i;
+// a length outside [Lq, T_max] gives 0 candidates (an all -1 row).
+__device__ __forceinline__ int row_candidates(int64_t row, int Lq, int q_start,
+                                              const int32_t* __restrict__ seq_lens, int T_max) {
+    const int i = (int)(row % Lq);
+    if (seq_lens == nullptr) return q_start + i + 1;
+    const int Tb = __ldg(seq_lens + row / Lq);
+    return (Tb >= Lq && Tb <= T_max) ? Tb - Lq + i + 1 : 0;
+}
+
 // Larger score -> larger key; -0.0 and +0.0 give the same key.
 __device__ __forceinline__ uint32_t order_key(float f) {
     uint32_t u = __float_as_uint(f);
@@ -138,6 +149,101 @@ __device__ void select_row(const float* __restrict__ src, int n, int k, int32_t*
         run_gt += tot_gt;
         run_eq += tot_eq;
         // warp_cnt is double-buffered, so one barrier per chunk suffices
+    }
+}
+
+// Block-wide: the bin d holding the k-th largest key of the row histogram,
+// and how many keys lie in higher bins.  hist in shared memory.
+template <int NT>
+__device__ void find_bin11(const uint32_t* hist, uint32_t k, uint32_t& d_out, uint32_t& above_out,
+                           uint32_t* warp_sum) {
+    constexpr int HBINS = 2048;
+    constexpr int PER = HBINS / NT;  // bins per thread, highest bins first
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t c[PER];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        c[j] = hist[HBINS - 1 - PER * threadIdx.x - j];
+        sum += c[j];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    uint32_t before_warp = 0;
+    for (int w = 0; w < warp; ++w) before_warp += warp_sum[w];
+    incl += before_warp;
+    const uint32_t excl = incl - sum;
+    if (excl < k && incl >= k) {  // exactly one thread
+        uint32_t before = excl;
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            if (before + c[j] >= k) {
+                d_out = (uint32_t)(HBINS - 1 - PER * threadIdx.x - j);
+                above_out = before;
+                break;
+            }
+            before += c[j];
+        }
+    }
+    __syncthreads();
+}
+
+// Block-wide radix select over m keys in shared memory: the need-th largest
+// key (tau) and how many keys equal to tau fall inside the top `need`.
+template <int NT>
+__device__ void select_smem(const uint32_t* keys, int m, uint32_t need, SelectState<NT / 32>& st) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) { st.prefix = 0; st.need = need; }
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int j = threadIdx.x; j < 256; j += NT) st.hist[j] = 0;
+        __syncthreads();
+        const uint32_t prefix = st.prefix;
+        const int m_round = (m + 31) & ~31;
+        for (int j = threadIdx.x; j < m_round; j += NT) {
+            bool live = j < m;
+            uint32_t key = live ? keys[j] : 0u;
+            live = live && (pass == 0 || (key >> (shift + 8)) == prefix);
+            const uint32_t digit = live ? ((key >> shift) & 255u) : 256u;
+            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+            if (live && lane == __ffs(peers) - 1) atomicAdd(&st.hist[digit], __popc(peers));
+        }
+        __syncthreads();
+        if (warp == 0) choose_digit(st);
+        __syncthreads();
+    }
+}
+
+// Block-wide radix select over m keys in shared memory whose top `pbits`
+// bits all equal `pval`: the need-th largest key (-> st.prefix) and how many
+// keys equal to it fall inside the top `need` (-> st.need).  Digits of up to
+// 8 bits; plain shared atomics (the keys of one bin are spread out).
+template <int NT>
+__device__ void select_smem_known(const uint32_t* keys, int m, uint32_t need, uint32_t pval,
+                                  int pbits, SelectState<NT / 32>& st) {
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) { st.prefix = pval; st.need = need; }
+    for (int rem = 32 - pbits; rem > 0;) {
+        const int wbits = rem < 8 ? rem : 8;
+        const int shift = rem - wbits;
+        for (int j = threadIdx.x; j < 256; j += NT) st.hist[j] = 0;
+        __syncthreads();
+        const uint32_t prefix = st.prefix;
+        for (int j = threadIdx.x; j < m; j += NT) {
+            const uint32_t key = keys[j];
+            if ((uint64_t)key >> rem == (uint64_t)prefix)
+                atomicAdd(&st.hist[(key >> shift) & ((1u << wbits) - 1u)], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) choose_digit(st, wbits);
+        __syncthreads();
+        rem -= wbits;
     }
 }
 

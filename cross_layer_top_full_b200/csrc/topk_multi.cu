@@ -125,97 +125,6 @@ topk_hist_kernel(const float* __restrict__ scores, int64_t ld, int Lq, int q_sta
     }
 }
 
-// Block-wide: the bin d holding the k-th largest key of the row histogram,
-// and how many keys lie in higher bins.  hist in shared memory.
-__device__ void find_bin(const uint32_t* hist, uint32_t k, uint32_t& d_out, uint32_t& above_out,
-                         uint32_t* warp_sum) {
-    constexpr int PER = HBINS / NT;  // bins per thread, highest bins first
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t c[PER];
-    uint32_t sum = 0;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-        c[j] = hist[HBINS - 1 - PER * threadIdx.x - j];
-        sum += c[j];
-    }
-    uint32_t incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-    }
-    if (lane == 31) warp_sum[warp] = incl;
-    __syncthreads();
-    uint32_t before_warp = 0;
-    for (int w = 0; w < warp; ++w) before_warp += warp_sum[w];
-    incl += before_warp;
-    const uint32_t excl = incl - sum;
-    if (excl < k && incl >= k) {  // exactly one thread
-        uint32_t before = excl;
-#pragma unroll
-        for (int j = 0; j < PER; ++j) {
-            if (before + c[j] >= k) {
-                d_out = (uint32_t)(HBINS - 1 - PER * threadIdx.x - j);
-                above_out = before;
-                break;
-            }
-            before += c[j];
-        }
-    }
-    __syncthreads();
-}
-
-// Block-wide radix select over m keys in shared memory: the need-th largest
-// key (tau) and how many keys equal to tau fall inside the top `need`.
-__device__ void select_smem(const uint32_t* keys, int m, uint32_t need, SelectState<NW>& st) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (threadIdx.x == 0) { st.prefix = 0; st.need = need; }
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        for (int j = threadIdx.x; j < 256; j += NT) st.hist[j] = 0;
-        __syncthreads();
-        const uint32_t prefix = st.prefix;
-        const int m_round = (m + 31) & ~31;
-        for (int j = threadIdx.x; j < m_round; j += NT) {
-            bool live = j < m;
-            uint32_t key = live ? keys[j] : 0u;
-            live = live && (pass == 0 || (key >> (shift + 8)) == prefix);
-            const uint32_t digit = live ? ((key >> shift) & 255u) : 256u;
-            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-            if (live && lane == __ffs(peers) - 1) atomicAdd(&st.hist[digit], __popc(peers));
-        }
-        __syncthreads();
-        if (warp == 0) choose_digit(st);
-        __syncthreads();
-    }
-}
-
-// Block-wide radix select over m keys in shared memory whose top `pbits`
-// bits all equal `pval`: the need-th largest key (-> st.prefix) and how many
-// keys equal to it fall inside the top `need` (-> st.need).  Digits of up to
-// 8 bits; plain shared atomics (the keys of one bin are spread out).
-__device__ void select_smem_known(const uint32_t* keys, int m, uint32_t need, uint32_t pval,
-                                  int pbits, SelectState<NW>& st) {
-    const int warp = threadIdx.x >> 5;
-    if (threadIdx.x == 0) { st.prefix = pval; st.need = need; }
-    for (int rem = 32 - pbits; rem > 0;) {
-        const int wbits = rem < 8 ? rem : 8;
-        const int shift = rem - wbits;
-        for (int j = threadIdx.x; j < 256; j += NT) st.hist[j] = 0;
-        __syncthreads();
-        const uint32_t prefix = st.prefix;
-        for (int j = threadIdx.x; j < m; j += NT) {
-            const uint32_t key = keys[j];
-            if ((uint64_t)key >> rem == (uint64_t)prefix)
-                atomicAdd(&st.hist[(key >> shift) & ((1u << wbits) - 1u)], 1u);
-        }
-        __syncthreads();
-        if (warp == 0) choose_digit(st, wbits);
-        __syncthreads();
-        rem -= wbits;
-    }
-}
-
 // ------------------------------------------------------------------------ K2
 __global__ void __launch_bounds__(NT)
 topk_cand_kernel(const float* __restrict__ scores, int64_t ld, int Lq, int q_start, int k,
@@ -238,7 +147,7 @@ topk_cand_kernel(const float* __restrict__ scores, int64_t ld, int Lq, int q_sta
     for (int b = threadIdx.x; b < HBINS; b += NT) h[b] = __ldcg(gh + b);
     if (threadIdx.x == 0) { sh_cnt = 0; sh_n = 0; }
     __syncthreads();
-    find_bin(h, (uint32_t)k, sh_d, sh_above, warp_sum);
+    find_bin11<NT>(h, (uint32_t)k, sh_d, sh_above, warp_sum);
     const uint32_t d = sh_d;
 
     // my chunk: count keys above bin d, append the keys of bin d
@@ -324,7 +233,7 @@ topk_cand_kernel(const float* __restrict__ scores, int64_t ld, int Lq, int q_sta
     for (int c = threadIdx.x; c < nch; c += NT) sel[c] = __ldcg(ws.chunk_gt + row * ws.nch + c);
     __syncthreads();
     const uint32_t need1 = (uint32_t)k - sh_above;   // keys still to take from bin d
-    select_smem_known(skey, m, need1, d, HBITS, st);
+    select_smem_known<NT>(skey, m, need1, d, HBITS, st);
     const uint32_t tau = st.prefix, need_eq = st.need;
     __syncthreads();
     // ties at tau: keep the need_eq smallest positions among the equal keys
@@ -340,7 +249,7 @@ topk_cand_kernel(const float* __restrict__ scores, int64_t ld, int Lq, int q_sta
     if (sh_cnt > need_eq) {
         for (int j = threadIdx.x; j < m; j += NT) spos[j] = skey[j] == tau ? ~spos[j] : 0u;
         __syncthreads();
-        select_smem(spos, m, need_eq, st);
+        select_smem<NT>(spos, m, need_eq, st);
         pos_cut = ~st.prefix;
     }
     __syncthreads();

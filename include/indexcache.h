@@ -230,7 +230,7 @@ ic_status ic_sparse_attn(const void* q, const void* kmat, int64_t k_row_stride,
  * cleared at the start of each call): calls whose kernels overlap on the GPU
  * race on it, so serialise them (one stream, one thread).
  */
-#define IC_NOALLOC_SCRATCH_BYTES ((16u << 20) + (64u << 10) + 512u)
+#define IC_NOALLOC_SCRATCH_BYTES ((16u << 20) + (128u << 10) + 512u)
 ic_status ic_sparse_attn_noalloc(const void* q, const void* kv, const int32_t* idx, int k,
                                  ic_rows r, float scale, void* out, int32_t* device_status,
                                  void* stream);
@@ -284,6 +284,89 @@ ic_status ic_layer_stack_forward(const char* pattern, int n_layers, const ic_lay
                                  const ic_stack_shape* shape, int32_t* idx_buf,
                                  int32_t* const* idx_out, void* ws, size_t ws_bytes,
                                  void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Variable-length batches over a paged KV cache                             */
+/* ------------------------------------------------------------------------ */
+/*
+ * The decode batch of a serving engine: every sequence has its own length,
+ * and every per-key cache (the indexer keys k_I, their FP8 scales, the
+ * latent KV rows) lives in fixed-size pages shared by all sequences, so a
+ * sequence grows by pages without moving data.  This is the layout behind
+ * the pages' throughput figure with the KV cache saturated (es page,
+ * section 3 "Resultados Clave"; de page, section 3 "Wichtige Ergebnisse");
+ * the pages do not describe the layout itself, and the serving system
+ * around it is not part of this library.
+ *
+ *   B            sequences; Lq query rows per sequence (1 for decode)
+ *   seq_lens     [B] int32, DEVICE: keys of sequence b (its context,
+ *                including the query rows' own keys); Lq <= seq_lens[b] <= T_max
+ *                (a length outside this range makes the sequence's rows
+ *                empty: no index, zero output, status bit IC_ERR_INDEX_RANGE)
+ *   T_max        upper bound of seq_lens (sizes the score rows and grids;
+ *                the host never reads seq_lens)
+ *   block_table  [B, max_pages] int32, DEVICE: physical page of logical page
+ *                j of sequence b.  Key position s of sequence b lives in
+ *                physical row block_table[b*max_pages + s/page_size] *
+ *                page_size + s % page_size of every paged cache.
+ *   page_size    rows per page: a multiple of 128
+ *   num_pages    pages of each paged cache (physical rows = num_pages*page_size)
+ * Query row i of sequence b sits at t = seq_lens[b] - Lq + i and its
+ * candidate keys are the logical positions 0..t.  Indices (top-k outputs and
+ * attention inputs) are LOGICAL positions.
+ */
+typedef struct {
+    int B;
+    int Lq;
+    int T_max;
+    const int32_t* seq_lens;
+    const int32_t* block_table;
+    int max_pages;
+    int page_size;
+    int num_pages;
+} ic_paged_rows;
+
+/* a1 over paged keys: scores[b,i,s] for logical s <= t as ic_indexer_scores.
+ *   k_pages        [num_pages*page_size, d_I] of dt (IC_BF16 or IC_FP8_E4M3)
+ *   k_scale_pages  [num_pages*page_size] float32 (IC_FP8_E4M3 only)
+ *   scores         [B, Lq, ld_scores] float32, ld_scores >= T_max, % 4 == 0
+ * Tensor-core shapes only: d_I == 128, H_I in {16,32,64,128}; other shapes
+ * and IC_F32 return IC_ERR_UNSUPPORTED.  Workspace: ic_indexer_workspace_size. */
+ic_status ic_indexer_scores_paged(const void* q_idx, const float* q_scale, const float* w,
+                                  const void* k_pages, const float* k_scale_pages, ic_dtype dt,
+                                  const ic_paged_rows* pr, int H_I, int d_I,
+                                  float* scores, int64_t ld_scores,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* a2 with per-sequence lengths: row (b, i) keeps the min(k, t+1) best of
+ * its t+1 candidates, t = seq_lens[b] - Lq + i, as ic_topk.  Only seq_lens,
+ * B, Lq and T_max of pr are read.  Workspace: ic_topk_varlen_workspace_size. */
+size_t ic_topk_varlen_workspace_size(const ic_paged_rows* pr, int k);
+ic_status ic_topk_varlen(const float* scores, int64_t ld_scores, const ic_paged_rows* pr, int k,
+                         int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+
+/* a4/a5 over paged latent KV rows (IC_BF16, Hq = 128, d_qk = 576, d_v = 512):
+ *   q         [B, Lq, 128, 576] bf16
+ *   kv_pages  [num_pages*page_size, 576] bf16 (V = the first 512 columns)
+ *   idx       [B, Lq, k] int32 logical positions in [0, t] or -1
+ *   out       [B, Lq, 128, 512] bf16
+ * Workspace: ic_sparse_attn_paged_workspace_size. */
+size_t ic_sparse_attn_paged_workspace_size(const ic_paged_rows* pr, int k);
+ic_status ic_sparse_attn_paged(const void* q, const void* kv_pages, const int32_t* idx, int k,
+                               const ic_paged_rows* pr, float scale, void* out,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* a3 over paged caches: ic_layer_stack_forward with every layer's k_idx,
+ * k_scale, kmat (== vmat) pointing at that layer's paged caches.  shape->rows
+ * is ignored (pr gives the rows); shape must name the tensor-core shapes
+ * (idx_dtype IC_BF16 or IC_FP8_E4M3, d_I 128; attn IC_BF16, 128 heads, 576 /
+ * 512, row strides 576). */
+size_t ic_paged_workspace_size(const ic_stack_shape* shape, const ic_paged_rows* pr);
+ic_status ic_layer_stack_forward_paged(const char* pattern, int n_layers,
+                                       const ic_layer_io* layers, const ic_stack_shape* shape,
+                                       const ic_paged_rows* pr, int32_t* idx_buf,
+                                       int32_t* const* idx_out, void* ws, size_t ws_bytes,
+                                       void* stream);
 
 #ifdef __cplusplus
 }

@@ -215,3 +215,68 @@ def test_binding_refuses_host_tensors_and_strided_views(lib):
     with pytest.raises(ValueError, match="contiguous"):
         ic.topk(_StridedDevice(), rows, 2, 1 << 40, _FakeTensor(4096))
     assert ic.kernel_launches(0) == before
+
+
+def test_paged_calls_validate_arguments(lib):
+    """The variable-length / paged calls refuse inconsistent batches before
+    any launch: host memory stands in for every device array here."""
+    ws = _FakeTensor(1 << 16)
+    lens = _FakeTensor(64)
+    table = _FakeTensor(256)
+
+    def pr(**kw):
+        d = dict(B=2, Lq=1, T_max=512, seq_lens=lens.addr, block_table=table.addr, max_pages=4,
+                 page_size=128, num_pages=8)
+        d.update(kw)
+        return ic.PagedRows(d["B"], d["Lq"], d["T_max"], d["seq_lens"], d["block_table"],
+                            d["max_pages"], d["page_size"], d["num_pages"])
+
+    before = ic.kernel_launches(0)
+
+    def attn(p, ws_bytes=1 << 16):
+        return lib.ic_sparse_attn_paged(1, 1, 1, 64, ctypes.byref(p), 0.1, 1, ws.addr, ws_bytes,
+                                        None)
+
+    assert attn(pr(page_size=100)) == -1            # not a multiple of 128
+    assert attn(pr(page_size=0)) == -1
+    assert attn(pr(max_pages=3)) == -1              # 3 pages of 128 cannot hold T_max = 512
+    assert attn(pr(seq_lens=None)) == -1
+    assert attn(pr(block_table=None)) == -1
+    assert attn(pr(T_max=0)) == -1                  # T_max < Lq
+    assert attn(pr(Lq=0)) == -1
+    assert attn(pr(num_pages=0)) == -1
+    assert attn(pr(), ws_bytes=16) == -4            # workspace too small
+    assert lib.ic_sparse_attn_paged(1, 1, 1, 0, ctypes.byref(pr()), 0.1, 1, ws.addr, 1 << 16,
+                                    None) == -1     # k = 0
+    # indexer: tensor-core shapes only; fp8 needs both scales
+    assert lib.ic_indexer_scores_paged(1, None, 1, 1, None, ic.F32, ctypes.byref(pr()), 64, 128,
+                                       1, 512, ws.addr, 1 << 16, None) == -3
+    assert lib.ic_indexer_scores_paged(1, None, 1, 1, None, ic.BF16, ctypes.byref(pr()), 64, 96,
+                                       1, 512, ws.addr, 1 << 16, None) == -3
+    assert lib.ic_indexer_scores_paged(1, None, 1, 1, None, ic.FP8_E4M3, ctypes.byref(pr()), 64,
+                                       128, 1, 512, ws.addr, 1 << 16, None) == -1
+    assert lib.ic_indexer_scores_paged(1, None, 1, 1, None, ic.BF16, ctypes.byref(pr()), 64, 128,
+                                       1, 510, ws.addr, 1 << 16, None) == -1   # ld < T_max
+    # top-k reads only the lengths: no block table needed, but a bad ld is refused
+    assert lib.ic_topk_varlen(1, 510, ctypes.byref(pr(block_table=None)), 8, 1, ws.addr, 1 << 16,
+                              None) == -1
+    assert lib.ic_topk_varlen(1, 512, ctypes.byref(pr(seq_lens=None)), 8, 1, ws.addr, 1 << 16,
+                              None) == -1
+    # the stack: tensor-core shapes only, and patterns checked first
+    sh = ic.StackShape(ic.Rows(2, 1, 511, 512), 64, 128, ic.BF16, 64, 128, 576, 512, ic.BF16,
+                       576, 576, 0.04)
+    big = _FakeTensor(ic.paged_workspace_size(sh, pr()))
+    layers = (ic.LayerIO * 2)()
+    assert lib.ic_layer_stack_forward_paged(b"SF", 2, layers, ctypes.byref(sh), ctypes.byref(pr()),
+                                            1, None, big.addr, big.nbytes, None) == -2
+    sh_f32 = ic.StackShape(ic.Rows(2, 1, 511, 512), 4, 32, ic.F32, 64, 8, 64, 64, ic.F32, 64, 64,
+                           0.1)
+    assert lib.ic_layer_stack_forward_paged(b"FS", 2, layers, ctypes.byref(sh_f32),
+                                            ctypes.byref(pr()), 1, None, big.addr, big.nbytes,
+                                            None) == -3
+    assert lib.ic_layer_stack_forward_paged(b"FS", 2, layers, ctypes.byref(sh), ctypes.byref(pr()),
+                                            1, None, big.addr, big.nbytes, None) == -1  # NULL layers
+    # an empty batch is a no-op
+    assert attn(pr(B=0, seq_lens=None, block_table=None)) == 0
+    assert ic.kernel_launches(0) == before
+    assert ic.paged_workspace_size(sh, pr()) >= ic.STATUS_BYTES + 2 * 512 * 4

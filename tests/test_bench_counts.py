@@ -133,3 +133,30 @@ def test_oracle_stage_clock_times_each_stage_and_restores_the_oracle():
     assert sum(clock.seconds.values()) <= spent
     cb = bench.cpu_baseline(wl, wl.pattern, rate, done, spent, "query rows", clock)
     assert cb["per_row_ms"] == per_row
+
+
+def test_overlap_matrix_matches_the_oracle():
+    """The all-pairs layer overlap matrix equals the oracle's topk_overlap,
+    pair by pair, on ragged (-1 padded) ascending rows."""
+    import numpy as np
+    import torch
+    import oracle
+    rng = np.random.default_rng(3)
+    T, k, rows, L = 60, 8, 7, 4
+    sets = []
+    for _ in range(L):
+        a = np.full((rows, k), -1, dtype=np.int32)
+        for r in range(rows):
+            m = int(rng.integers(1, k + 1))
+            a[r, :m] = np.sort(rng.choice(T, m, replace=False))
+        sets.append(a)
+    s_sum, s_min, n = bench.overlap_matrix([torch.from_numpy(a) for a in sets], T)
+    assert n == rows
+    for l in range(L):
+        for m in range(L):
+            ref = oracle.topk_overlap(sets[l], sets[m])
+            assert s_sum[l, m].item() == pytest.approx(ref.sum())
+            assert s_min[l, m].item() == pytest.approx(ref.min())
+        assert s_sum[l, l].item() == pytest.approx(rows)
+    js = bench.overlap_json(s_sum, s_min, n, "test")
+    assert js["layers"] == L and len(js["mean"]) == L and js["mean"][0][0] == 1.0

@@ -61,6 +61,7 @@ def test_c_client_calls_return_before_the_device(c_report):
     assert r["ok_string"] == "IC_OK"
     assert r["last_error_before"] == ""
     assert r["bad_pattern"] == -2 and r["short_pattern"] == -2   # IC_ERR_PATTERN
+    assert r["bad_page_size"] == -1 and r["paged_no_ws"] == -4
     assert r["no_ws"] == -4          # IC_ERR_WORKSPACE: NULL workspace
     assert r["bad_k"] == -1          # IC_ERR_INVALID_ARG: k = 0
     assert r["workspace_size"] > 0
@@ -73,7 +74,8 @@ def _ctypes_layout(cls):
 
 
 @pytest.mark.parametrize("cname,cls", [("ic_rows", ic.Rows), ("ic_stack_shape", ic.StackShape),
-                                       ("ic_layer_io", ic.LayerIO)])
+                                       ("ic_layer_io", ic.LayerIO),
+                                       ("ic_paged_rows", ic.PagedRows)])
 def test_binding_structs_have_the_c_layout(c_report, cname, cls):
     c = dict(c_report[cname])
     assert c.pop("size") == ctypes.sizeof(cls)
@@ -92,7 +94,7 @@ _SCALARS = {
     "uint64_t": ctypes.c_uint64, "ic_rows": ic.Rows,
 }
 _POINTEES = {"ic_stack_shape": ic.StackShape, "ic_layer_io": ic.LayerIO,
-             "int32_t": ctypes.c_int32}
+             "ic_paged_rows": ic.PagedRows, "int32_t": ctypes.c_int32}
 
 
 def _prototypes():

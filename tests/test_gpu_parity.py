@@ -192,6 +192,14 @@ def test_indexer_general_inputs_within_tolerance(dev, dtype):
                                     ((3, 1, 32767, 32768), 2048), # decode rows, cached
                                     ((2, 3, 40000, 40003), 2048), # few long rows of unequal length
                                     ((1, 2, 199998, 200000), 2048),
+                                    # one cluster per row: 8, 4, 2 and 1 CTAs per row
+                                    ((32, 1, 32767, 32768), 2048),
+                                    ((64, 1, 9999, 10000), 2048),
+                                    ((100, 1, 5999, 6000), 2048),
+                                    # cluster rows of which two keep every candidate (n <= k)
+                                    ((2, 4, 4998, 5002), 5000),
+                                    # rows too long for a cluster's shared memory: three launches
+                                    ((2, 1, 399999, 400000), 2048),
                                     # row caches of 46.9 KiB and exactly 48 KiB of shared memory
                                     # (plus the static select state: past the default limit)
                                     ((1, 300, 11700, 12000), 2048),
@@ -206,6 +214,22 @@ def test_topk_is_bit_exact_on_identical_scores(dev, rows, k, ties):
     torch.cuda.synchronize()
     ref = oracle.topk_indices(host64(scores), q_start, k)
     assert np.array_equal(host64(idx), ref)
+
+
+@pytest.mark.parametrize("rows", [(8, 1, 199999, 200000), (32, 1, 32767, 32768)])
+def test_decode_topk_is_one_launch(dev, rows):
+    """Decode rows (the two decode workloads' shapes) take the one-launch
+    cluster path, bit-exact against the oracle."""
+    B, Lq, q_start, T = rows
+    k = 2048
+    scores = synth.random_scores(B, Lq, T, dev, seed=B)
+    idx = torch.full((B, Lq, k), -7, dtype=torch.int32, device=dev)
+    ws = _ws(ic.topk_workspace_size(rows, k), dev)
+    n0 = ic.kernel_launches(2)
+    ic.topk(scores, rows, k, idx, ws)
+    torch.cuda.synchronize()
+    assert ic.kernel_launches(2) - n0 == 1
+    assert np.array_equal(host64(idx), oracle.topk_indices(host64(scores), q_start, k))
 
 
 def test_topk_long_rows_of_equal_scores(dev):
