@@ -110,13 +110,28 @@ class Stack:
         ic.layer_stack_forward(pattern, self.layers, self.shape, self.idx, self.ws, stream=stream)
 
     def stage_step(self, pattern, ev):
-        """The same step as separate C-ABI calls, with CUDA events around each."""
+        """The same step as separate C-ABI calls, with CUDA events around each.
+        Decode F layers run the fused key selection (ic_indexer_topk, the
+        stack's path: stage "select"); the un-fused indexer and top-k are
+        timed after it as references (stages "indexer" and "topk", not part
+        of the step's path)."""
         wl = self.wl
         for l, kind in enumerate(pattern):
             L = self.layers[l]
             if kind == "F":
-                e0, e1, e2 = ev.new(), ev.new(), ev.new()
-                e0.record()
+                if fused_selection(wl):
+                    e = ev.new()
+                    e.record()
+                    ic.indexer_topk(L["q_idx"], L["w"], L["k_idx"], self.rows, wl.k, self.idx,
+                                    self.ws, q_scale=L["q_scale"], k_scale=L["k_scale"],
+                                    dtype=DT[wl.idx_dtype])
+                    e0 = ev.new()
+                    e0.record()
+                    ev.add("select", e, e0)
+                else:
+                    e0 = ev.new()
+                    e0.record()
+                e1, e2 = ev.new(), ev.new()
                 ic.indexer_scores(L["q_idx"], L["w"], L["k_idx"], self.rows, self.scores, self.ws,
                                   q_scale=L["q_scale"], k_scale=L["k_scale"],
                                   dtype=DT[wl.idx_dtype])
@@ -164,6 +179,21 @@ class Events:
 
 
 # ----------------------------------------------------------------------------- algorithmic work
+def fused_selection(wl):
+    """Whether the library runs an F layer's indexer and top-k as one fused
+    kernel for this workload (decode rows on the tensor-core shapes): the
+    library's own rule, restated."""
+    T_max = wl.q_start + wl.L
+    return (wl.L <= 2 and wl.idx_dtype in ("bf16", "e4m3") and wl.d_I == 128
+            and wl.H_I in (16, 32, 64, 128) and wl.B * wl.L <= 148 and T_max > wl.k
+            and T_max >= 4096)
+
+
+def path_stages(wl):
+    """The stages one step runs, in the stack's path."""
+    return ("select", "attention") if fused_selection(wl) else ("indexer", "topk", "attention")
+
+
 def algorithmic(wl):
     """Per-launch algorithmic work of each stage (pages' definitions, all rows)."""
     rows = [wl.q_start + i for i in range(wl.L)]
@@ -177,6 +207,9 @@ def algorithmic(wl):
         "indexer_bytes": wl.B * (wl.T * wl.d_I * ib + wl.L * wl.H_I * (wl.d_I * ib + 4))
         + 4.0 * pairs,
         "topk_bytes": 4.0 * pairs + 4.0 * wl.B * wl.L * wl.k,
+        # fused selection: the indexer's reads and the indices written, no scores
+        "select_bytes": wl.B * (wl.T * wl.d_I * ib + wl.L * wl.H_I * (wl.d_I * ib + 4))
+        + (wl.B * wl.T * 4.0 if wl.idx_dtype == "e4m3" else 0.0) + 4.0 * wl.B * wl.L * wl.k,
         "attn_flop": 2.0 * wl.Hq * (wl.d_qk + wl.d_v) * visits,
         "attn_bytes": visits * kv_w * ab + wl.B * wl.L * wl.Hq * (wl.d_qk + wl.d_v) * ab
         + 4.0 * wl.B * wl.L * wl.k,
@@ -195,6 +228,8 @@ def stage_bound(wl, work, stage):
     if stage == "indexer":
         tensor = wl.L > 1
         return tensor, work["indexer_flop"] if tensor else work["indexer_bytes"]
+    if stage == "select":
+        return False, work["select_bytes"]
     return False, work["topk_bytes"]
 
 
@@ -219,6 +254,7 @@ def stage_roofline(wl, work, stage, per_launch_ms, peak="burst", per_pass=1):
     tensor, num = stage_bound(wl, work, stage)
     fp8 = stage == "indexer" and wl.idx_dtype == "e4m3"
     roof = _roof(num, per_launch_ms * per_pass, tensor, fp8, peak)
+    roof["in_step_path"] = stage in path_stages(wl)
     roof["ms_per_launch"] = per_launch_ms
     return roof
 
@@ -229,7 +265,7 @@ def roofline(wl, work, total_ms, launches, per_pass=1, peak="sustained"):
     algorithmic work of one pass of a stage over all rows (``algorithmic``;
     summed over the chunks of a chunked run), which takes ``per_pass``
     launches.  ``peak``: "burst" or "sustained" bf16 figure."""
-    dom = max(total_ms, key=lambda k: total_ms[k])
+    dom = max((k for k in total_ms if k in path_stages(wl)), key=lambda k: total_ms[k])
     passes = launches[dom] / per_pass
     per_pass_ms = total_ms[dom] / passes
     tensor, num = stage_bound(wl, work, dom)
@@ -656,9 +692,10 @@ def measure_stack(wl, pattern, dev, pg, rank, world, *, steps, warmup, graph, e2
     roof, dom = roofline(wl, work, totals, counts, peak=kind)
     roof["traffic"] = _traffic(dom, wl.name)
     by_stage = {k: stage_roofline(wl, work, k, avg[k], kind) for k in stages}
-    # share of the step spent choosing keys (indexer + top-k)
-    total_stage = sum(totals.values())
-    sel_share = (totals.get("indexer", 0.0) + totals.get("topk", 0.0)) / total_stage
+    # share of the step spent choosing keys (the selection stages of the path)
+    path = path_stages(wl)
+    total_stage = sum(totals[k] for k in path if k in totals)
+    sel_share = sum(totals.get(k, 0.0) for k in path if k != "attention") / total_stage
     bytes_in = st.bytes_per_step(pattern)
     del st
     gc.collect()

@@ -20,6 +20,7 @@ __all__ = [
     "F32", "BF16", "FP8_E4M3", "STATUS_BYTES",
     "status_string", "version", "kernel_launches", "workspace_init", "read_status",
     "indexer_workspace_size", "indexer_scores", "topk_workspace_size", "topk",
+    "indexer_topk_workspace_size", "indexer_topk",
     "sparse_attn_workspace_size", "sparse_attn", "sparse_attn_noalloc", "workspace_size",
     "layer_stack_forward", "indexer_scores_paged", "topk_varlen_workspace_size", "topk_varlen",
     "sparse_attn_paged_workspace_size", "sparse_attn_paged", "paged_workspace_size",
@@ -86,6 +87,10 @@ _SIG = {
     "ic_indexer_workspace_size": (ctypes.c_size_t, [Rows, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "ic_indexer_scores": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, Rows, ctypes.c_int,
                                          ctypes.c_int, _P, ctypes.c_int64, _P, ctypes.c_size_t, _P]),
+    "ic_indexer_topk_workspace_size": (ctypes.c_size_t, [Rows, ctypes.c_int, ctypes.c_int,
+                                                         ctypes.c_int, ctypes.c_int]),
+    "ic_indexer_topk": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, Rows, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_size_t, _P]),
     "ic_topk_workspace_size": (ctypes.c_size_t, [Rows, ctypes.c_int]),
     "ic_topk": (ctypes.c_int, [_P, ctypes.c_int64, Rows, ctypes.c_int, _P, _P, ctypes.c_size_t, _P]),
     "ic_sparse_attn_workspace_size": (ctypes.c_size_t, [Rows, ctypes.c_int, ctypes.c_int,
@@ -242,6 +247,22 @@ def indexer_scores(q_idx, w, k_idx, rows, scores, ws, *, q_scale=None, k_scale=N
     _check(lib().ic_indexer_scores(_ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(k_idx), _ptr(k_scale),
                                    dt, r, H_I, d_I, _ptr(scores), ld, _ptr(ws), _nbytes(ws),
                                    _stream(stream)), "ic_indexer_scores")
+
+
+def indexer_topk_workspace_size(rows, H_I: int, d_I: int, dtype: int, k: int) -> int:
+    return int(lib().ic_indexer_topk_workspace_size(_rows(rows), H_I, d_I, dtype, k))
+
+
+def indexer_topk(q_idx, w, k_idx, rows, k: int, idx, ws, *, q_scale=None, k_scale=None,
+                 dtype: Optional[int] = None, stream=None) -> None:
+    """An F layer's key selection: indexer scores and top-k in one call (one
+    fused kernel for decode rows)."""
+    r = _rows(rows)
+    dt = _dtype_of(q_idx) if dtype is None else dtype
+    H_I, d_I = q_idx.shape[-2], q_idx.shape[-1]
+    _check(lib().ic_indexer_topk(_ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(k_idx), _ptr(k_scale),
+                                 dt, r, H_I, d_I, k, _ptr(idx), _ptr(ws), _nbytes(ws),
+                                 _stream(stream)), "ic_indexer_topk")
 
 
 def topk_workspace_size(rows, k: int) -> int:

@@ -21,6 +21,10 @@ void count_launch(int kind) {
     g_launches[IC_LK_ALL].fetch_add(1, std::memory_order_relaxed);
     if (kind == IC_LK_INDEXER_TC) g_launches[IC_LK_INDEXER].fetch_add(1, std::memory_order_relaxed);
     if (kind == IC_LK_ATTN_TC) g_launches[IC_LK_ATTN].fetch_add(1, std::memory_order_relaxed);
+    if (kind == IC_LK_SELECT) {  // one fused launch does an F layer's indexer and top-k
+        g_launches[IC_LK_INDEXER].fetch_add(1, std::memory_order_relaxed);
+        g_launches[IC_LK_TOPK].fetch_add(1, std::memory_order_relaxed);
+    }
     if (kind > 0 && kind < IC_LK_KINDS) g_launches[kind].fetch_add(1, std::memory_order_relaxed);
 }
 
@@ -135,6 +139,23 @@ ic_status run_topk(const float* scores, int64_t ld, ic_rows r, int k, int32_t* i
     return launch_topk_rows(scores, ld, r, k, idx, s);
 }
 
+// An F layer's key selection: fused for decode shapes, else indexer scores
+// into `scores` then top-k.
+ic_status run_select(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
+                     const float* k_scale, ic_dtype dt, ic_rows r, int H_I, int d_I, int k,
+                     int32_t* idx, float* scores, int64_t ld, uint32_t* status, void* scratch,
+                     size_t scratch_bytes, cudaStream_t s) {
+    if (select_fused_applies(dt, H_I, d_I, r, k)) {
+        const ic_status st = launch_select_fused(q_idx, q_scale, w, k_idx, k_scale, dt, r, H_I, k,
+                                                 idx, status, s);
+        if (st != IC_ERR_UNSUPPORTED) return st;
+    }
+    ic_status st = run_indexer(q_idx, q_scale, w, k_idx, k_scale, dt, r, H_I, d_I, scores, ld,
+                               status, s);
+    if (st != IC_OK) return st;
+    return run_topk(scores, ld, r, k, idx, scratch, scratch_bytes, s);
+}
+
 ic_status run_attn(const void* q, const void* kmat, int64_t ks, const void* vmat, int64_t vs,
                    const int32_t* idx, int k, ic_dtype dt, ic_rows r, int Hq, int d_qk, int d_v,
                    float scale, void* out, uint32_t* status, void* scratch, size_t scratch_bytes,
@@ -241,6 +262,30 @@ ic_status ic_topk(const float* scores, int64_t ld_scores, ic_rows r, int k, int3
                     (cudaStream_t)stream);
 }
 
+size_t ic_indexer_topk_workspace_size(ic_rows r, int H_I, int d_I, ic_dtype dt, int k) {
+    (void)H_I; (void)d_I; (void)dt;
+    return IC_STATUS_BYTES + align_up(scores_bytes(r)) + align_up(topk_multi_scratch_bytes(r, k));
+}
+
+ic_status ic_indexer_topk(const void* q_idx, const float* q_scale, const float* w,
+                          const void* k_idx, const float* k_scale, ic_dtype dt, ic_rows r, int H_I,
+                          int d_I, int k, int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+    if (!rows_ok(r) || !indexer_args_ok(dt, H_I, d_I) || k < 1 || k > 16384)
+        return IC_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, ic_indexer_topk_workspace_size(r, H_I, d_I, dt, k)))
+        return IC_ERR_WORKSPACE;
+    if (rows_empty(r)) return IC_OK;
+    if (!q_idx || !w || !k_idx || !idx) return IC_ERR_INVALID_ARG;
+    if (dt == IC_FP8_E4M3 && (!q_scale || !k_scale)) return IC_ERR_INVALID_ARG;
+    if (dt != IC_FP8_E4M3 && (q_scale || k_scale)) return IC_ERR_INVALID_ARG;
+    float* scores = reinterpret_cast<float*>(scratch_of(ws));
+    const int64_t ld = ((int64_t)r.T + 3) / 4 * 4;
+    char* tail = scratch_of(ws) + align_up(scores_bytes(r));
+    return run_select(q_idx, q_scale, w, k_idx, k_scale, dt, r, H_I, d_I, k, idx, scores, ld,
+                      status_of(ws), tail, ws_bytes - IC_STATUS_BYTES - align_up(scores_bytes(r)),
+                      (cudaStream_t)stream);
+}
+
 size_t ic_sparse_attn_workspace_size(ic_rows r, int k, int Hq, int d_qk, int d_v, ic_dtype dt) {
     return IC_STATUS_BYTES + align_up(attn_scratch(r, k, Hq, d_qk, d_v, dt));
 }
@@ -309,10 +354,9 @@ ic_status ic_layer_stack_forward(const char* pattern, int n_layers, const ic_lay
     for (int l = 0; l < n_layers; ++l) {
         const ic_layer_io& L = layers[l];
         if (pattern[l] == 'F') {  // the one conditional branch of IndexCache
-            ic_status st = run_indexer(L.q_idx, L.q_scale, L.w, L.k_idx, L.k_scale, sh->idx_dtype,
-                                       r, sh->H_I, sh->d_I, scores, ld, status, s);
-            if (st != IC_OK) return st;
-            st = run_topk(scores, ld, r, sh->k, idx_buf, attn_ws, attn_ws_bytes, s);
+            const ic_status st = run_select(L.q_idx, L.q_scale, L.w, L.k_idx, L.k_scale,
+                                            sh->idx_dtype, r, sh->H_I, sh->d_I, sh->k, idx_buf,
+                                            scores, ld, status, attn_ws, attn_ws_bytes, s);
             if (st != IC_OK) return st;
         }
         ic_status st = run_attn(L.q, L.kmat, sh->k_row_stride, L.vmat, sh->v_row_stride, idx_buf,
@@ -418,11 +462,18 @@ ic_status ic_layer_stack_forward_paged(const char* pattern, int n_layers, const 
     for (int l = 0; l < n_layers; ++l) {
         const ic_layer_io& L = layers[l];
         if (pattern[l] == 'F') {  // the one conditional branch of IndexCache
-            ic_status st = launch_indexer_tc_paged(L.q_idx, L.q_scale, L.w, L.k_idx, L.k_scale,
-                                                   sh->idx_dtype, *pr, sh->H_I, sh->d_I, scores,
-                                                   ld, status, s);
-            if (st != IC_OK) return st;
-            st = run_topk_varlen(scores, ld, pr, sh->k, idx_buf, s);
+            ic_status st = IC_ERR_UNSUPPORTED;
+            if (select_fused_applies(sh->idx_dtype, sh->H_I, sh->d_I, r, sh->k))
+                st = launch_select_fused_paged(L.q_idx, L.q_scale, L.w, L.k_idx, L.k_scale,
+                                               sh->idx_dtype, *pr, sh->H_I, sh->k, idx_buf, status,
+                                               s);
+            if (st == IC_ERR_UNSUPPORTED) {
+                st = launch_indexer_tc_paged(L.q_idx, L.q_scale, L.w, L.k_idx, L.k_scale,
+                                             sh->idx_dtype, *pr, sh->H_I, sh->d_I, scores, ld,
+                                             status, s);
+                if (st != IC_OK) return st;
+                st = run_topk_varlen(scores, ld, pr, sh->k, idx_buf, s);
+            }
             if (st != IC_OK) return st;
         }
         ic_status st = launch_attn_tc_paged(L.q, L.kmat, idx_buf, sh->k, *pr, sh->scale, L.out,

@@ -15,7 +15,7 @@
 // Launch kinds counted by ic_kernel_launches.
 enum {
     IC_LK_ALL = 0, IC_LK_INDEXER = 1, IC_LK_TOPK = 2, IC_LK_ATTN = 3, IC_LK_COMBINE = 4,
-    IC_LK_INDEXER_TC = 5, IC_LK_ATTN_TC = 6, IC_LK_KINDS = 7
+    IC_LK_INDEXER_TC = 5, IC_LK_ATTN_TC = 6, IC_LK_SELECT = 7, IC_LK_KINDS = 8
 };
 
 namespace ic {
@@ -90,6 +90,16 @@ size_t attn_tc_scratch_bytes(ic_rows r, int k, int64_t max_units = kNoUnitLimit)
 ic_status launch_attn_tc(const void* q, const void* kv, int64_t ks, const int32_t* idx, int k,
                          ic_rows r, float scale, void* out, uint32_t* status, void* scratch,
                          size_t scratch_bytes, cudaStream_t s, int64_t max_units = kNoUnitLimit);
+
+// Fused decode key selection (indexer scores kept in shared memory + top-k).
+bool select_fused_applies(ic_dtype dt, int H_I, int d_I, ic_rows r, int k);
+ic_status launch_select_fused(const void* q_idx, const float* q_scale, const float* w,
+                              const void* k_idx, const float* k_scale, ic_dtype dt, ic_rows r,
+                              int H_I, int k, int32_t* idx, uint32_t* status, cudaStream_t s);
+ic_status launch_select_fused_paged(const void* q_idx, const float* q_scale, const float* w,
+                                    const void* k_pages, const float* k_scale_pages, ic_dtype dt,
+                                    const ic_paged_rows& pr, int H_I, int k, int32_t* idx,
+                                    uint32_t* status, cudaStream_t s);
 
 // Paged / variable-length variants (ic_paged_rows: per-sequence lengths and a
 // block table; see include/indexcache.h).

@@ -112,8 +112,9 @@ ic_status ic_selftest_wait_timeout(void* ws, size_t ws_bytes, void* stream);
 /* Number of kernels this library has launched in this process, by kind:
  * 0 = all, 1 = indexer, 2 = top-k, 3 = attention, 4 = split-k combine,
  * 5 = indexer launches that took the tensor-core path, 6 = attention
- * launches that took the tensor-core path.  A host-side diagnostic counter
- * (thread-safe). */
+ * launches that took the tensor-core path, 7 = fused decode key selections
+ * (each also counted once under 1 and once under 2).  A host-side diagnostic
+ * counter (thread-safe). */
 uint64_t ic_kernel_launches(int kind);
 
 /* ------------------------------------------------------------------------ */
@@ -165,6 +166,28 @@ ic_status ic_indexer_scores(const void* q_idx, const float* q_scale, const float
 size_t ic_topk_workspace_size(ic_rows r, int k);
 ic_status ic_topk(const float* scores, int64_t ld_scores, ic_rows r, int k, int32_t* idx,
                   void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* a1 + a2 in one call: an F layer's key selection                           */
+/* ------------------------------------------------------------------------ */
+/*
+ * The indexer scores of ic_indexer_scores followed by the top-k of ic_topk,
+ * with the same inputs, layouts and rules: the same indices, bit for bit
+ * (the scores are computed by the same arithmetic in the same order).  For
+ * decode-shaped rows (Lq <= 2, at most one row per SM, more than 4096
+ * candidates) on the tensor-core shapes the two run as ONE kernel: one
+ * thread-block cluster per row keeps the row's scores in shared memory and
+ * selects from there, so no score row is written to memory.  Otherwise the
+ * scores go through the workspace.  (IndexCache's F layer computes exactly
+ * this selection and caches it: es page, section 2 "Arquitectura del Método".)
+ *   idx  [B, Lq, k] int32 (output), as ic_topk
+ * Workspace: ic_indexer_topk_workspace_size.
+ */
+size_t ic_indexer_topk_workspace_size(ic_rows r, int H_I, int d_I, ic_dtype dt, int k);
+ic_status ic_indexer_topk(const void* q_idx, const float* q_scale, const float* w,
+                          const void* k_idx, const float* k_scale, ic_dtype dt, ic_rows r,
+                          int H_I, int d_I, int k, int32_t* idx, void* ws, size_t ws_bytes,
+                          void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* a4/a5  Sparse multi-query attention (every layer)                         */

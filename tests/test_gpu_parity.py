@@ -250,6 +250,44 @@ def test_topk_long_rows_of_equal_scores(dev):
     assert np.array_equal(host64(idx), ref)
 
 
+# ------------------------------------------------------------------------- fused selection
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("rows", [(8, 1, 199999, 200000),     # the FP8 decode workload's shape
+                                  (32, 1, 32767, 32768),      # the bf16 decode workload's shape
+                                  (3, 2, 9998, 10000),        # two query rows per sequence
+                                  (1, 1, 5000, 5001)])        # one row: the most CTAs per row
+def test_fused_selection_equals_indexer_then_topk(dev, dtype, rows):
+    """ic_indexer_topk on decode rows runs ONE kernel (the indexer's scores
+    kept in shared memory, selected there) and gives exactly the indices of
+    ic_indexer_scores followed by ic_topk: the same arithmetic, bit for bit.
+    The indices also obey the band rule against the oracle's float64 scores
+    (first sequence)."""
+    B, Lq, q_start, T = rows
+    k = 2048
+    wl = synth.Workload("sel", B, Lq, T, q_start, 64, 128, k, 128, 576, 512, dtype, "bf16", True,
+                        "F", 51, 1 / 8, 128 ** -0.5, 128 ** -0.5, 1.0, 1.0, heavy=16,
+                        heavy_gain=4.0)
+    inp = synth.layer_inputs(wl, 0, dev, attention=False)
+    ld = (T + 3) // 4 * 4
+    scores = torch.empty(B, Lq, ld, device=dev)
+    ws = _ws(ic.indexer_topk_workspace_size(rows, 64, 128, DT[dtype], k), dev)
+    ic.indexer_scores(inp["q_I"], inp["w"], inp["k_I"], rows, scores, ws, q_scale=inp.get("q_scale"),
+                      k_scale=inp.get("k_scale"), dtype=DT[dtype])
+    ref = torch.empty(B, Lq, k, dtype=torch.int32, device=dev)
+    ic.topk(scores, rows, k, ref, ws)
+    got = torch.full((B, Lq, k), -7, dtype=torch.int32, device=dev)
+    n_sel, n_ix = ic.kernel_launches(7), ic.kernel_launches(1)
+    ic.indexer_topk(inp["q_I"], inp["w"], inp["k_I"], rows, k, got, ws, q_scale=inp.get("q_scale"),
+                    k_scale=inp.get("k_scale"), dtype=DT[dtype])
+    torch.cuda.synchronize()
+    assert ic.read_status(ws) == 0
+    assert ic.kernel_launches(7) - n_sel == 1 and ic.kernel_launches(1) - n_ix == 1
+    assert torch.equal(got, ref)
+    sub = {key: v[:1] for key, v in inp.items()}
+    sc = _oracle_scores(sub, q_start, dtype)
+    check_topk_band(host64(got[:1]), sc, q_start, k)
+
+
 # ------------------------------------------------------------------------- attention
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("Hq,d_qk,d_v,latent", [(8, 64, 64, False), (128, 576, 512, True),
