@@ -148,6 +148,14 @@ class Stack:
             e4.record()
             ev.add("attention", e3, e4)
 
+    def own_selection(self, l):
+        """Layer l's own top-k (its indexer run as if the layer were F)."""
+        L = self.layers[l]
+        ic.indexer_scores(L["q_idx"], L["w"], L["k_idx"], self.rows, self.scores, self.ws,
+                          q_scale=L["q_scale"], k_scale=L["k_scale"], dtype=DT[self.wl.idx_dtype])
+        ic.topk(self.scores, self.rows, self.wl.k, self.idx, self.ws)
+        return self.idx.view(-1, self.wl.k).clone()
+
     def bytes_per_step(self, pattern):
         """H2D bytes of one step's inputs (F layers carry indexer inputs)."""
         n = 0
@@ -157,6 +165,78 @@ class Stack:
                     continue
                 n += t.numel() * t.element_size()
         return n
+
+
+class PagedStack(Stack):
+    """Device-resident inputs of a variable-length batch over paged caches:
+    every layer's k_I / KV caches in shuffled 128-row pages, one block table
+    and one set of sequence lengths for the batch."""
+
+    def __init__(self, wl, dev, rank=0):
+        wl = replica_workload(wl, rank)
+        self.wl = wl
+        self.dev = dev
+        self.seq, self.table, self.num_pages = synth.paged_batch(wl, dev)
+        self.lens = self.seq.cpu().tolist()
+        self.inputs = [synth.paged_layer_inputs(wl, l, self.num_pages, dev)
+                       for l in range(wl.n_layers)]
+        self.outs = [torch.empty(wl.B, wl.L, wl.Hq, wl.d_v, dtype=torch.bfloat16, device=dev)
+                     for _ in range(wl.n_layers)]
+        self.pr = ic.paged_rows(self.seq, self.table, wl.T, wl.page, self.num_pages, wl.L)
+        self.rows = ic.Rows(wl.B, wl.L, wl.T - wl.L, wl.T)
+        self.shape = ic.StackShape(self.rows, wl.H_I, wl.d_I, DT[wl.idx_dtype], wl.k, wl.Hq,
+                                   wl.d_qk, wl.d_v, DT[wl.attn_dtype], wl.d_qk, wl.d_qk, wl.scale)
+        need = max(ic.paged_workspace_size(self.shape, self.pr),
+                   ic.indexer_topk_paged_workspace_size(self.pr, wl.k),
+                   ic.sparse_attn_paged_workspace_size(self.pr, wl.k))
+        self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        ic.workspace_init(self.ws)
+        self.idx = torch.empty(wl.B, wl.L, wl.k, dtype=torch.int32, device=dev)
+        self.layers = self._layer_dicts(self.inputs, self.outs)
+        self.ld = (wl.T + 3) // 4 * 4
+        self.scores = torch.empty(wl.B, wl.L, self.ld, dtype=torch.float32, device=dev)
+        # physical cache row of each sequence's newest key (the decode step's own row)
+        last = (self.seq.to(torch.int64) - 1)
+        self.new_rows = (self.table.to(torch.int64).gather(1, (last // wl.page)[:, None])[:, 0]
+                         * wl.page + last % wl.page)
+
+    def step(self, pattern, stream=None):
+        ic.layer_stack_forward_paged(pattern, self.layers, self.shape, self.pr, self.idx, self.ws,
+                                     stream=stream)
+
+    def own_selection(self, l):
+        L = self.layers[l]
+        ic.indexer_topk_paged(L["q_idx"], L["w"], L["k_idx"], self.pr, self.wl.k, self.idx,
+                              self.ws, q_scale=L["q_scale"], k_scale_pages=L["k_scale"],
+                              dtype=DT[self.wl.idx_dtype])
+        return self.idx.view(-1, self.wl.k).clone()
+
+    def stage_step(self, pattern, ev):
+        """As Stack.stage_step, through the paged calls."""
+        wl = self.wl
+        for l, kind in enumerate(pattern):
+            L = self.layers[l]
+            if kind == "F":
+                e, e0, e1, e2 = ev.new(), ev.new(), ev.new(), ev.new()
+                e.record()
+                ic.indexer_topk_paged(L["q_idx"], L["w"], L["k_idx"], self.pr, wl.k, self.idx,
+                                      self.ws, q_scale=L["q_scale"], k_scale_pages=L["k_scale"],
+                                      dtype=DT[wl.idx_dtype])
+                e0.record()
+                ic.indexer_scores_paged(L["q_idx"], L["w"], L["k_idx"], self.pr, self.scores,
+                                        self.ws, q_scale=L["q_scale"], k_scale_pages=L["k_scale"],
+                                        dtype=DT[wl.idx_dtype])
+                e1.record()
+                ic.topk_varlen(self.scores, self.pr, wl.k, self.idx, self.ws)
+                e2.record()
+                ev.add("select", e, e0)
+                ev.add("indexer", e0, e1)
+                ev.add("topk", e1, e2)
+            e3, e4 = ev.new(), ev.new()
+            e3.record()
+            ic.sparse_attn_paged(L["q"], L["kmat"], self.idx, self.pr, wl.scale, L["out"], self.ws)
+            e4.record()
+            ev.add("attention", e3, e4)
 
 
 class Events:
@@ -194,22 +274,29 @@ def path_stages(wl):
     return ("select", "attention") if fused_selection(wl) else ("indexer", "topk", "attention")
 
 
-def algorithmic(wl):
-    """Per-launch algorithmic work of each stage (pages' definitions, all rows)."""
-    rows = [wl.q_start + i for i in range(wl.L)]
-    pairs = wl.B * sum(t + 1 for t in rows)                      # causal (query, key) pairs
-    visits = wl.B * sum(min(wl.k, t + 1) for t in rows)          # selected KV rows visited
+def algorithmic(wl, lens=None):
+    """Per-launch algorithmic work of each stage (pages' definitions, all rows).
+    lens: per-sequence key counts of a variable-length batch (default: every
+    sequence wl.T keys, queries from wl.q_start)."""
+    if lens is None:
+        rows = [wl.q_start + i for i in range(wl.L)] * wl.B       # t of every query row
+        keys = wl.B * wl.T
+    else:
+        rows = [n - wl.L + i for n in lens for i in range(wl.L)]
+        keys = sum(lens)
+    pairs = sum(t + 1 for t in rows)                              # causal (query, key) pairs
+    visits = sum(min(wl.k, t + 1) for t in rows)                  # selected KV rows visited
     ib = {"f32": 4, "bf16": 2, "e4m3": 1}[wl.idx_dtype]
     ab = {"f32": 4, "bf16": 2}[wl.attn_dtype]
     kv_w = wl.d_qk if wl.latent else wl.d_qk + wl.d_v
+    q_side = wl.B * wl.L * wl.H_I * (wl.d_I * ib + 4)
     d = {
         "indexer_flop": 2.0 * wl.H_I * wl.d_I * pairs,
-        "indexer_bytes": wl.B * (wl.T * wl.d_I * ib + wl.L * wl.H_I * (wl.d_I * ib + 4))
-        + 4.0 * pairs,
+        "indexer_bytes": keys * wl.d_I * ib + q_side + 4.0 * pairs,
         "topk_bytes": 4.0 * pairs + 4.0 * wl.B * wl.L * wl.k,
         # fused selection: the indexer's reads and the indices written, no scores
-        "select_bytes": wl.B * (wl.T * wl.d_I * ib + wl.L * wl.H_I * (wl.d_I * ib + 4))
-        + (wl.B * wl.T * 4.0 if wl.idx_dtype == "e4m3" else 0.0) + 4.0 * wl.B * wl.L * wl.k,
+        "select_bytes": keys * wl.d_I * ib + q_side
+        + (keys * 4.0 if wl.idx_dtype == "e4m3" else 0.0) + 4.0 * wl.B * wl.L * wl.k,
         "attn_flop": 2.0 * wl.Hq * (wl.d_qk + wl.d_v) * visits,
         "attn_bytes": visits * kv_w * ab + wl.B * wl.L * wl.Hq * (wl.d_qk + wl.d_v) * ab
         + 4.0 * wl.B * wl.L * wl.k,
@@ -428,6 +515,11 @@ def oracle_sample(wl, pattern, budget_s, clock=None):
     second, rows done, seconds)."""
     import dataclasses
     import oracle
+    if wl.page:
+        # a paged batch: the oracle reads plain per-sequence arrays; sample
+        # sequences of the batch's mean length
+        mean = (wl.len_min + wl.T) // 2
+        wl = dataclasses.replace(wl, T=mean, q_start=mean - wl.L, page=0, len_min=0)
     rng = np.random.default_rng(0)
     done, spent, n = 0, 0.0, 1
     sub_pattern = oracle_layers(wl, pattern)
@@ -488,7 +580,8 @@ def _oracle_inputs(wl):
 
 
 # ----------------------------------------------------------------------------- main
-DEFAULT_DECODE = (("decode_b32_t32k_bf16", 500), ("decode_b8_t200k_fp8", 150))
+DEFAULT_DECODE = (("decode_b32_t32k_bf16", 500), ("decode_b8_t200k_fp8", 150),
+                  ("decode_b32_varlen_paged_bf16", 500))
 
 
 def main():
@@ -544,6 +637,20 @@ def main():
                                   e2e=not args.no_e2e,
                                   cpu_budget=None if args.no_cpu_baseline else args.cpu_budget / 2)
             line["decode"][name] = decode_entry(entry)
+        # the FP8 prefill indexer (e4m3 operands, per-token scales) on the
+        # same 8K prefill: its indexer stage against the e4m3 tensor peak
+        fwl = synth.WORKLOADS["prefill_8k_fp8"]
+        entry = measure_stack(fwl, fwl.pattern, dev, pg, rank, world, steps=args.steps,
+                              warmup=args.warmup, graph=False, e2e=False,
+                              cpu_budget=None if args.no_cpu_baseline else args.cpu_budget / 3)
+        line["prefill_fp8"] = {
+            "metric": "prefill tok/s (IndexCache pattern) with the FP8 indexer",
+            "value": entry["value"], "unit": entry["unit"], "ms_per_step": entry["ms_per_step"],
+            "all_f": entry["all_f"], "config": entry["config"], "stages_ms": entry["stages_ms"],
+            "indexer_roofline": entry["roofline_by_stage"]["indexer"],
+            "roofline_by_stage": entry["roofline_by_stage"],
+            "cpu_baseline": entry["cpu_baseline"], "gpu_launches": entry["gpu_launches"],
+            "clocks": entry["clocks"], "device_status": entry["device_status"]}
     if rank == 0:
         print(json.dumps(line), flush=True)
     _finish(pg)
@@ -595,7 +702,7 @@ def measure_stack(wl, pattern, dev, pg, rank, world, *, steps, warmup, graph, e2
     return its JSON line (as a dict)."""
     import gc
     tokens_per_step = wl.B * wl.L
-    st = Stack(wl, dev, rank)
+    st = (PagedStack if wl.page else Stack)(wl, dev, rank)
     all_f = "F" * len(pattern)
 
     def timed(fn, n):
@@ -669,13 +776,7 @@ def measure_stack(wl, pattern, dev, pg, rank, world, *, steps, warmup, graph, e2
 
     # untimed: every layer's own top-k (each running its own indexer) and the
     # all-pairs layer overlap matrix a pattern search would consume
-    own = []
-    for l in range(len(pattern)):
-        L_ = st.layers[l]
-        ic.indexer_scores(L_["q_idx"], L_["w"], L_["k_idx"], st.rows, st.scores, st.ws,
-                          q_scale=L_["q_scale"], k_scale=L_["k_scale"], dtype=DT[wl.idx_dtype])
-        ic.topk(st.scores, st.rows, wl.k, st.idx, st.ws)
-        own.append(st.idx.view(-1, wl.k).clone())
+    own = [st.own_selection(l) for l in range(len(pattern))]
     s_sum, s_min, n_rows = overlap_matrix(own, wl.T)
     overlap = overlap_json(s_sum, s_min, n_rows, "%s, all %d layers, %d query rows"
                            % (wl.name, len(pattern), n_rows))
@@ -684,7 +785,8 @@ def measure_stack(wl, pattern, dev, pg, rank, world, *, steps, warmup, graph, e2
 
     per_step_ms = ms / steps
     value = whole_job_rate(tokens_per_step, world, per_step_ms)
-    work = algorithmic(wl)
+    lens = getattr(st, "lens", None)
+    work = algorithmic(wl, lens)
     avg = {k: float(np.mean(v)) for k, v in stages.items()}
     kind = peak_kind(clk)
     totals = {k: sum(v) for k, v in stages.items()}
@@ -697,6 +799,9 @@ def measure_stack(wl, pattern, dev, pg, rank, world, *, steps, warmup, graph, e2
     total_stage = sum(totals[k] for k in path if k in totals)
     sel_share = sum(totals.get(k, 0.0) for k in path if k != "attention") / total_stage
     bytes_in = st.bytes_per_step(pattern)
+    paged_cfg = ({"page_size": wl.page, "num_pages": st.num_pages, "seq_len_min": min(lens),
+                  "seq_len_mean": sum(lens) / len(lens), "seq_len_max": max(lens)}
+                 if wl.page else None)
     del st
     gc.collect()
     torch.cuda.empty_cache()
@@ -717,7 +822,8 @@ def measure_stack(wl, pattern, dev, pg, rank, world, *, steps, warmup, graph, e2
                    "H_I": wl.H_I, "d_I": wl.d_I, "k": wl.k, "Hq": wl.Hq, "d_qk": wl.d_qk,
                    "d_v": wl.d_v, "indexer_dtype": wl.idx_dtype,
                    "parallelism": "replicas x%d" % world,
-                   "l2": "inputs larger than L2 (%.2f GB read per step)" % (bytes_in / 1e9)},
+                   "l2": "inputs larger than L2 (%.2f GB read per step)" % (bytes_in / 1e9),
+                   **({"paged": paged_cfg} if paged_cfg else {})},
         "all_f": {"pattern": all_f, "ms_per_step": ms_all_f / steps,
                   "value": tokens_per_step * world / (ms_all_f / steps / 1e3),
                   "speedup_of_pattern": ms_all_f / ms},
@@ -1015,23 +1121,34 @@ CACHE_KEYS = ("kv", "k", "v", "k_I", "k_scale")
 def run_e2e(st, pattern, steps, dev, pg):
     """Same metric through the public API from pinned host buffers: every step
     copies that step's inputs host->device, runs the stack through
-    ic_layer_stack_forward and copies EVERY layer's output back to pinned
+    ic_layer_stack_forward (ic_layer_stack_forward_paged for a paged batch)
+    and copies EVERY layer's output back to pinned
     host memory (each layer is an independent synthetic layer, so all of
     them are the step's result).  Prefill copies every input of the step.
     Decode keeps the KV / K_I caches resident on the device (serving state)
     and copies the new token's queries, weights and its own cache rows
-    (position T-1).  The copies are torch copy_ calls on the launch stream
+    (position T-1, or each sequence's newest row in its pages).  The copies
+    are torch copy_ / index_copy_ calls on the launch stream
     around the C-ABI call."""
     wl = st.wl
     decode = wl.L == 1
+    paged = hasattr(st, "new_rows")
     host = []
     h2d = 0
+    stage = {}
     for l, kind in enumerate(pattern):
         d = {}
         for key, t in st.inputs[l].items():
             if kind == "S" and key in ("q_I", "w", "k_I", "q_scale", "k_scale"):
                 continue
-            src = t[:, wl.T - 1] if (decode and key in CACHE_KEYS) else t
+            if decode and key in CACHE_KEYS:
+                # the step's own cache rows: position T-1 (dense) or each
+                # sequence's newest row in its pages (paged)
+                src = t.index_select(0, st.new_rows) if paged else t[:, wl.T - 1]
+                if paged:
+                    stage[(l, key)] = torch.empty_like(src)
+            else:
+                src = t
             d[key] = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
             d[key].copy_(src)
             h2d += src.numel() * src.element_size()
@@ -1042,7 +1159,11 @@ def run_e2e(st, pattern, steps, dev, pg):
     def step():
         for l, d in enumerate(host):
             for key, t in d.items():
-                if decode and key in CACHE_KEYS:
+                if decode and key in CACHE_KEYS and paged:
+                    tmp = stage[(l, key)]
+                    tmp.copy_(t, non_blocking=True)
+                    st.inputs[l][key].index_copy_(0, st.new_rows, tmp)
+                elif decode and key in CACHE_KEYS:
                     st.inputs[l][key][:, wl.T - 1].copy_(t, non_blocking=True)
                 else:
                     st.inputs[l][key].copy_(t, non_blocking=True)

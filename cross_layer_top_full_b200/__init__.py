@@ -23,6 +23,7 @@ __all__ = [
     "indexer_topk_workspace_size", "indexer_topk",
     "sparse_attn_workspace_size", "sparse_attn", "sparse_attn_noalloc", "workspace_size",
     "layer_stack_forward", "indexer_scores_paged", "topk_varlen_workspace_size", "topk_varlen",
+    "indexer_topk_paged_workspace_size", "indexer_topk_paged",
     "sparse_attn_paged_workspace_size", "sparse_attn_paged", "paged_workspace_size",
     "layer_stack_forward_paged",
 ]
@@ -108,6 +109,11 @@ _SIG = {
                                                ctypes.POINTER(PagedRows), ctypes.c_int,
                                                ctypes.c_int, _P, ctypes.c_int64, _P,
                                                ctypes.c_size_t, _P]),
+    "ic_indexer_topk_paged_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(PagedRows),
+                                                               ctypes.c_int]),
+    "ic_indexer_topk_paged": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int,
+                                             ctypes.POINTER(PagedRows), ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, _P, _P, ctypes.c_size_t, _P]),
     "ic_topk_varlen_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(PagedRows), ctypes.c_int]),
     "ic_topk_varlen": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.POINTER(PagedRows), ctypes.c_int,
                                       _P, _P, ctypes.c_size_t, _P]),
@@ -345,6 +351,20 @@ def indexer_scores_paged(q_idx, w, k_pages, pr: PagedRows, scores, ws, *, q_scal
                                          _ptr(k_scale_pages), dt, ctypes.byref(pr), H_I, d_I,
                                          _ptr(scores), ld, _ptr(ws), _nbytes(ws), _stream(stream)),
            "ic_indexer_scores_paged")
+
+
+def indexer_topk_paged_workspace_size(pr: PagedRows, k: int) -> int:
+    return int(lib().ic_indexer_topk_paged_workspace_size(ctypes.byref(pr), k))
+
+
+def indexer_topk_paged(q_idx, w, k_pages, pr: PagedRows, k: int, idx, ws, *, q_scale=None,
+                       k_scale_pages=None, dtype: Optional[int] = None, stream=None) -> None:
+    dt = _dtype_of(q_idx) if dtype is None else dtype
+    H_I, d_I = q_idx.shape[-2], q_idx.shape[-1]
+    _check(lib().ic_indexer_topk_paged(_ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(k_pages),
+                                       _ptr(k_scale_pages), dt, ctypes.byref(pr), H_I, d_I, k,
+                                       _ptr(idx), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "ic_indexer_topk_paged")
 
 
 def topk_varlen_workspace_size(pr: PagedRows, k: int) -> int:

@@ -389,6 +389,39 @@ ic_status ic_indexer_scores_paged(const void* q_idx, const float* q_scale, const
                                    scores, ld_scores, status_of(ws), (cudaStream_t)stream);
 }
 
+size_t ic_indexer_topk_paged_workspace_size(const ic_paged_rows* pr, int k) {
+    (void)k;
+    if (pr == nullptr) return IC_STATUS_BYTES;
+    return IC_STATUS_BYTES + align_up(scores_bytes(plan_rows(pr)));
+}
+
+ic_status ic_indexer_topk_paged(const void* q_idx, const float* q_scale, const float* w,
+                                const void* k_pages, const float* k_scale_pages, ic_dtype dt,
+                                const ic_paged_rows* pr, int H_I, int d_I, int k, int32_t* idx,
+                                void* ws, size_t ws_bytes, void* stream) {
+    if (!paged_ok(pr, true) || !indexer_args_ok(dt, H_I, d_I) || k < 1 || k > 16384)
+        return IC_ERR_INVALID_ARG;
+    if (!indexer_tc_supported(dt, H_I, d_I)) return IC_ERR_UNSUPPORTED;
+    if (!ws_ok(ws, ws_bytes, ic_indexer_topk_paged_workspace_size(pr, k))) return IC_ERR_WORKSPACE;
+    if (pr->B == 0) return IC_OK;
+    if (!q_idx || !w || !k_pages || !idx) return IC_ERR_INVALID_ARG;
+    if (dt == IC_FP8_E4M3 && (!q_scale || !k_scale_pages)) return IC_ERR_INVALID_ARG;
+    if (dt != IC_FP8_E4M3 && (q_scale || k_scale_pages)) return IC_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    const ic_rows r = plan_rows(pr);
+    if (select_fused_applies(dt, H_I, d_I, r, k)) {
+        const ic_status st = launch_select_fused_paged(q_idx, q_scale, w, k_pages, k_scale_pages,
+                                                       dt, *pr, H_I, k, idx, status_of(ws), s);
+        if (st != IC_ERR_UNSUPPORTED) return st;
+    }
+    float* scores = reinterpret_cast<float*>(scratch_of(ws));
+    const int64_t ld = ((int64_t)r.T + 3) / 4 * 4;
+    const ic_status st = launch_indexer_tc_paged(q_idx, q_scale, w, k_pages, k_scale_pages, dt, *pr,
+                                                 H_I, d_I, scores, ld, status_of(ws), s);
+    if (st != IC_OK) return st;
+    return run_topk_varlen(scores, ld, pr, k, idx, s);
+}
+
 size_t ic_topk_varlen_workspace_size(const ic_paged_rows* pr, int k) {
     (void)pr; (void)k;
     return IC_STATUS_BYTES;

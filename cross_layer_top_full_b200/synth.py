@@ -24,6 +24,9 @@ reading notes in each entry):
   12 layers FSSFSSSSFSSS; k_I^(l) = base + 0.3 * noise^(l).
 * ``decode_b8_t200k_fp8``  8 sequences x 200000 keys, (FSSS)x12; indexer
   operands as E4M3 codes with one float32 scale per token (absmax/448).
+* ``decode_b32_varlen_paged_bf16`` 32 sequences of lengths uniform in
+  [4096, 32768], one new query each, FSSSFSSS, caches in 128-row pages
+  shuffled over one physical cache (paged_batch / paged_layer_inputs).
 """
 from __future__ import annotations
 
@@ -34,7 +37,8 @@ from typing import Dict, Optional
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "layer_inputs", "heavy_hitters", "fp8_per_token"]
+__all__ = ["Workload", "WORKLOADS", "layer_inputs", "heavy_hitters", "fp8_per_token",
+           "paged_batch", "paged_layer_inputs"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -64,6 +68,8 @@ class Workload:
     heavy_gain: float = 1.0
     chunk: int = 0          # chunked prefill: query rows per chunk (0 = one pass)
     kI_noise: float = 0.0   # chunked prefill: per-layer key noise relative to base
+    len_min: int = 0        # paged batches: sequence lengths uniform in [len_min, T]
+    page: int = 0           # paged batches: rows per page (0 = dense caches)
 
     @property
     def scale(self) -> float:
@@ -111,6 +117,14 @@ WORKLOADS: Dict[str, Workload] = {
         latent=True, pattern="FSSFSSSSFSSS", seed=3, w_std=1 / 8,
         qI_std=1 / math.sqrt(128), kI_std=1 / math.sqrt(128), q_std=1.0, kv_std=1.0,
         chunk=4096, kI_noise=0.3),
+    # a decode batch of mixed lengths over paged caches (the serving layout):
+    # the bf16 decode workload's shapes, lengths uniform in [4096, 32768],
+    # 128-row pages shuffled over one cache
+    "decode_b32_varlen_paged_bf16": Workload(
+        "decode_b32_varlen_paged_bf16", B=32, L=1, T=32768, q_start=32767, H_I=64, d_I=128,
+        k=2048, Hq=128, d_qk=576, d_v=512, idx_dtype="bf16", attn_dtype="bf16", latent=True,
+        pattern="FSSSFSSS", seed=5, w_std=1 / 8, qI_std=1 / math.sqrt(128),
+        kI_std=1 / math.sqrt(128), q_std=1.0, kv_std=1 / math.sqrt(576), len_min=4096, page=128),
     "decode_b8_t200k_fp8": Workload(
         "decode_b8_t200k_fp8", B=8, L=1, T=200000, q_start=199999, H_I=64, d_I=128, k=2048,
         Hq=128, d_qk=576, d_v=512, idx_dtype="e4m3", attn_dtype="bf16", latent=True,
@@ -225,6 +239,56 @@ def layer_inputs(wl: Workload, layer: int, device="cpu", *, indexer: bool = True
         else:
             out["k"] = _randn((B, T, wl.d_qk), wl.kv_std, device, wl.seed, "k", layer, dtype=adt)
             out["v"] = _randn((B, T, wl.d_v), wl.kv_std, device, wl.seed, "v", layer, dtype=adt)
+    return out
+
+
+def paged_batch(wl: Workload, device="cpu"):
+    """Geometry of a paged workload: (seq_lens [B] int32, block_table [B,
+    max_pages] int32, num_pages).  Lengths are uniform in [len_min, T] (the
+    first sequence T long, so T is reached); every sequence's pages are
+    distinct physical pages in a seeded random order; unused table entries
+    are -1."""
+    assert wl.page, "paged workload expected"
+    g = _gen("cpu", wl.seed, "paged")
+    lens = torch.randint(wl.len_min, wl.T + 1, (wl.B,), generator=g)
+    lens[0] = wl.T
+    P = wl.page
+    pages_per = (lens + P - 1) // P
+    max_pages = (wl.T + P - 1) // P
+    num_pages = int(pages_per.sum())
+    perm = torch.randperm(num_pages, generator=g).to(torch.int32)
+    table = torch.full((wl.B, max_pages), -1, dtype=torch.int32)
+    c = 0
+    for b in range(wl.B):
+        n = int(pages_per[b])
+        table[b, :n] = perm[c:c + n]
+        c += n
+    return lens.to(torch.int32).to(device), table.to(device), num_pages
+
+
+def paged_layer_inputs(wl: Workload, layer: int, num_pages: int, device="cpu") -> Dict[str, torch.Tensor]:
+    """Inputs of one layer of a paged workload: 'q_I' [B,L,H_I,d_I], 'w'
+    [B,L,H_I], 'q' [B,L,Hq,d_qk] as in layer_inputs, and the paged caches
+    'k_I' [num_pages*page, d_I] and 'kv' [num_pages*page, d_qk] (+ 'q_scale',
+    'k_scale' for e4m3), every physical row drawn with the workload's
+    distributions."""
+    rows = num_pages * wl.page
+    out: Dict[str, torch.Tensor] = {}
+    qI = _randn((wl.B, wl.L, wl.H_I, wl.d_I), wl.qI_std, device, wl.seed, "qI", layer, 0)
+    out["w"] = _randn((wl.B, wl.L, wl.H_I), wl.w_std, device, wl.seed, "w", layer, 0)
+    kI = _randn((rows, wl.d_I), wl.kI_std, device, wl.seed, "kI_pages", layer)
+    if wl.idx_dtype == "e4m3":
+        out["q_I"], out["q_scale"] = fp8_per_token(qI, 2)
+        out["k_I"], out["k_scale"] = fp8_per_token(kI, 1)
+    else:
+        dt = _store_dtype(wl.idx_dtype)
+        out["q_I"] = qI.to(dt).contiguous()
+        out["k_I"] = kI.to(dt).contiguous()
+    del qI, kI
+    adt = _store_dtype(wl.attn_dtype)
+    out["q"] = _randn((wl.B, wl.L, wl.Hq, wl.d_qk), wl.q_std, device, wl.seed, "q", layer, 0,
+                      dtype=adt)
+    out["kv"] = _randn((rows, wl.d_qk), wl.kv_std, device, wl.seed, "kv_pages", layer, dtype=adt)
     return out
 
 

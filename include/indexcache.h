@@ -361,6 +361,15 @@ ic_status ic_indexer_scores_paged(const void* q_idx, const float* q_scale, const
                                   float* scores, int64_t ld_scores,
                                   void* ws, size_t ws_bytes, void* stream);
 
+/* a1 + a2 over paged keys: the indices of ic_indexer_scores_paged followed
+ * by ic_topk_varlen, bit for bit (one fused kernel for decode-shaped rows, as
+ * ic_indexer_topk).  Workspace: ic_indexer_topk_paged_workspace_size. */
+size_t ic_indexer_topk_paged_workspace_size(const ic_paged_rows* pr, int k);
+ic_status ic_indexer_topk_paged(const void* q_idx, const float* q_scale, const float* w,
+                                const void* k_pages, const float* k_scale_pages, ic_dtype dt,
+                                const ic_paged_rows* pr, int H_I, int d_I, int k, int32_t* idx,
+                                void* ws, size_t ws_bytes, void* stream);
+
 /* a2 with per-sequence lengths: row (b, i) keeps the min(k, t+1) best of
  * its t+1 candidates, t = seq_lens[b] - Lq + i, as ic_topk.  Only seq_lens,
  * B, Lq and T_max of pr are read.  Workspace: ic_topk_varlen_workspace_size. */

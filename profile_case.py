@@ -29,7 +29,7 @@ DT = {"f32": ic.F32, "bf16": ic.BF16, "e4m3": ic.FP8_E4M3}
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--stage", choices=["indexer", "topk", "attention"], required=True)
+    ap.add_argument("--stage", choices=["indexer", "topk", "select", "attention"], required=True)
     ap.add_argument("--workload", default="prefill_8k_bf16")
     ap.add_argument("--rows", type=int, default=512, help="query rows kept per sequence")
     ap.add_argument("--batch", type=int, default=0, help="sequences kept (0 = all)")
@@ -54,7 +54,9 @@ def main():
     kmat = inp["kv"] if wl.latent else inp["k"]
     vmat = inp["kv"] if wl.latent else inp["v"]
     ws = torch.empty(max(ic.sparse_attn_workspace_size(R, wl.k, wl.Hq, wl.d_qk, wl.d_v,
-                                                       DT[wl.attn_dtype]), 1 << 16),
+                                                       DT[wl.attn_dtype]),
+                         ic.indexer_topk_workspace_size(R, wl.H_I, wl.d_I, DT[wl.idx_dtype], wl.k),
+                         1 << 16),
                      dtype=torch.uint8, device=dev)
     ic.workspace_init(ws)
     out = torch.empty(B, rows, wl.Hq, wl.d_v, device=dev,
@@ -68,6 +70,11 @@ def main():
     def topk():
         ic.topk(scores, R, wl.k, idx, ws)
 
+    def select():
+        ic.indexer_topk(inp["q_I"], inp["w"], inp["k_I"], R, wl.k, idx, ws,
+                        q_scale=inp.get("q_scale"), k_scale=inp.get("k_scale"),
+                        dtype=DT[wl.idx_dtype])
+
     def attention():
         ic.sparse_attn(inp["q"], kmat, wl.d_qk, vmat, wl.d_qk if wl.latent else wl.d_v, idx, R,
                        wl.d_v, wl.scale, out, ws, dtype=DT[wl.attn_dtype])
@@ -75,7 +82,7 @@ def main():
     # inputs of the later stages come from the earlier ones (untimed)
     indexer()
     topk()
-    fn = {"indexer": indexer, "topk": topk, "attention": attention}[args.stage]
+    fn = {"indexer": indexer, "topk": topk, "select": select, "attention": attention}[args.stage]
     fn()  # untimed first launch (function attributes, module load)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
