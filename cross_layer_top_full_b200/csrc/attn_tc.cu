@@ -62,8 +62,8 @@
 // per-unit masks, barriers (~227 KB).
 //
 // Decode (few query rows): each row's k indices are split over several CTA
-// pairs, which write unnormalised (O, m, l) partials, (m, l) per CTA half;
-// a small combine kernel merges them by log-sum-exp.
+// pairs, which write unnormalised partials (O as bf16; m, l as float32, per
+// CTA half); a small combine kernel merges them by log-sum-exp.
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 
@@ -182,7 +182,7 @@ struct AttnArgs {
     const __nv_bfloat16* kv;
     const int32_t* idx;
     __nv_bfloat16* out;
-    float* part_o;      // [units][128][512]   (split-k only)
+    __nv_bfloat16* part_o;  // [units][128][512] unnormalised O (split-k only)
     float2* part_ml;    // [units][2][128]     (split-k only; (m, l) of each CTA half)
     uint32_t* status;
     int k, B, Lq, q_start, T;
@@ -633,11 +633,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                             dst[v] = pk;
                         }
                     } else {
-                        float4* dst = reinterpret_cast<float4*>(args.part_o + ((int64_t)u.unit * HQ + h) * DV + col);
+                        // unnormalised partial O as bf16 (the combine scales and normalises)
+                        uint4* dst = reinterpret_cast<uint4*>(args.part_o + ((int64_t)u.unit * HQ + h) * DV + col);
 #pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                                 __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+                        for (int v = 0; v < 4; ++v) {
+                            uint4 pk;
+                            pk.x = pack_bf16(__uint_as_float(o[8 * v + 0]), __uint_as_float(o[8 * v + 1]));
+                            pk.y = pack_bf16(__uint_as_float(o[8 * v + 2]), __uint_as_float(o[8 * v + 3]));
+                            pk.z = pack_bf16(__uint_as_float(o[8 * v + 4]), __uint_as_float(o[8 * v + 5]));
+                            pk.w = pack_bf16(__uint_as_float(o[8 * v + 6]), __uint_as_float(o[8 * v + 7]));
+                            dst[v] = pk;
+                        }
                     }
                 }
                 tc_fence_before();
@@ -799,9 +805,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
 }
 
 // Merge split-k partials: out = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c,
-// with (m_c, l_c) of the CTA half that produced the columns.
+// with (m_c, l_c) of the CTA half that produced the columns (O_c in bf16:
+// 2^-9 relative, inside the attention tolerance).
 __global__ void __launch_bounds__(128)
-attn_combine_kernel(const float* __restrict__ part_o, const float2* __restrict__ part_ml,
+attn_combine_kernel(const __nv_bfloat16* __restrict__ part_o, const float2* __restrict__ part_ml,
                     int splits, __nv_bfloat16* __restrict__ out) {
     const int64_t row = blockIdx.x;
     const int h = blockIdx.y;
@@ -821,11 +828,11 @@ attn_combine_kernel(const float* __restrict__ part_o, const float2* __restrict__
             if (!(ml.y > 0.f)) continue;
             const float wgt = exp2f(ml.x - M);
             den += wgt * ml.y;
-            const float4 o = *reinterpret_cast<const float4*>(part_o + (u * HQ + h) * DV + d);
-            num.x += wgt * o.x;
-            num.y += wgt * o.y;
-            num.z += wgt * o.z;
-            num.w += wgt * o.w;
+            const uint2 o = *reinterpret_cast<const uint2*>(part_o + (u * HQ + h) * DV + d);
+            num.x += wgt * __uint_as_float(o.x << 16);
+            num.y += wgt * __uint_as_float(o.x & 0xffff0000u);
+            num.z += wgt * __uint_as_float(o.y << 16);
+            num.w += wgt * __uint_as_float(o.y & 0xffff0000u);
         }
     }
     const float inv = den > 0.f ? 1.f / den : 0.f;
@@ -908,7 +915,7 @@ size_t attn_tc_scratch_bytes(ic_rows r, int k, int64_t max_units) {
     plan_splits(r, k, splits, kps, max_units);
     if (splits <= 1) return 0;
     const size_t units = (size_t)r.B * r.Lq * splits;
-    return units * HQ * DV * sizeof(float) + 256 + units * 2 * HQ * sizeof(float2);
+    return units * HQ * DV * sizeof(__nv_bfloat16) + 256 + units * 2 * HQ * sizeof(float2);
 }
 
 namespace {
@@ -976,10 +983,10 @@ ic_status attn_tc_core(const void* q, const void* kv, const int32_t* idx, int k,
     if (a.splits > 1) {
         if (scratch_bytes < attn_tc_scratch_bytes(r, k, max_units) || scratch == nullptr)
             return IC_ERR_WORKSPACE;
-        a.part_o = static_cast<float*>(scratch);
-        a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(scratch) +
-                                              (size_t)units * HQ * DV * sizeof(float) + 256 -
-                                              (((size_t)units * HQ * DV * sizeof(float)) & 255));
+        const size_t o_bytes = (size_t)units * HQ * DV * sizeof(__nv_bfloat16);
+        a.part_o = static_cast<__nv_bfloat16*>(scratch);
+        a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(scratch) + o_bytes + 256 -
+                                              (o_bytes & 255));
     }
     if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES) != cudaSuccess)

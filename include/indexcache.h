@@ -234,7 +234,7 @@ ic_status ic_sparse_attn(const void* q, const void* kmat, int64_t k_row_stride,
  * Same arguments, layouts and results as ic_sparse_attn with
  * kmat = vmat = kv and row strides 576, except that the split-k partials of
  * decode live in a fixed device array inside the library of
- * IC_NOALLOC_SCRATCH_BYTES bytes (about 16 MiB; every GPU that loads the
+ * IC_NOALLOC_SCRATCH_BYTES bytes (about 8 MiB; every GPU that loads the
  * library holds it until the process exits), room for 64 partial rows
  * (query rows x splits).  Among its split counts this call only considers
  * those that keep B*Lq*splits <= 64, so it may split less finely than
@@ -253,7 +253,7 @@ ic_status ic_sparse_attn(const void* q, const void* kmat, int64_t k_row_stride,
  * cleared at the start of each call): calls whose kernels overlap on the GPU
  * race on it, so serialise them (one stream, one thread).
  */
-#define IC_NOALLOC_SCRATCH_BYTES ((16u << 20) + (128u << 10) + 512u)
+#define IC_NOALLOC_SCRATCH_BYTES ((8u << 20) + (128u << 10) + 512u)
 ic_status ic_sparse_attn_noalloc(const void* q, const void* kv, const int32_t* idx, int k,
                                  ic_rows r, float scale, void* out, int32_t* device_status,
                                  void* stream);
