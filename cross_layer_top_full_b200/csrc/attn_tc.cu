@@ -61,6 +61,13 @@
 // tiles of 16 KB + 256 B of per-head offsets (written by the partner),
 // per-unit masks, barriers (~227 KB).
 //
+// Every wait is bounded (sm100.cuh); a wait that runs out records its site
+// in the second status word: 1-3 gather (info_empty, scan_done, kv_empty),
+// 4-6 exchange (info_full, s_full, peer_free), 7-11 softmax (info_full,
+// own_full, x_full, o_done, o_final), 12-20 S issuer (info_full, q_empty,
+// q_full, q_tmem_full, kv_full, s_free, next info_full, next q_empty, drain),
+// 21-24 P V issuer (info_full, p_full, o_free, drain).
+//
 // Decode (few query rows): each row's k indices are split over several CTA
 // pairs, which write unnormalised partials (O as bf16; m, l as float32, per
 // CTA half); a small combine kernel merges them by log-sum-exp.
@@ -298,7 +305,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             const Unit u = decode_unit(args, seq);
             const int32_t* idx_row = args.idx + (int64_t)u.row * args.k;
             const int ip = n & 1;
-            if (!warp_wait(&bars->info_empty[ip], ((n >> 1) & 1) ^ 1, status, abort)) break;
+            if (!warp_wait(&bars->info_empty[ip], ((n >> 1) & 1) ^ 1, status, abort, 1)) break;
             // validity masks of the unit's blocks and its last valid index; the
             // loads go out SCAN_BATCH at a time so the scan costs a few memory
             // round trips, not one per 32*GW indices
@@ -330,7 +337,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             if (lane == 0) bars->red[ip][warp] = last;
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->scan_done[ip]);
-            if (!warp_wait(&bars->scan_done[ip], (n >> 1) & 1, status, abort)) break;
+            if (!warp_wait(&bars->scan_done[ip], (n >> 1) & 1, status, abort, 2)) break;
             last = bars->red[ip][0];
 #pragma unroll
             for (int w = 1; w < GW; ++w) last = max(last, bars->red[ip][w]);
@@ -355,7 +362,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     v_next = (lane < KPW && e1 < u.e1) ? idx_row[e1] : -1;
                 }
                 const int row_lane = idx_valid(v_lane, u.t, args.T) ? kv_row(args, u.b, v_lane) : oob_row;
-                if (!warp_wait(&bars->kv_empty[s], ((g / NSTAGE) & 1) ^ 1, status, abort)) {
+                if (!warp_wait(&bars->kv_empty[s], ((g / NSTAGE) & 1) ^ 1, status, abort, 3)) {
                     ok_all = false;
                     break;
                 }
@@ -387,6 +394,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             }
             if (!ok_all) break;
         }
+        // drain: every gather this warp issued has landed before the CTA may
+        // exit (on the abort path some were never consumed by an S MMA); a
+        // stage another warp never filled gives up after 50 ms
+        if (lane == 0)
+            for (uint32_t j = g > (uint32_t)NSTAGE ? g - NSTAGE : 0; j < g; ++j)
+                mbar_wait_drain(&bars->kv_full[j % NSTAGE], (j / NSTAGE) & 1, 50000000ull);
+        __syncwarp();
     } else if (warp < W_Y) {
         // ------------------------------------------------------------ exchange
         const int quad = warp & 3;                // TMEM lanes 32*quad .. +31
@@ -400,7 +414,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         bool ok = true;
         for (int seq = pair; seq < args.n_units && ok; seq += n_pairs, ++n) {
             const int ip = n & 1;
-            if (!warp_wait(&bars->info_full[ip], (n >> 1) & 1, status, abort)) break;
+            if (!warp_wait(&bars->info_full[ip], (n >> 1) & 1, status, abort, 4)) break;
             const int nb = bars->n_blocks[ip];
             __syncwarp();
             if (nb > 0) {
@@ -430,7 +444,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             for (int j = 0; j < nb; ++j, ++g) {
                 const int sb = g % NSBUF;
                 const int slot = g & 1;
-                if (!warp_wait(&bars->s_full[sb], (g / NSBUF) & 1, status, abort)) { ok = false; break; }
+                if (!warp_wait(&bars->s_full[sb], (g / NSBUF) & 1, status, abort, 5)) { ok = false; break; }
                 tc_fence_after();
                 float x[NB];
                 {
@@ -473,7 +487,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 // two heads' offsets per 32-bit word: lane 2i sends heads 2i, 2i+1
                 const uint32_t m16_odd = __shfl_down_sync(0xffffffffu, m16, 1);
                 // the partner's softmax warp q must have read this inbox slot (block g-2)
-                if (!warp_wait_cluster(&bars->peer_free[slot][quad], ((g >> 1) & 1) ^ 1, status, abort)) {
+                if (!warp_wait_cluster(&bars->peer_free[slot][quad], ((g >> 1) & 1) ^ 1, status, abort, 6)) {
                     ok = false;
                     break;
                 }
@@ -505,7 +519,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         for (int seq = pair; seq < args.n_units && ok; seq += n_pairs, ++n) {
             const Unit u = decode_unit(args, seq);
             const int ip = n & 1;
-            if (!warp_wait(&bars->info_full[ip], (n >> 1) & 1, status, abort)) { ok = false; break; }
+            if (!warp_wait(&bars->info_full[ip], (n >> 1) & 1, status, abort, 7)) { ok = false; break; }
             const int nb = bars->n_blocks[ip];
             float m_use = 0.f;      // running max (log2 units); meaningful once m_set
             bool m_set = false;
@@ -517,7 +531,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 const uint32_t m_lo = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j];
                 const uint32_t m_hi = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j + 1];
                 // S(g) is final in TMEM and the exchange warp has read it
-                if (!warp_wait(&bars->own_full[sb][quad], (g / NSBUF) & 1, status, abort)) {
+                if (!warp_wait(&bars->own_full[sb][quad], (g / NSBUF) & 1, status, abort, 8)) {
                     ok = false;
                     break;
                 }
@@ -525,7 +539,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 uint32_t s0[32], s1[32], par[NB / 2];
                 tmem_ld32(t_lane + TM_S + 64 * sb, s0);
                 tmem_ld32(t_lane + TM_S + 64 * sb + 32, s1);
-                if (!warp_wait_cluster(&bars->x_full[slot][quad], (g >> 1) & 1, status, abort)) {
+                if (!warp_wait_cluster(&bars->x_full[slot][quad], (g >> 1) & 1, status, abort, 9)) {
                     ok = false;
                     break;
                 }
@@ -585,7 +599,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 l = (rescale ? l * alpha : l) + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
                 if (rescale) {
                     // O and l must hold P V of block g-1 before they are rescaled
-                    if (!warp_wait(&bars->o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, status, abort)) {
+                    if (!warp_wait(&bars->o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, status, abort, 10)) {
                         ok = false;
                         break;
                     }
@@ -611,7 +625,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             const bool split = args.splits > 1;
             float l_all = 0.f;
             if (nb > 0) {
-                if (!warp_wait(&bars->o_final, o_use & 1, status, abort)) { ok = false; break; }
+                if (!warp_wait(&bars->o_final, o_use & 1, status, abort, 11)) { ok = false; break; }
                 tc_fence_after();
                 l_all = m_set ? l : 0.f;
                 const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
@@ -684,24 +698,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     nb = nb_next;
                     nb_next = -1;
                 } else {
-                    if (!mbar_wait(&bars->info_full[n & 1], (n >> 1) & 1, status, abort)) break;
+                    if (!mbar_wait(&bars->info_full[n & 1], (n >> 1) & 1, status, abort, 12)) break;
                     nb = bars->n_blocks[n & 1];
                     mbar_arrive(&bars->info_empty[n & 1]);
                 }
                 if (nb == 0) continue;
                 if (!q_loaded_next) {
-                    if (o_use > 0 && !mbar_wait(&bars->q_empty, (o_use - 1) & 1, status, abort)) break;
+                    if (o_use > 0 && !mbar_wait(&bars->q_empty, (o_use - 1) & 1, status, abort, 13)) break;
                     load_q(seq);
                 }
                 q_loaded_next = false;
-                if (!mbar_wait(&bars->q_full, o_use & 1, status, abort) ||
-                    !mbar_wait(&bars->q_tmem_full, o_use & 1, status, abort))
+                if (!mbar_wait(&bars->q_full, o_use & 1, status, abort, 14) ||
+                    !mbar_wait(&bars->q_tmem_full, o_use & 1, status, abort, 15))
                     break;
                 for (int j = 0; j < nb; ++j, ++g) {
                     const int sb = g % NSBUF;
                     const int ks = g % NSTAGE;
-                    if (!mbar_wait(&bars->kv_full[ks], (g / NSTAGE) & 1, status, abort) ||
-                        !mbar_wait(&bars->s_free[sb], ((g / NSBUF) & 1) ^ 1, status, abort)) {
+                    if (!mbar_wait(&bars->kv_full[ks], (g / NSTAGE) & 1, status, abort, 16) ||
+                        !mbar_wait(&bars->s_free[sb], ((g / NSBUF) & 1) ^ 1, status, abort, 17)) {
                         ok = false;
                         break;
                     }
@@ -736,11 +750,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 mma_commit(&bars->q_empty);
                 if (seq + n_pairs < args.n_units) {
                     const int n1 = n + 1;
-                    if (!mbar_wait(&bars->info_full[n1 & 1], (n1 >> 1) & 1, status, abort)) break;
+                    if (!mbar_wait(&bars->info_full[n1 & 1], (n1 >> 1) & 1, status, abort, 18)) break;
                     nb_next = bars->n_blocks[n1 & 1];
                     mbar_arrive(&bars->info_empty[n1 & 1]);
                     if (nb_next > 0) {
-                        if (!mbar_wait(&bars->q_empty, o_use & 1, status, abort)) break;
+                        if (!mbar_wait(&bars->q_empty, o_use & 1, status, abort, 19)) break;
                         load_q(seq + n_pairs);
                         q_loaded_next = true;
                     }
@@ -749,7 +763,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             }
             if (issued) {
                 mma_commit(&bars->drain[0]);   // every MMA this thread issued has finished
-                mbar_wait(&bars->drain[0], 0, status, abort);
+                mbar_wait(&bars->drain[0], 0, status, abort, 20);
             }
         }
     } else {
@@ -760,14 +774,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             bool issued = false, ok = true;
             int n = 0;
             for (int seq = pair; seq < args.n_units && ok; seq += n_pairs, ++n) {
-                if (!mbar_wait(&bars->info_full[n & 1], (n >> 1) & 1, status, abort)) break;
+                if (!mbar_wait(&bars->info_full[n & 1], (n >> 1) & 1, status, abort, 21)) break;
                 const int nb = bars->n_blocks[n & 1];
                 mbar_arrive(&bars->info_empty[n & 1]);
                 if (nb == 0) continue;
                 for (int j = 0; j < nb; ++j, ++g) {
                     const int sb = g % NSBUF;
-                    if (!mbar_wait(&bars->p_full[sb], (g / NSBUF) & 1, status, abort) ||
-                        (j == 0 && o_use > 0 && !mbar_wait(&bars->o_free, (o_use - 1) & 1, status, abort))) {
+                    if (!mbar_wait(&bars->p_full[sb], (g / NSBUF) & 1, status, abort, 22) ||
+                        (j == 0 && o_use > 0 && !mbar_wait(&bars->o_free, (o_use - 1) & 1, status, abort, 23))) {
                         ok = false;
                         break;
                     }
@@ -790,7 +804,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             }
             if (issued) {
                 mma_commit(&bars->drain[1]);
-                mbar_wait(&bars->drain[1], 0, status, abort);
+                mbar_wait(&bars->drain[1], 0, status, abort, 24);
             }
         }
     }

@@ -87,11 +87,19 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 #endif
 }
 
+// Record a wait that ran out of time: the timeout bit, and in the second
+// word of the status area the site (a small id naming the wait, and the
+// CTA) of the first such wait, for diagnosis.
+__device__ __forceinline__ void flag_timeout(uint32_t* status, uint32_t site) {
+    flag_status(status, IC_DEV_TIMEOUT);
+    if (status) atomicCAS(status + 1, 0u, (site & 0xffu) | ((uint32_t)blockIdx.x << 8));
+}
+
 // Wait until the phase with the given parity of `bar` has completed.
-// Returns false (and flags IC_DEV_TIMEOUT, raises *abort) on timeout, or
-// returns false at once if *abort is already raised.
+// Returns false (and flags IC_DEV_TIMEOUT with `site`, raises *abort) on
+// timeout, or returns false at once if *abort is already raised.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
-                                          volatile int* abort) {
+                                          volatile int* abort, uint32_t site = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t n = 0;; ++n) {
@@ -99,11 +107,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
         if ((n & 63u) == 63u) {
             if (*abort) return false;
             if (globaltimer() - t0 > IC_WAIT_LIMIT_NS) {
-                flag_status(status, IC_DEV_TIMEOUT);
+                flag_timeout(status, site);
                 *abort = 1;
                 return false;
             }
         }
+    }
+}
+
+// A wait that ignores the abort flag, with its own limit: for draining a
+// CTA's own in-flight copies before it exits on the abort path.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t n = 0;; ++n) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
+        if ((n & 63u) == 63u && globaltimer() - t0 > limit_ns) return false;
     }
 }
 
@@ -335,7 +354,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster_sleep(uint64_t* bar, uint3
 
 // Bounded wait with cluster-scope acquire (for barriers other CTAs arrive on).
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* status,
-                                                  volatile int* abort) {
+                                                  volatile int* abort, uint32_t site = 0) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t n = 0;; ++n) {
@@ -343,7 +362,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
         if ((n & 63u) == 63u) {
             if (*abort) return false;
             if (globaltimer() - t0 > IC_WAIT_LIMIT_NS) {
-                flag_status(status, IC_DEV_TIMEOUT);
+                flag_timeout(status, site);
                 *abort = 1;
                 return false;
             }
@@ -406,18 +425,18 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // Every lane gets the same answer, so a timeout can never leave part of a
 // warp inside a warp-synchronous operation.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
-                                          volatile int* abort) {
+                                          volatile int* abort, uint32_t site = 0) {
     int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status, abort) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status, abort, site) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;
 }
 
 __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* status,
-                                                  volatile int* abort) {
+                                                  volatile int* abort, uint32_t site = 0) {
     int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait_cluster(bar, parity, status, abort) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_cluster(bar, parity, status, abort, site) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;

@@ -373,7 +373,8 @@ def test_latent_attention_sharp_logits(dev, gain, rows, k):
     ic.sparse_attn(q, kv, 576, kv, 576, idx, rows, 512, 576 ** -0.5, out, ws)
     torch.cuda.synchronize()
     assert ic.kernel_launches(6) - tc0 == 1
-    assert ic.read_status(ws) == 0
+    site = int(ws[4:8].view(torch.int32).item())     # the first wait that ran out, if any
+    assert ic.read_status(ws) == 0, "wait site %d of CTA %d ran out" % (site & 255, site >> 8)
     qh, kvh = host64(q), host64(kv)
     # the test really is sharp: base-2 logits of the first row reach tens
     logit2 = (qh[0, 0] @ kvh[0, :T].T) * 576 ** -0.5 / np.log(2)
