@@ -160,3 +160,19 @@ def test_overlap_matrix_matches_the_oracle():
         assert s_sum[l, l].item() == pytest.approx(rows)
     js = bench.overlap_json(s_sum, s_min, n, "test")
     assert js["layers"] == L and len(js["mean"]) == L and js["mean"][0][0] == 1.0
+
+
+def test_varlen_counts_follow_the_sequence_lengths():
+    """A variable-length batch: pairs, visits and bytes from each sequence's
+    own length (closed forms per sequence), and the fused selection's bytes
+    carry no score traffic."""
+    wl = synth.WORKLOADS["decode_b32_varlen_paged_bf16"]
+    lens = [32768, 5000, 4096, 20000]
+    w = bench.algorithmic(wl, lens)
+    assert w["pairs"] == sum(lens)                        # one query row at t = n - 1 each
+    assert w["visits"] == sum(min(wl.k, n) for n in lens)
+    q_side = wl.B * 1 * wl.H_I * (wl.d_I * 2 + 4)
+    assert w["indexer_bytes"] == pytest.approx(sum(lens) * wl.d_I * 2 + q_side + 4 * sum(lens))
+    assert w["select_bytes"] == pytest.approx(sum(lens) * wl.d_I * 2 + q_side + 4 * wl.B * wl.k)
+    assert bench.path_stages(wl) == ("select", "attention")
+    assert bench.path_stages(synth.WORKLOADS["prefill_8k_bf16"]) == ("indexer", "topk", "attention")
