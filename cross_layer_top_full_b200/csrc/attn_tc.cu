@@ -116,15 +116,16 @@ constexpr int TMEM_COLS = 512;
 constexpr uint32_t TM_O = 0;
 constexpr uint32_t TM_S = 256;                      // S/P buffer b at TM_S + 64 b
 constexpr uint32_t TM_QT = TM_S + 64 * NSBUF;       // Q_r slice 3 (32 cols) + rope (16 cols), bf16 pairs
+constexpr uint32_t TM_MX = TM_QT + 48;              // block maximum of the full logits, per S buffer
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_THRESHOLD = 8.f;            // log2 units
-static_assert(TM_QT + 48 <= TMEM_COLS, "tensor memory budget");
+static_assert(TM_MX + NSBUF <= TMEM_COLS, "tensor memory budget");
 
 struct __align__(8) AttnBars {
     uint64_t q_full, q_empty, q_tmem_full;
     uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
     uint64_t s_full[NSBUF], s_free[NSBUF];
-    uint64_t own_full[NSBUF][4];    // exchange warp q has read S of the buffer: P may overwrite it
+    uint64_t own_full[NSBUF][4];    // exchange warp q: the buffer holds the full logits and their max
     uint64_t p_full[NSBUF];         // softmax warps -> MMA: P in TMEM
     uint64_t x_full[2][4];          // [inbox slot][quad]: the partner's 32 rows (counted in bytes)
     uint64_t peer_free[2][4];       // the partner's softmax warp q has read its inbox slot
@@ -408,6 +409,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t x_remote = map_to_rank(smem_base + OFF_X + h * 128, peer);
         const uint32_t xoff_remote = map_to_rank(smem_base + OFF_XOFF + (h >> 1) * 4, peer);
+        const uint32_t free_remote0 = map_to_rank(smem_u32(&bars->peer_free[0][quad]), peer);
+        const uint32_t free_remote1 = map_to_rank(smem_u32(&bars->peer_free[1][quad]), peer);
         const float sl2 = args.scale_log2;
         uint32_t g = 0;
         int n = 0;
@@ -444,6 +447,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             for (int j = 0; j < nb; ++j, ++g) {
                 const int sb = g % NSBUF;
                 const int slot = g & 1;
+                // arm this CTA's inbox slot for the partner's half of block g
+                if (lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD + X_OFF_QUAD);
                 if (!warp_wait(&bars->s_full[sb], (g / NSBUF) & 1, status, abort, 5)) { ok = false; break; }
                 tc_fence_after();
                 float x[NB];
@@ -458,49 +463,86 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                         x[32 + c] = __uint_as_float(r1[c]) * sl2;
                     }
                 }
-                // S(g) is in registers: the softmax warp of this quadrant may now
-                // read it and overwrite it with P
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
                 // the offset is the largest VALID partial logit of the block (keys
-                // of invalid indices are zero rows whose logits would pull it off)
+                // of invalid indices are zero rows whose logits would pull it off);
+                // invalid keys become -inf from here on
                 const uint32_t m_lo = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j];
                 const uint32_t m_hi = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j + 1];
-                float mb;
-                if ((m_lo & m_hi) != 0xffffffffu) {
-                    float xm[NB];
+                const bool holes = (m_lo & m_hi) != 0xffffffffu;
+                if (holes) {
 #pragma unroll
                     for (int c = 0; c < NB; ++c)
-                        xm[c] = (((c < 32 ? m_lo : m_hi) >> (c & 31)) & 1u) ? x[c] : -INFINITY;
-                    mb = max64(xm);
-                } else {
-                    mb = max64(x);
+                        if (!(((c < 32 ? m_lo : m_hi) >> (c & 31)) & 1u)) x[c] = -INFINITY;
                 }
+                const float mb = max64(x);
                 // offset as float16 (saturated); the differences are taken from
                 // the rounded offset, so offset + difference rebuilds the value
                 const uint32_t m16 = half2_sat(mb, 0.f) & 0xffffu;
                 const float mf = f16_lo(m16);
-                uint32_t d[NB / 2];
-#pragma unroll
-                for (int c = 0; c < NB / 2; ++c) d[c] = half2_sat(x[2 * c] - mf, x[2 * c + 1] - mf);
                 // two heads' offsets per 32-bit word: lane 2i sends heads 2i, 2i+1
                 const uint32_t m16_odd = __shfl_down_sync(0xffffffffu, m16, 1);
-                // the partner's softmax warp q must have read this inbox slot (block g-2)
+                // the partner's exchange warp q must have read this inbox slot (block g-2)
                 if (!warp_wait_cluster(&bars->peer_free[slot][quad], ((g >> 1) & 1) ^ 1, status, abort, 6)) {
                     ok = false;
                     break;
                 }
-                // row h of the partner's inbox; each st.async counts its bytes on
-                // the partner's x_full (no fence or arrive on this side)
-                const uint32_t xr = x_remote + slot * X_TILE;
-                const uint32_t br = map_to_rank(smem_u32(&bars->x_full[slot][quad]), peer);
+                {
+                    // row h of the partner's inbox, 16 bytes (8 keys) at a time; each
+                    // st.async counts its bytes on the partner's x_full (no fence or
+                    // arrive on this side)
+                    const uint32_t xr = x_remote + slot * X_TILE;
+                    const uint32_t br = map_to_rank(smem_u32(&bars->x_full[slot][quad]), peer);
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    st_async_v4(xr + ((c ^ (h & 7)) << 4), d[4 * c], d[4 * c + 1], d[4 * c + 2],
-                                d[4 * c + 3], br);
-                if ((lane & 1) == 0)
-                    st_async_b32(xoff_remote + slot * X_OFF, m16 | (m16_odd << 16), br);
+                    for (int c = 0; c < 8; ++c)
+                        st_async_v4(xr + ((c ^ (h & 7)) << 4),
+                                    half2_sat(x[8 * c + 0] - mf, x[8 * c + 1] - mf),
+                                    half2_sat(x[8 * c + 2] - mf, x[8 * c + 3] - mf),
+                                    half2_sat(x[8 * c + 4] - mf, x[8 * c + 5] - mf),
+                                    half2_sat(x[8 * c + 6] - mf, x[8 * c + 7] - mf), br);
+                    if ((lane & 1) == 0)
+                        st_async_b32(xoff_remote + slot * X_OFF, m16 | (m16_odd << 16), br);
+                }
+                // the partner's half of block g: full logits = own (float32) +
+                // the partner's offset + float16 difference
+                if (!warp_wait_cluster(&bars->x_full[slot][quad], (g >> 1) & 1, status, abort, 9)) {
+                    ok = false;
+                    break;
+                }
+                {
+                    const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + slot * X_TILE + h * 128);
+                    const uint32_t ow = reinterpret_cast<const uint32_t*>(smem + OFF_XOFF + slot * X_OFF)[h >> 1];
+                    const float pf = (h & 1) ? f16_hi(ow) : f16_lo(ow);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 w4 = xp[c ^ (h & 7)];
+                        const uint32_t pw4[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            x[8 * c + 2 * e] += add_f16_f32((unsigned short)(pw4[e] & 0xffffu), pf);
+                            x[8 * c + 2 * e + 1] += add_f16_f32((unsigned short)(pw4[e] >> 16), pf);
+                        }
+                    }
+                }
+                // every inbox value of this slot has been read: hand it back
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote_relaxed(slot ? free_remote1 : free_remote0);
+                const float mloc = max64(x);
+                // full logits over S, their maximum in its column: the softmax warp's input
+                {
+                    uint32_t w0[32], w1[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        w0[c] = __float_as_uint(x[c]);
+                        w1[c] = __float_as_uint(x[32 + c]);
+                    }
+                    tmem_st32(t_lane + TM_S + 64 * sb, w0);
+                    tmem_st32(t_lane + TM_S + 64 * sb + 32, w1);
+                    tmem_st1(t_lane + TM_MX + sb, __float_as_uint(mloc));
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
             }
             // the unit's masks have been read: the gather warps may refill them
             __syncwarp();
@@ -511,8 +553,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         const int quad = warp & 3;
         const int h = quad * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
-        const uint32_t free_remote0 = map_to_rank(smem_u32(&bars->peer_free[0][quad]), peer);
-        const uint32_t free_remote1 = map_to_rank(smem_u32(&bars->peer_free[1][quad]), peer);
         uint32_t g = 0, o_use = 0;
         int n = 0;
         bool ok = true;
@@ -526,61 +566,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             float l = 0.f;          // running sum of the bf16-rounded P
             for (int j = 0; j < nb; ++j, ++g) {
                 const int sb = g % NSBUF;
-                const int slot = g & 1;
-                if (lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD + X_OFF_QUAD);
-                const uint32_t m_lo = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j];
-                const uint32_t m_hi = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j + 1];
-                // S(g) is final in TMEM and the exchange warp has read it
+                // the exchange warp has put the block's full logits (invalid keys
+                // -inf) over S and their maximum in its column
                 if (!warp_wait(&bars->own_full[sb][quad], (g / NSBUF) & 1, status, abort, 8)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                uint32_t s0[32], s1[32], par[NB / 2];
-                tmem_ld32(t_lane + TM_S + 64 * sb, s0);
-                tmem_ld32(t_lane + TM_S + 64 * sb + 32, s1);
-                if (!warp_wait_cluster(&bars->x_full[slot][quad], (g >> 1) & 1, status, abort, 9)) {
-                    ok = false;
-                    break;
-                }
-                float pf;
-                {
-                    const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + slot * X_TILE + h * 128);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 w4 = xp[c ^ (h & 7)];
-                        par[4 * c] = w4.x;
-                        par[4 * c + 1] = w4.y;
-                        par[4 * c + 2] = w4.z;
-                        par[4 * c + 3] = w4.w;
-                    }
-                    const uint32_t ow = reinterpret_cast<const uint32_t*>(smem + OFF_XOFF + slot * X_OFF)[h >> 1];
-                    pf = (h & 1) ? f16_hi(ow) : f16_lo(ow);
-                }
-                tmem_ld_wait();
-                // full logits of the 64 keys (log2 units): own half in float32 plus
-                // the partner's (offset + float16 difference); masked keys -> -inf
                 float sv[NB];
+                float mloc;
+                {
+                    uint32_t s0[32], s1[32];
+                    tmem_ld32(t_lane + TM_S + 64 * sb, s0);
+                    tmem_ld32(t_lane + TM_S + 64 * sb + 32, s1);
+                    mloc = __uint_as_float(tmem_ld1(t_lane + TM_MX + sb));
+                    tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < NB / 2; ++c) {
-                    sv[c] = fmaf(__uint_as_float(s0[c]), args.scale_log2,
-                                 add_f16_f32((unsigned short)((c & 1) ? (par[c >> 1] >> 16) : (par[c >> 1] & 0xffffu)), pf));
-                    sv[32 + c] = fmaf(__uint_as_float(s1[c]), args.scale_log2,
-                                      add_f16_f32((unsigned short)((c & 1) ? (par[16 + (c >> 1)] >> 16)
-                                                                           : (par[16 + (c >> 1)] & 0xffffu)), pf));
-                }
-                if ((m_lo & m_hi) != 0xffffffffu) {
-#pragma unroll
-                    for (int kk = 0; kk < NB; ++kk) {
-                        const uint32_t mw = kk < 32 ? m_lo : m_hi;
-                        if (!((mw >> (kk & 31)) & 1u)) sv[kk] = -INFINITY;
+                    for (int c = 0; c < 32; ++c) {
+                        sv[c] = __uint_as_float(s0[c]);
+                        sv[32 + c] = __uint_as_float(s1[c]);
                     }
                 }
-                const float mloc = max64(sv);
-                // every inbox value of this slot has been consumed (mloc depends on
-                // all of them): hand the slot back to the partner's exchange warp
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote_relaxed(slot ? free_remote1 : free_remote0);
                 bool rescale = false;
                 float alpha = 1.f;
                 if (mloc > -INFINITY && (!m_set || mloc > m_use + RESCALE_THRESHOLD)) {
