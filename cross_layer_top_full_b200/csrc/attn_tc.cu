@@ -603,7 +603,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     ps[x & 3] += __uint_as_float(pw[x] << 16) + __uint_as_float(pw[x] & 0xffff0000u);
                 }
                 l = (rescale ? l * alpha : l) + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-                if (rescale) {
+                // The decision is per head (lane), but the O rescale below is
+                // warp-collective (the wait shuffles over the whole warp and the
+                // TMEM loads and stores are .aligned): the warp takes it when any
+                // of its heads needs it, and the other heads scale by 1.
+                if (__any_sync(0xffffffffu, rescale)) {
+                    const float a = rescale ? alpha : 1.f;
                     // O and l must hold P V of block g-1 before they are rescaled
                     if (!warp_wait(&bars->o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, status, abort, 10)) {
                         ok = false;
@@ -616,7 +621,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                         tmem_ld32(t_lane + TM_O + 32 * c, o);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+                        for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * a);
                         tmem_st32(t_lane + TM_O + 32 * c, o);
                     }
                 }
