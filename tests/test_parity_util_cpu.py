@@ -68,11 +68,14 @@ def test_check_attention():
     bad[1, 2, 3, 4] += 2 * attn_bound(ref[1, 2, 3, 4])
     with pytest.raises(AssertionError, match="diff"):
         check_attention(bad, ref, "planted")
-    # the bound is the larger of the two terms, not their sum: an error of
-    # 1.5e-2 on an output of 1.0 fails (the sum form would allow 2e-2)
-    one = np.ones((4, 8))
+    # the bound is the sum of the two terms: on an output of 1.0 an error of
+    # 1.9e-2 passes elementwise and 2.1e-2 fails
+    one = np.ones((40, 80))
+    near = one.copy()
+    near[2, 3] += 1.9e-2
+    check_attention(near, one, "near")
     bad = one.copy()
-    bad[2, 3] += 1.5e-2
+    bad[2, 3] += 2.1e-2
     with pytest.raises(AssertionError, match="diff"):
         check_attention(bad, one, "planted")
     bad = ref.copy()
