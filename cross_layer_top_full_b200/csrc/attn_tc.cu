@@ -14,15 +14,18 @@
 // every selected row (value columns 256r..256r+255 and rope columns
 // 512+32r..512+32r+31), computes the partial logits S_r = Q_r K_r^T on the
 // tensor core, scales them to base-2 units and sends them to its partner
-// through distributed shared memory: per head, the block's largest valid
-// partial logit m as float16 and every partial logit's difference from m as
-// float16.  Near the row maximum, where the softmax weights are decided, the
-// differences are small, so the float16 rounding (2^-11 of the difference)
-// stays far inside the attention tolerance even for sharp logits of tens of
-// base-2 units.  Each CTA adds its own half in float32, straight from TMEM,
-// to the partner's reconstructed half and runs the online softmax; each then
-// accumulates its own 256 value columns, O_r += P V_r, in TMEM, normalised by
-// its own softmax sum.  No key byte is gathered twice and no flop is done
+// through distributed shared memory as 16-bit fixed point: per head and
+// block, an offset m at or above the largest valid partial logit and a
+// power-of-two step fitted to the block's range, each value sent as
+// (m - x) / step.  A key can decide the softmax while its partial logit on
+// one CTA lies far below that CTA's block maximum (the other half makes up
+// for it), so the rounding must not grow with the distance from m as a
+// float16 difference's does: here it is at most one step, range / 2^15, for
+// every key, which keeps sharp logits of a hundred and more base-2 units
+// inside the attention tolerance.  Each CTA adds its own half in float32,
+// straight from TMEM, to the partner's rebuilt half; each then runs the
+// online softmax and accumulates its own 256 value columns, O_r += P V_r, in
+// TMEM, normalised by its own softmax sum.  No key byte is gathered twice and no flop is done
 // twice.
 //
 // Per CTA (448 threads), persistent over work units (one unit = one query
@@ -36,13 +39,14 @@
 //   warps 4-7  exchange (thread = head = TMEM lane): at the start of a unit,
 //              the unit's Q_r columns that the S MMA reads from TMEM (value
 //              slice 3 and the 32 rope columns); per 64-key block, partial S
-//              from TMEM -> base 2 -> (block maximum, float16 differences),
+//              from TMEM -> base 2 -> (offset, step, 16-bit codes),
 //              sent straight into the partner's inbox with st.async (counted
-//              in bytes on the partner's mbarrier); they run ahead of the
-//              softmax warps, so the exchange latency of block j+1 hides
-//              behind the softmax of block j;
-//   warps 8-11 softmax (thread = head): own (float32) + partner logits, row max,
-//              online softmax in base 2 with lazy rescaling (O is rescaled
+//              in bytes on the partner's mbarrier); software-pipelined by one
+//              block, they then rebuild block j-1's full logits (own float32
+//              half + the partner's) and its maximum into TMEM, so the
+//              exchange latency hides behind the next block's work;
+//   warps 8-11 softmax (thread = head): from the full logits and the block
+//              maximum, online softmax in base 2 with lazy rescaling (O is rescaled
 //              only when the running max grows by more than 2^8), P as bf16
 //              into TMEM over the S columns, the row sum l of the same
 //              rounded P, final normalisation and store;
@@ -57,8 +61,9 @@
 // TMEM: O at columns 0..255, three S/P buffers at 256..447, Q_r slice 3 and
 // rope columns at 448..495.  Keeping that part of Q_r in TMEM frees the
 // shared memory for a fourth KV stage.
-// Shared memory: Q_r slices 0-2 48 KB, 4 KV stages of 36 KB, 2 float16 inbox
-// tiles of 16 KB + 256 B of per-head offsets (written by the partner),
+// Shared memory: Q_r slices 0-2 48 KB, 4 KV stages of 36 KB, 2 inbox tiles of
+// 16-bit fixed-point logits (16 KB) + 512 B of per-head offset/step words
+// (written by the partner),
 // per-unit masks, barriers (~227 KB).
 //
 // Every wait is bounded (sm100.cuh); a wait that runs out records its site
@@ -93,17 +98,17 @@ constexpr int KV_ROPE = NB * 64;     // the 32 rope columns of a key block
 constexpr int KV_STAGE = 4 * KV_ATOM + KV_ROPE;     // 36 KB
 constexpr int NSTAGE = 4;
 constexpr int NSBUF = 3;                            // S/P buffers in TMEM
-constexpr int X_TILE = HQ * NB * 2;                 // 16 KB of float16 logit differences
+constexpr int X_TILE = HQ * NB * 2;                 // 16 KB of 16-bit fixed-point partial logits
 constexpr int X_QUAD = X_TILE / 4;                  // the 32 rows of one TMEM lane quadrant
-constexpr int X_OFF = HQ * 2;                       // per-head float16 offsets of one inbox slot
+constexpr int X_OFF = HQ * 4;                       // per-head offset/step words of one inbox slot
 constexpr int X_OFF_QUAD = X_OFF / 4;
 constexpr int MAX_UNIT_BLOCKS = 32;                 // at most 2048 indices per unit
 constexpr int Q_SMEM_ATOMS = 3;                     // value slices 0-2 of Q_r in shared memory;
                                                     // slice 3 and the rope columns live in TMEM
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = Q_SMEM_ATOMS * Q_ATOM;       // 48 KB
-constexpr int OFF_X = OFF_KV + NSTAGE * KV_STAGE;   // partner's float16 logit differences
-constexpr int OFF_XOFF = OFF_X + 2 * X_TILE;        // partner's float16 per-head offsets
+constexpr int OFF_X = OFF_KV + NSTAGE * KV_STAGE;   // partner's fixed-point partial logits
+constexpr int OFF_XOFF = OFF_X + 2 * X_TILE;        // partner's per-head offset/step words
 constexpr int OFF_MASK = OFF_XOFF + 2 * X_OFF;
 constexpr int OFF_BARS = OFF_MASK + 2 * MAX_UNIT_BLOCKS * 8;
 constexpr int GW = 4;                               // gather warps
@@ -140,7 +145,9 @@ struct __align__(8) AttnBars {
     int red[2][4];
 };
 
-constexpr size_t SMEM_BYTES = 1024 + OFF_BARS + sizeof(AttnBars);
+// the dynamic shared memory base is at least 16-byte aligned, so rounding it
+// up to the 1024-byte alignment of the swizzled tiles takes at most 1008 bytes
+constexpr size_t SMEM_BYTES = 1008 + OFF_BARS + sizeof(AttnBars);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 __device__ __forceinline__ bool idx_valid(int v, int t, int T) { return v >= 0 && v <= t && v < T; }
@@ -150,29 +157,80 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-// float16 pair {lo = a, hi = b}, saturated to the finite float16 range
-__device__ __forceinline__ uint32_t half2_sat(float a, float b) {
-    uint32_t r;
-    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
-    return r;
-}
-
-// a (float16, exact in float32) + c, one float32 rounding
-__device__ __forceinline__ float add_f16_f32(unsigned short a, float c) {
-    float d;
-    asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(a), "f"(c));
-    return d;
-}
-
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
 
-// float16 -> float32 of the low / high half of a packed pair
-__device__ __forceinline__ float f16_lo(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v & 0xffffu))); }
-__device__ __forceinline__ float f16_hi(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
+__device__ __forceinline__ float min3(float a, float b, float c) {
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// The partner's half of a key block crosses as 16-bit fixed point, per head:
+// x ~ m - u * step with u an unsigned 16-bit integer, m at or above the
+// block's largest valid partial logit (a bfloat16, rounded up) and step the
+// power of two that spreads the block's range over [0, 2^16).  So every valid
+// value is rebuilt to within one step, which shrinks with the block's range,
+// not with the logit's magnitude as a float16 difference would.  Invalid keys
+// (-inf) encode as 65535; they are -inf on the receiving side already.
+struct XCode {
+    float scale, ms;    // 1/step and m/step (both exact)
+    uint32_t word;      // bfloat16 m in bits 0-15, the float32 exponent field of step in 16-23
+};
+
+__device__ __forceinline__ XCode x_encoder(float mb, float mn) {
+    uint32_t mbits = __float_as_uint(mb);
+    mbits = (mbits >> 31) ? (mbits & 0xffff0000u) : ((mbits + 0xffffu) & 0xffff0000u);
+    const float m = __uint_as_float(mbits);
+    const float range = m - mn;
+    int k = 0;                                      // step = 2^-k
+    if (range > 0.f && range < INFINITY)            // range in [2^e, 2^(e+1)): k = 15 - e
+        k = min(30, max(-30, 142 - (int)((__float_as_uint(range) >> 23) & 0xffu)));
+    XCode c;
+    c.scale = __uint_as_float((uint32_t)(127 + k) << 23);
+    c.ms = m * c.scale;
+    c.word = (mbits >> 16) | ((uint32_t)(127 - k) << 16);
+    return c;
+}
+
+// two values {lo = a, hi = b} as 16-bit codes (m - x) / step, rounded, at most 65535
+__device__ __forceinline__ uint32_t x_encode2(const XCode& c, float a, float b) {
+    const float ua = fminf(fmaf(a, -c.scale, c.ms), 65535.f) + 8388608.f;   // 2^23 + u
+    const float ub = fminf(fmaf(b, -c.scale, c.ms), 65535.f) + 8388608.f;
+    return __byte_perm(__float_as_uint(ua), __float_as_uint(ub), 0x5410);
+}
+
+// the value of the low / high code of a packed pair under offset m and step
+__device__ __forceinline__ float x_decode_lo(uint32_t w, float m, float step) {
+    return fmaf(-(__uint_as_float((w & 0xffffu) | 0x4b000000u) - 8388608.f), step, m);
+}
+__device__ __forceinline__ float x_decode_hi(uint32_t w, float m, float step) {
+    return fmaf(-(__uint_as_float(__byte_perm(w, 0x4b000000u, 0x7632)) - 8388608.f), step, m);
+}
+
+// This thread's (head's) own partial logits of a 64-key S buffer in base-2
+// units, the keys of invalid indices (mask bits 0) set to -inf.
+__device__ __forceinline__ void own_logits(uint32_t taddr, float sl2, const uint32_t* mask2,
+                                           float (&x)[NB]) {
+    uint32_t r0[32], r1[32];
+    tmem_ld32(taddr, r0);
+    tmem_ld32(taddr + 32, r1);
+    const uint32_t m_lo = mask2[0], m_hi = mask2[1];
+    tmem_ld_wait();
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        x[c] = __uint_as_float(r0[c]) * sl2;
+        x[32 + c] = __uint_as_float(r1[c]) * sl2;
+    }
+    if ((m_lo & m_hi) != 0xffffffffu) {
+#pragma unroll
+        for (int c = 0; c < NB; ++c)
+            if (!(((c < 32 ? m_lo : m_hi) >> (c & 31)) & 1u)) x[c] = -INFINITY;
+    }
+}
 
 // largest of 64 values
 __device__ __forceinline__ float max64(const float (&v)[NB]) {
@@ -183,6 +241,25 @@ __device__ __forceinline__ float max64(const float (&v)[NB]) {
 #pragma unroll
     for (int x = 2; x + 1 < 21; x += 2) m = max3(m, mx[x], mx[x + 1]);
     return fmaxf(m, mx[20]);
+}
+
+// smallest of 64 values
+__device__ __forceinline__ float min64(const float (&v)[NB]) {
+    float mn[21];
+#pragma unroll
+    for (int x = 0; x < 21; ++x) mn[x] = min3(v[3 * x], v[3 * x + 1], v[3 * x + 2]);
+    float m = min3(mn[0], mn[1], v[63]);
+#pragma unroll
+    for (int x = 2; x + 1 < 21; x += 2) m = min3(m, mn[x], mn[x + 1]);
+    return fminf(m, mn[20]);
+}
+
+// smallest of the values above -inf (+inf if there is none)
+__device__ __forceinline__ float min64_finite(const float (&v)[NB]) {
+    float m = INFINITY;
+#pragma unroll
+    for (int c = 0; c < NB; ++c) m = fminf(m, v[c] > -INFINITY ? v[c] : INFINITY);
+    return m;
 }
 
 struct AttnArgs {
@@ -408,7 +485,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         const int h = quad * 32 + lane;           // head of this thread
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t x_remote = map_to_rank(smem_base + OFF_X + h * 128, peer);
-        const uint32_t xoff_remote = map_to_rank(smem_base + OFF_XOFF + (h >> 1) * 4, peer);
+        const uint32_t xoff_remote = map_to_rank(smem_base + OFF_XOFF + h * 4, peer);
         const uint32_t free_remote0 = map_to_rank(smem_u32(&bars->peer_free[0][quad]), peer);
         const uint32_t free_remote1 = map_to_rank(smem_u32(&bars->peer_free[1][quad]), peer);
         const float sl2 = args.scale_log2;
@@ -444,106 +521,101 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->q_tmem_full);
             }
-            for (int j = 0; j < nb; ++j, ++g) {
-                const int sb = g % NSBUF;
-                const int slot = g & 1;
-                // arm this CTA's inbox slot for the partner's half of block g
-                if (lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD + X_OFF_QUAD);
-                if (!warp_wait(&bars->s_full[sb], (g / NSBUF) & 1, status, abort, 5)) { ok = false; break; }
-                tc_fence_after();
-                float x[NB];
-                {
-                    uint32_t r0[32], r1[32];
-                    tmem_ld32(t_lane + TM_S + 64 * sb, r0);
-                    tmem_ld32(t_lane + TM_S + 64 * sb + 32, r1);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        x[c] = __uint_as_float(r0[c]) * sl2;
-                        x[32 + c] = __uint_as_float(r1[c]) * sl2;
+            // Software-pipelined by one block: iteration j sends block j of the
+            // unit, then finishes block j-1 (whose partner half has had the time
+            // of the send to arrive), so the exchange latency overlaps the next
+            // block's work.  S(j-1) is still intact in TMEM when it is finished:
+            // only the full logits of block j-1 overwrite it, and the next S MMA
+            // into its buffer waits for the P V of block j-1.
+            for (int j = 0; j <= nb; ++j) {
+                if (j < nb) {
+                    const uint32_t gs = g + j;
+                    const int sb = gs % NSBUF;
+                    const int slot = gs & 1;
+                    // arm this CTA's inbox slot for the partner's half of block gs
+                    if (lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD + X_OFF_QUAD);
+                    if (!warp_wait(&bars->s_full[sb], (gs / NSBUF) & 1, status, abort, 5)) { ok = false; break; }
+                    tc_fence_after();
+                    float x[NB];
+                    own_logits(t_lane + TM_S + 64 * sb, sl2, masks + ip * 2 * MAX_UNIT_BLOCKS + 2 * j, x);
+                    // the encoding's offset and step come from the block's largest and
+                    // smallest VALID partial logits (invalid keys are -inf from here on)
+                    const float mb = max64(x);
+                    float mn = min64(x);
+                    if (mn == -INFINITY) mn = min64_finite(x);      // a block with invalid keys
+                    const XCode xc = x_encoder(mb, mn);
+                    // the partner's exchange warp q must have finished this inbox slot
+                    // (block gs-2)
+                    if (!warp_wait_cluster(&bars->peer_free[slot][quad], ((gs >> 1) & 1) ^ 1, status, abort, 6)) {
+                        ok = false;
+                        break;
                     }
-                }
-                // the offset is the largest VALID partial logit of the block (keys
-                // of invalid indices are zero rows whose logits would pull it off);
-                // invalid keys become -inf from here on
-                const uint32_t m_lo = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j];
-                const uint32_t m_hi = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j + 1];
-                const bool holes = (m_lo & m_hi) != 0xffffffffu;
-                if (holes) {
-#pragma unroll
-                    for (int c = 0; c < NB; ++c)
-                        if (!(((c < 32 ? m_lo : m_hi) >> (c & 31)) & 1u)) x[c] = -INFINITY;
-                }
-                const float mb = max64(x);
-                // offset as float16 (saturated); the differences are taken from
-                // the rounded offset, so offset + difference rebuilds the value
-                const uint32_t m16 = half2_sat(mb, 0.f) & 0xffffu;
-                const float mf = f16_lo(m16);
-                // two heads' offsets per 32-bit word: lane 2i sends heads 2i, 2i+1
-                const uint32_t m16_odd = __shfl_down_sync(0xffffffffu, m16, 1);
-                // the partner's exchange warp q must have read this inbox slot (block g-2)
-                if (!warp_wait_cluster(&bars->peer_free[slot][quad], ((g >> 1) & 1) ^ 1, status, abort, 6)) {
-                    ok = false;
-                    break;
-                }
-                {
-                    // row h of the partner's inbox, 16 bytes (8 keys) at a time; each
-                    // st.async counts its bytes on the partner's x_full (no fence or
-                    // arrive on this side)
+                    // row h of the partner's inbox, 16 bytes (8 keys) at a time, and
+                    // the head's offset/step word; each st.async counts its bytes on the
+                    // partner's x_full (no fence or arrive on this side)
                     const uint32_t xr = x_remote + slot * X_TILE;
                     const uint32_t br = map_to_rank(smem_u32(&bars->x_full[slot][quad]), peer);
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
                         st_async_v4(xr + ((c ^ (h & 7)) << 4),
-                                    half2_sat(x[8 * c + 0] - mf, x[8 * c + 1] - mf),
-                                    half2_sat(x[8 * c + 2] - mf, x[8 * c + 3] - mf),
-                                    half2_sat(x[8 * c + 4] - mf, x[8 * c + 5] - mf),
-                                    half2_sat(x[8 * c + 6] - mf, x[8 * c + 7] - mf), br);
-                    if ((lane & 1) == 0)
-                        st_async_b32(xoff_remote + slot * X_OFF, m16 | (m16_odd << 16), br);
+                                    x_encode2(xc, x[8 * c + 0], x[8 * c + 1]),
+                                    x_encode2(xc, x[8 * c + 2], x[8 * c + 3]),
+                                    x_encode2(xc, x[8 * c + 4], x[8 * c + 5]),
+                                    x_encode2(xc, x[8 * c + 6], x[8 * c + 7]), br);
+                    st_async_b32(xoff_remote + slot * X_OFF, xc.word, br);
                 }
-                // the partner's half of block g: full logits = own (float32) +
-                // the partner's offset + float16 difference
-                if (!warp_wait_cluster(&bars->x_full[slot][quad], (g >> 1) & 1, status, abort, 9)) {
-                    ok = false;
-                    break;
-                }
-                {
-                    const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + slot * X_TILE + h * 128);
-                    const uint32_t ow = reinterpret_cast<const uint32_t*>(smem + OFF_XOFF + slot * X_OFF)[h >> 1];
-                    const float pf = (h & 1) ? f16_hi(ow) : f16_lo(ow);
+                if (j >= 1) {
+                    const uint32_t gf = g + j - 1;
+                    const int sb = gf % NSBUF;
+                    const int slot = gf & 1;
+                    // the partner's half of block gf
+                    if (!warp_wait_cluster(&bars->x_full[slot][quad], (gf >> 1) & 1, status, abort, 9)) {
+                        ok = false;
+                        break;
+                    }
+                    // full logits = own half (float32, read again from TMEM) + the
+                    // partner's half rebuilt from its fixed-point codes
+                    float x[NB];
+                    own_logits(t_lane + TM_S + 64 * sb, sl2, masks + ip * 2 * MAX_UNIT_BLOCKS + 2 * (j - 1), x);
+                    {
+                        const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + slot * X_TILE + h * 128);
+                        const uint32_t ow = reinterpret_cast<const uint32_t*>(smem + OFF_XOFF + slot * X_OFF)[h];
+                        const float pm = __uint_as_float(ow << 16);
+                        const float pstep = __uint_as_float(((ow >> 16) & 0xffu) << 23);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 w4 = xp[c ^ (h & 7)];
-                        const uint32_t pw4[4] = {w4.x, w4.y, w4.z, w4.w};
+                        for (int c = 0; c < 8; ++c) {
+                            const uint4 w4 = xp[c ^ (h & 7)];
+                            const uint32_t pw4[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            x[8 * c + 2 * e] += add_f16_f32((unsigned short)(pw4[e] & 0xffffu), pf);
-                            x[8 * c + 2 * e + 1] += add_f16_f32((unsigned short)(pw4[e] >> 16), pf);
+                            for (int e = 0; e < 4; ++e) {
+                                x[8 * c + 2 * e] += x_decode_lo(pw4[e], pm, pstep);
+                                x[8 * c + 2 * e + 1] += x_decode_hi(pw4[e], pm, pstep);
+                            }
                         }
                     }
-                }
-                // every inbox value of this slot has been read: hand it back
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote_relaxed(slot ? free_remote1 : free_remote0);
-                const float mloc = max64(x);
-                // full logits over S, their maximum in its column: the softmax warp's input
-                {
-                    uint32_t w0[32], w1[32];
+                    // every inbox value of this slot has been read: hand it back
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote_relaxed(slot ? free_remote1 : free_remote0);
+                    const float mloc = max64(x);
+                    // full logits over S, their maximum in its column: the softmax warp's input
+                    {
+                        uint32_t w0[32], w1[32];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        w0[c] = __float_as_uint(x[c]);
-                        w1[c] = __float_as_uint(x[32 + c]);
+                        for (int c = 0; c < 32; ++c) {
+                            w0[c] = __float_as_uint(x[c]);
+                            w1[c] = __float_as_uint(x[32 + c]);
+                        }
+                        tmem_st32(t_lane + TM_S + 64 * sb, w0);
+                        tmem_st32(t_lane + TM_S + 64 * sb + 32, w1);
+                        tmem_st1(t_lane + TM_MX + sb, __float_as_uint(mloc));
                     }
-                    tmem_st32(t_lane + TM_S + 64 * sb, w0);
-                    tmem_st32(t_lane + TM_S + 64 * sb + 32, w1);
-                    tmem_st1(t_lane + TM_MX + sb, __float_as_uint(mloc));
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
                 }
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
             }
+            g += nb;
             // the unit's masks have been read: the gather warps may refill them
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->info_empty[ip]);
