@@ -11,14 +11,13 @@
   position scores at least tau - 1e-3|tau|; no duplicates, all in [0, t],
   ascending, -1 padded, exactly min(k, t+1) kept.
 * attention: "within 1e-2 max abs and 1e-2 relative" read elementwise as
-  |gpu - oracle| <= 1e-2 + 1e-2 |oracle| (numpy's isclose / torch's
-  allclose form of an absolute and a relative tolerance), plus the
-  aggregate ||gpu - oracle||_2 <= 1e-2 ||oracle||_2.  A pure 1e-2 absolute
+  |gpu - oracle| <= max(1e-2, 1e-2 |oracle|): 1e-2 absolute, relaxed to 1e-2
+  relative only where the output is larger than 1 (a pure 1e-2 absolute
   bound cannot hold for bf16 outputs of magnitude >= 2, whose rounding step
-  alone is 2^-7 or more.  The stricter max(1e-2, 1e-2 |oracle|) cannot hold
-  for bf16-P attention at sharp logits either: the bf16 rounding of the
-  softmax weights (the P.V operand) and of the output leave errors of
-  about 1e-2 on outputs near 1 there (q x8: 0.0102 at an output of -1.005).
+  alone is 2^-7 or more), plus the aggregate
+  ||gpu - oracle||_2 <= 1e-2 ||oracle||_2.  The bf16 rounding of the softmax
+  weights (the P.V operand) and of the output stays about 4e-3 inside it
+  even at sharp logits (base-2 logits of 100 and more).
 """
 import numpy as np
 import torch
@@ -97,8 +96,8 @@ def check_topk_band(idx: np.ndarray, ref_scores: np.ndarray, q_start: int, k: in
 
 
 def attn_bound(ref: np.ndarray) -> np.ndarray:
-    """Elementwise attention bound 1e-2 + 1e-2 |ref|."""
-    return ATTN_ATOL + ATTN_RTOL * np.abs(ref)
+    """Elementwise attention bound max(1e-2, 1e-2 |ref|)."""
+    return np.maximum(ATTN_ATOL, ATTN_RTOL * np.abs(ref))
 
 
 def check_attention(gpu: np.ndarray, ref: np.ndarray, what: str = "") -> None:
@@ -111,6 +110,6 @@ def check_attention(gpu: np.ndarray, ref: np.ndarray, what: str = "") -> None:
     rel = float(np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-30))
     if worst > 0:
         at = np.unravel_index(int(np.argmax(excess)), d.shape)
-        raise AssertionError("%s |diff| %g > %g + %g*|ref| at %s (ref %g)"
+        raise AssertionError("%s |diff| %g > max(%g, %g*|ref|) at %s (ref %g)"
                              % (what, d[at], ATTN_ATOL, ATTN_RTOL, at, ref[at]))
     assert rel <= ATTN_REL_L2, "%s rel L2 = %g" % (what, rel)

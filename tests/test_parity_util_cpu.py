@@ -68,16 +68,18 @@ def test_check_attention():
     bad[1, 2, 3, 4] += 2 * attn_bound(ref[1, 2, 3, 4])
     with pytest.raises(AssertionError, match="diff"):
         check_attention(bad, ref, "planted")
-    # the bound is the sum of the two terms: on an output of 1.0 an error of
-    # 1.9e-2 passes elementwise and 2.1e-2 fails
-    one = np.ones((40, 80))
-    near = one.copy()
-    near[2, 3] += 1.9e-2
-    check_attention(near, one, "near")
-    bad = one.copy()
-    bad[2, 3] += 2.1e-2
-    with pytest.raises(AssertionError, match="diff"):
-        check_attention(bad, one, "planted")
+    # the bound is the larger of the two terms, not their sum: on an output of
+    # 0.5 an error of 0.9e-2 passes and 1.1e-2 fails; on an output of 4.0,
+    # 3.9e-2 passes and 4.1e-2 fails
+    for v, ok_err, bad_err in ((0.5, 0.9e-2, 1.1e-2), (4.0, 3.9e-2, 4.1e-2)):
+        base = np.full((40, 80), v)
+        near = base.copy()
+        near[2, 3] += ok_err
+        check_attention(near, base, "near")
+        bad = base.copy()
+        bad[2, 3] += bad_err
+        with pytest.raises(AssertionError, match="diff"):
+            check_attention(bad, base, "planted")
     bad = ref.copy()
     bad[0, 0, 0, 0] = np.nan
     with pytest.raises(AssertionError, match="non-finite"):
