@@ -101,12 +101,18 @@ bool paged_ok(const ic_paged_rows* pr, bool need_pages) {
 }
 
 // Planning rows of a paged batch: every sequence as long as T_max.
+// Every score row starts on a 16-byte boundary (the cluster and multi-CTA
+// top-k kernels read rows as 16-byte vectors).
+bool rows_16b_aligned(const float* scores, int64_t ld) {
+    return ((uintptr_t)scores & 15) == 0 && (ld & 3) == 0;
+}
+
 ic_rows plan_rows(const ic_paged_rows* pr) { return ic_rows{pr->B, pr->Lq, pr->T_max - pr->Lq, pr->T_max}; }
 
 ic_status run_topk_varlen(const float* scores, int64_t ld, const ic_paged_rows* pr, int k,
                           int32_t* idx, cudaStream_t s) {
     const ic_rows r = plan_rows(pr);
-    if (topk_cluster_applies(r, k) && ((uintptr_t)scores & 15) == 0)
+    if (topk_cluster_applies(r, k) && rows_16b_aligned(scores, ld))
         return launch_topk_cluster(scores, ld, r, k, idx, s, pr->seq_lens);
     return launch_topk_rows(scores, ld, r, k, idx, s, pr->seq_lens);
 }
@@ -131,9 +137,9 @@ ic_status run_topk(const float* scores, int64_t ld, ic_rows r, int k, int32_t* i
     // the cluster and multi-CTA paths read 16-byte vectors: they need 16-byte
     // aligned rows.  Few long rows (decode): one cluster per row, one launch;
     // rows too long for the cluster's shared memory: three launches.
-    if (topk_cluster_applies(r, k) && ((uintptr_t)scores & 15) == 0)
+    if (topk_cluster_applies(r, k) && rows_16b_aligned(scores, ld))
         return launch_topk_cluster(scores, ld, r, k, idx, s);
-    if (topk_multi_applies(r, k) && scratch != nullptr && ((uintptr_t)scores & 15) == 0 &&
+    if (topk_multi_applies(r, k) && scratch != nullptr && rows_16b_aligned(scores, ld) &&
         scratch_bytes >= topk_multi_scratch_bytes(r, k))
         return launch_topk_multi(scores, ld, r, k, idx, scratch, s);
     return launch_topk_rows(scores, ld, r, k, idx, s);

@@ -68,9 +68,14 @@ __device__ __forceinline__ uint32_t map_rank(const void* p, uint32_t rank) {
     return r;
 }
 
+// Cluster-wide barrier of all threads.  A CTA barrier first brings every
+// warp of the CTA to this point converged; the cluster barrier itself is the
+// non-.aligned form, whose arrive and wait each thread may execute on its
+// own, so its correctness does not rest on how the compiler reconverges a
+// warp after divergent code.
 __device__ __forceinline__ void cluster_barrier() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                     : "memory");
+    __syncthreads();
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
 
 // One warp: among the `m` counts c[0..m-1] (index 0 = the LOWEST bin of the
