@@ -41,10 +41,10 @@
 //              slice 3 and the 32 rope columns); per 64-key block, partial S
 //              from TMEM -> base 2 -> (offset, step, 16-bit codes),
 //              sent straight into the partner's inbox with st.async (counted
-//              in bytes on the partner's mbarrier); software-pipelined by one
-//              block, they then rebuild block j-1's full logits (own float32
-//              half + the partner's) and its maximum into TMEM, so the
-//              exchange latency hides behind the next block's work;
+//              in bytes on the partner's mbarrier); once the partner's half
+//              is in, they rebuild the block's full logits (own float32 half,
+//              still in registers, + the partner's) and their maximum into
+//              TMEM;
 //   warps 8-11 softmax (thread = head): from the full logits and the block
 //              maximum, online softmax in base 2 with lazy rescaling (O is rescaled
 //              only when the running max grows by more than 2^8), P as bf16
@@ -521,23 +521,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->q_tmem_full);
             }
-            // Software-pipelined by one block: iteration j sends block j of the
-            // unit, then finishes block j-1 (whose partner half has had the time
-            // of the send to arrive), so the exchange latency overlaps the next
-            // block's work.  S(j-1) is still intact in TMEM when it is finished:
-            // only the full logits of block j-1 overwrite it, and the next S MMA
-            // into its buffer waits for the P V of block j-1.
-            for (int j = 0; j <= nb; ++j) {
-                if (j < nb) {
-                    const uint32_t gs = g + j;
-                    const int sb = gs % NSBUF;
-                    const int slot = gs & 1;
-                    // arm this CTA's inbox slot for the partner's half of block gs
-                    if (lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD + X_OFF_QUAD);
-                    if (!warp_wait(&bars->s_full[sb], (gs / NSBUF) & 1, status, abort, 5)) { ok = false; break; }
-                    tc_fence_after();
-                    float x[NB];
-                    own_logits(t_lane + TM_S + 64 * sb, sl2, masks + ip * 2 * MAX_UNIT_BLOCKS + 2 * j, x);
+            // Per block: send this CTA's half, then finish the block as soon as
+            // the partner's half is in.  (Finishing block j only after sending
+            // block j+1 would tie it to S(j+1), whose buffer waits for P V of
+            // block j-2: a two-block cycle instead of a three-block one.)
+            for (int j = 0; j < nb; ++j) {
+                const uint32_t gs = g + j;
+                const int sb = gs % NSBUF;
+                const int slot = gs & 1;
+                // arm this CTA's inbox slot for the partner's half of block gs
+                if (lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD + X_OFF_QUAD);
+                if (!warp_wait(&bars->s_full[sb], (gs / NSBUF) & 1, status, abort, 5)) { ok = false; break; }
+                tc_fence_after();
+                float x[NB];
+                own_logits(t_lane + TM_S + 64 * sb, sl2, masks + ip * 2 * MAX_UNIT_BLOCKS + 2 * j, x);
+                {
                     // the encoding's offset and step come from the block's largest and
                     // smallest VALID partial logits (invalid keys are -inf from here on)
                     const float mb = max64(x);
@@ -564,56 +562,49 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                                     x_encode2(xc, x[8 * c + 6], x[8 * c + 7]), br);
                     st_async_b32(xoff_remote + slot * X_OFF, xc.word, br);
                 }
-                if (j >= 1) {
-                    const uint32_t gf = g + j - 1;
-                    const int sb = gf % NSBUF;
-                    const int slot = gf & 1;
-                    // the partner's half of block gf
-                    if (!warp_wait_cluster(&bars->x_full[slot][quad], (gf >> 1) & 1, status, abort, 9)) {
-                        ok = false;
-                        break;
-                    }
-                    // full logits = own half (float32, read again from TMEM) + the
-                    // partner's half rebuilt from its fixed-point codes
-                    float x[NB];
-                    own_logits(t_lane + TM_S + 64 * sb, sl2, masks + ip * 2 * MAX_UNIT_BLOCKS + 2 * (j - 1), x);
-                    {
-                        const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + slot * X_TILE + h * 128);
-                        const uint32_t ow = reinterpret_cast<const uint32_t*>(smem + OFF_XOFF + slot * X_OFF)[h];
-                        const float pm = __uint_as_float(ow << 16);
-                        const float pstep = __uint_as_float(((ow >> 16) & 0xffu) << 23);
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const uint4 w4 = xp[c ^ (h & 7)];
-                            const uint32_t pw4[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                x[8 * c + 2 * e] += x_decode_lo(pw4[e], pm, pstep);
-                                x[8 * c + 2 * e + 1] += x_decode_hi(pw4[e], pm, pstep);
-                            }
-                        }
-                    }
-                    // every inbox value of this slot has been read: hand it back
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_remote_relaxed(slot ? free_remote1 : free_remote0);
-                    const float mloc = max64(x);
-                    // full logits over S, their maximum in its column: the softmax warp's input
-                    {
-                        uint32_t w0[32], w1[32];
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            w0[c] = __float_as_uint(x[c]);
-                            w1[c] = __float_as_uint(x[32 + c]);
-                        }
-                        tmem_st32(t_lane + TM_S + 64 * sb, w0);
-                        tmem_st32(t_lane + TM_S + 64 * sb + 32, w1);
-                        tmem_st1(t_lane + TM_MX + sb, __float_as_uint(mloc));
-                    }
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
+                // the partner's half of block gs
+                if (!warp_wait_cluster(&bars->x_full[slot][quad], (gs >> 1) & 1, status, abort, 9)) {
+                    ok = false;
+                    break;
                 }
+                // full logits = own half (float32, still in registers) + the
+                // partner's half rebuilt from its fixed-point codes
+                {
+                    const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + slot * X_TILE + h * 128);
+                    const uint32_t ow = reinterpret_cast<const uint32_t*>(smem + OFF_XOFF + slot * X_OFF)[h];
+                    const float pm = __uint_as_float(ow << 16);
+                    const float pstep = __uint_as_float(((ow >> 16) & 0xffu) << 23);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 w4 = xp[c ^ (h & 7)];
+                        const uint32_t pw4[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            x[8 * c + 2 * e] += x_decode_lo(pw4[e], pm, pstep);
+                            x[8 * c + 2 * e + 1] += x_decode_hi(pw4[e], pm, pstep);
+                        }
+                    }
+                }
+                // every inbox value of this slot has been read: hand it back
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote_relaxed(slot ? free_remote1 : free_remote0);
+                const float mloc = max64(x);
+                // full logits over S, their maximum in its column: the softmax warp's input
+                {
+                    uint32_t w0[32], w1[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        w0[c] = __float_as_uint(x[c]);
+                        w1[c] = __float_as_uint(x[32 + c]);
+                    }
+                    tmem_st32(t_lane + TM_S + 64 * sb, w0);
+                    tmem_st32(t_lane + TM_S + 64 * sb + 32, w1);
+                    tmem_st1(t_lane + TM_MX + sb, __float_as_uint(mloc));
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
             }
             g += nb;
             // the unit's masks have been read: the gather warps may refill them

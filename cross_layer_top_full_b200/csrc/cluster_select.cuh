@@ -183,10 +183,12 @@ __device__ void cluster_select(ClusterSmem<NT / 32>& S, const uint32_t* keys, in
             {
                 uint32_t tot = lane < (int)CL ? ld_dsmem(map_rank(&S.slice_tot, (uint32_t)lane)) : 0u;
                 // top-down: slice CL-1 holds the highest bins
-                uint32_t mine = 0;
                 const int pos = lane;                       // top-down position
                 const int sl = (int)CL - 1 - pos;
-                mine = (pos < (int)CL) ? __shfl_sync(0xffffffffu, tot, sl < 0 ? 0 : sl) : 0u;
+                // every lane takes part in the shuffle (a full-mask shuffle that
+                // some lanes skip never completes); lanes past CL then drop it
+                const uint32_t from_sl = __shfl_sync(0xffffffffu, tot, sl < 0 ? 0 : sl);
+                const uint32_t mine = pos < (int)CL ? from_sl : 0u;
                 uint32_t incl = mine;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
