@@ -41,12 +41,11 @@
 //              slice 3 and the 32 rope columns); per 64-key block, partial S
 //              from TMEM -> base 2 -> (offset, step, 16-bit codes),
 //              sent straight into the partner's inbox with st.async (counted
-//              in bytes on the partner's mbarrier); once the partner's half
-//              is in, they rebuild the block's full logits (own float32 half,
-//              still in registers, + the partner's) and their maximum into
-//              TMEM;
-//   warps 8-11 softmax (thread = head): from the full logits and the block
-//              maximum, online softmax in base 2 with lazy rescaling (O is rescaled
+//              in bytes on the partner's mbarrier); they run ahead of the
+//              softmax warps by up to the two inbox slots;
+//   warps 8-11 softmax (thread = head): own half (float32, from TMEM) + the
+//              partner's rebuilt half, row max, online softmax in base 2 with
+//              lazy rescaling (O is rescaled
 //              only when the running max grows by more than 2^8), P as bf16
 //              into TMEM over the S columns, the row sum l of the same
 //              rounded P, final normalisation and store;
@@ -121,16 +120,15 @@ constexpr int TMEM_COLS = 512;
 constexpr uint32_t TM_O = 0;
 constexpr uint32_t TM_S = 256;                      // S/P buffer b at TM_S + 64 b
 constexpr uint32_t TM_QT = TM_S + 64 * NSBUF;       // Q_r slice 3 (32 cols) + rope (16 cols), bf16 pairs
-constexpr uint32_t TM_MX = TM_QT + 48;              // block maximum of the full logits, per S buffer
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_THRESHOLD = 8.f;            // log2 units
-static_assert(TM_MX + NSBUF <= TMEM_COLS, "tensor memory budget");
+static_assert(TM_QT + 48 <= TMEM_COLS, "tensor memory budget");
 
 struct __align__(8) AttnBars {
     uint64_t q_full, q_empty, q_tmem_full;
     uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
     uint64_t s_full[NSBUF], s_free[NSBUF];
-    uint64_t own_full[NSBUF][4];    // exchange warp q: the buffer holds the full logits and their max
+    uint64_t own_full[NSBUF][4];    // exchange warp q has read S of the buffer
     uint64_t p_full[NSBUF];         // softmax warps -> MMA: P in TMEM
     uint64_t x_full[2][4];          // [inbox slot][quad]: the partner's 32 rows (counted in bytes)
     uint64_t peer_free[2][4];       // the partner's softmax warp q has read its inbox slot
@@ -486,8 +484,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t x_remote = map_to_rank(smem_base + OFF_X + h * 128, peer);
         const uint32_t xoff_remote = map_to_rank(smem_base + OFF_XOFF + h * 4, peer);
-        const uint32_t free_remote0 = map_to_rank(smem_u32(&bars->peer_free[0][quad]), peer);
-        const uint32_t free_remote1 = map_to_rank(smem_u32(&bars->peer_free[1][quad]), peer);
         const float sl2 = args.scale_log2;
         uint32_t g = 0;
         int n = 0;
@@ -521,90 +517,47 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->q_tmem_full);
             }
-            // Per block: send this CTA's half, then finish the block as soon as
-            // the partner's half is in.  (Finishing block j only after sending
-            // block j+1 would tie it to S(j+1), whose buffer waits for P V of
-            // block j-2: a two-block cycle instead of a three-block one.)
+            // Per block: this CTA's half of the logits to the partner.  The
+            // softmax warp of the quadrant combines the two halves; this warp
+            // runs ahead of it by up to the two inbox slots.
             for (int j = 0; j < nb; ++j) {
                 const uint32_t gs = g + j;
                 const int sb = gs % NSBUF;
                 const int slot = gs & 1;
-                // arm this CTA's inbox slot for the partner's half of block gs
-                if (lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD + X_OFF_QUAD);
                 if (!warp_wait(&bars->s_full[sb], (gs / NSBUF) & 1, status, abort, 5)) { ok = false; break; }
                 tc_fence_after();
                 float x[NB];
                 own_logits(t_lane + TM_S + 64 * sb, sl2, masks + ip * 2 * MAX_UNIT_BLOCKS + 2 * j, x);
-                {
-                    // the encoding's offset and step come from the block's largest and
-                    // smallest VALID partial logits (invalid keys are -inf from here on)
-                    const float mb = max64(x);
-                    float mn = min64(x);
-                    if (mn == -INFINITY) mn = min64_finite(x);      // a block with invalid keys
-                    const XCode xc = x_encoder(mb, mn);
-                    // the partner's exchange warp q must have finished this inbox slot
-                    // (block gs-2)
-                    if (!warp_wait_cluster(&bars->peer_free[slot][quad], ((gs >> 1) & 1) ^ 1, status, abort, 6)) {
-                        ok = false;
-                        break;
-                    }
-                    // row h of the partner's inbox, 16 bytes (8 keys) at a time, and
-                    // the head's offset/step word; each st.async counts its bytes on the
-                    // partner's x_full (no fence or arrive on this side)
-                    const uint32_t xr = x_remote + slot * X_TILE;
-                    const uint32_t br = map_to_rank(smem_u32(&bars->x_full[slot][quad]), peer);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        st_async_v4(xr + ((c ^ (h & 7)) << 4),
-                                    x_encode2(xc, x[8 * c + 0], x[8 * c + 1]),
-                                    x_encode2(xc, x[8 * c + 2], x[8 * c + 3]),
-                                    x_encode2(xc, x[8 * c + 4], x[8 * c + 5]),
-                                    x_encode2(xc, x[8 * c + 6], x[8 * c + 7]), br);
-                    st_async_b32(xoff_remote + slot * X_OFF, xc.word, br);
-                }
-                // the partner's half of block gs
-                if (!warp_wait_cluster(&bars->x_full[slot][quad], (gs >> 1) & 1, status, abort, 9)) {
-                    ok = false;
-                    break;
-                }
-                // full logits = own half (float32, still in registers) + the
-                // partner's half rebuilt from its fixed-point codes
-                {
-                    const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + slot * X_TILE + h * 128);
-                    const uint32_t ow = reinterpret_cast<const uint32_t*>(smem + OFF_XOFF + slot * X_OFF)[h];
-                    const float pm = __uint_as_float(ow << 16);
-                    const float pstep = __uint_as_float(((ow >> 16) & 0xffu) << 23);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 w4 = xp[c ^ (h & 7)];
-                        const uint32_t pw4[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            x[8 * c + 2 * e] += x_decode_lo(pw4[e], pm, pstep);
-                            x[8 * c + 2 * e + 1] += x_decode_hi(pw4[e], pm, pstep);
-                        }
-                    }
-                }
-                // every inbox value of this slot has been read: hand it back
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote_relaxed(slot ? free_remote1 : free_remote0);
-                const float mloc = max64(x);
-                // full logits over S, their maximum in its column: the softmax warp's input
-                {
-                    uint32_t w0[32], w1[32];
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        w0[c] = __float_as_uint(x[c]);
-                        w1[c] = __float_as_uint(x[32 + c]);
-                    }
-                    tmem_st32(t_lane + TM_S + 64 * sb, w0);
-                    tmem_st32(t_lane + TM_S + 64 * sb + 32, w1);
-                    tmem_st1(t_lane + TM_MX + sb, __float_as_uint(mloc));
-                }
-                tmem_st_wait();
+                // S(gs) has been read: the softmax warp may read it too and then
+                // overwrite it with P
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
+                // the encoding's offset and step come from the block's largest and
+                // smallest VALID partial logits (invalid keys are -inf from here on)
+                const float mb = max64(x);
+                float mn = min64(x);
+                if (mn == -INFINITY) mn = min64_finite(x);      // a block with invalid keys
+                const XCode xc = x_encoder(mb, mn);
+                // the partner's softmax warp q must have finished this inbox slot
+                // (block gs-2)
+                if (!warp_wait_cluster(&bars->peer_free[slot][quad], ((gs >> 1) & 1) ^ 1, status, abort, 6)) {
+                    ok = false;
+                    break;
+                }
+                // row h of the partner's inbox, 16 bytes (8 keys) at a time, and
+                // the head's offset/step word; each st.async counts its bytes on the
+                // partner's x_full (no fence or arrive on this side)
+                const uint32_t xr = x_remote + slot * X_TILE;
+                const uint32_t br = map_to_rank(smem_u32(&bars->x_full[slot][quad]), peer);
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_async_v4(xr + ((c ^ (h & 7)) << 4),
+                                x_encode2(xc, x[8 * c + 0], x[8 * c + 1]),
+                                x_encode2(xc, x[8 * c + 2], x[8 * c + 3]),
+                                x_encode2(xc, x[8 * c + 4], x[8 * c + 5]),
+                                x_encode2(xc, x[8 * c + 6], x[8 * c + 7]), br);
+                st_async_b32(xoff_remote + slot * X_OFF, xc.word, br);
             }
             g += nb;
             // the unit's masks have been read: the gather warps may refill them
@@ -616,6 +569,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         const int quad = warp & 3;
         const int h = quad * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+        const uint32_t free_remote0 = map_to_rank(smem_u32(&bars->peer_free[0][quad]), peer);
+        const uint32_t free_remote1 = map_to_rank(smem_u32(&bars->peer_free[1][quad]), peer);
+        const float sl2 = args.scale_log2;
         uint32_t g = 0, o_use = 0;
         int n = 0;
         bool ok = true;
@@ -629,27 +585,59 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             float l = 0.f;          // running sum of the bf16-rounded P
             for (int j = 0; j < nb; ++j, ++g) {
                 const int sb = g % NSBUF;
-                // the exchange warp has put the block's full logits (invalid keys
-                // -inf) over S and their maximum in its column
+                const int slot = g & 1;
+                // arm this CTA's inbox slot for the partner's half of block g
+                if (lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD + X_OFF_QUAD);
+                const uint32_t m_lo = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j];
+                const uint32_t m_hi = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j + 1];
+                // S(g) is final in TMEM and the exchange warp has read it
                 if (!warp_wait(&bars->own_full[sb][quad], (g / NSBUF) & 1, status, abort, 8)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                uint32_t s0[32], s1[32];
+                tmem_ld32(t_lane + TM_S + 64 * sb, s0);
+                tmem_ld32(t_lane + TM_S + 64 * sb + 32, s1);
+                // the partner's half of block g
+                if (!warp_wait_cluster(&bars->x_full[slot][quad], (g >> 1) & 1, status, abort, 9)) {
+                    tmem_ld_wait();          // no TMEM load outlives the loop
+                    ok = false;
+                    break;
+                }
+                const uint32_t ow = reinterpret_cast<const uint32_t*>(smem + OFF_XOFF + slot * X_OFF)[h];
+                const float pm = __uint_as_float(ow << 16);
+                const float pstep = __uint_as_float(((ow >> 16) & 0xffu) << 23);
+                const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + slot * X_TILE + h * 128);
+                tmem_ld_wait();
+                // full logits of the 64 keys in base 2: own half (float32) plus the
+                // partner's half rebuilt from its codes; invalid keys -inf
                 float sv[NB];
-                float mloc;
-                {
-                    uint32_t s0[32], s1[32];
-                    tmem_ld32(t_lane + TM_S + 64 * sb, s0);
-                    tmem_ld32(t_lane + TM_S + 64 * sb + 32, s1);
-                    mloc = __uint_as_float(tmem_ld1(t_lane + TM_MX + sb));
-                    tmem_ld_wait();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        sv[c] = __uint_as_float(s0[c]);
-                        sv[32 + c] = __uint_as_float(s1[c]);
+                for (int cc = 0; cc < 8; ++cc) {
+                    const uint4 w4 = xp[cc ^ (h & 7)];                 // keys 8cc .. 8cc+7
+                    const uint32_t pw4[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int key = 8 * cc + e;
+                        const float raw = __uint_as_float(key < 32 ? s0[key] : s1[key - 32]);
+                        const float part = (e & 1) ? x_decode_hi(pw4[e >> 1], pm, pstep)
+                                                   : x_decode_lo(pw4[e >> 1], pm, pstep);
+                        sv[key] = fmaf(raw, sl2, part);
                     }
                 }
+                if ((m_lo & m_hi) != 0xffffffffu) {
+#pragma unroll
+                    for (int kk = 0; kk < NB; ++kk) {
+                        const uint32_t mw = kk < 32 ? m_lo : m_hi;
+                        if (!((mw >> (kk & 31)) & 1u)) sv[kk] = -INFINITY;
+                    }
+                }
+                const float mloc = max64(sv);
+                // every inbox value of this slot has been consumed (mloc depends on
+                // all of them): hand the slot back to the partner's exchange warp
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote_relaxed(slot ? free_remote1 : free_remote0);
                 bool rescale = false;
                 float alpha = 1.f;
                 if (mloc > -INFINITY && (!m_set || mloc > m_use + RESCALE_THRESHOLD)) {
