@@ -7,23 +7,28 @@
 // summary, es page, section 1): the k largest scores, ties to the smaller
 // position, -0.0 = +0.0; kept positions written ascending.
 //
-// The key of the k-th largest score, tau, is found digit by digit, most
-// significant first (11, 11 and 10 bits):
-//   1. every CTA histograms the digit of its keys that still match the
-//      digits chosen so far (warp-aggregated shared-memory atomics);
-//   2. cluster barrier; CTA c sums bins [c*W/CL, (c+1)*W/CL) of all CL
-//      histograms through distributed shared memory, and their total;
-//   3. cluster barrier; every CTA reads the CL slice totals, finds the slice
-//      and then, in its owner's reduced bins, the bin that holds the
-//      need-th largest remaining key, and appends that digit.
-// Then each CTA counts its keys above tau and equal to tau; after one more
-// cluster barrier every CTA knows, from all counts, where its kept positions
-// go and how many of its equal-to-tau keys to keep (the smaller positions
-// first, so segments of lower rank keep theirs first), and writes them in
-// position order.  Every wait is a hardware cluster barrier that all CTAs of
-// the cluster reach in the same sequence: no flag, no spin-wait, no global
-// workspace.
+// The key of the k-th largest score, tau, is found as follows:
+//   1. every CTA histograms the top 11 bits of its keys (warp-aggregated
+//      shared-memory atomics); cluster barrier; every CTA sums all CL
+//      histograms through distributed shared memory (the same sums in every
+//      CTA) and finds the bin d0 that holds the k-th largest key;
+//   2. if the whole cluster holds few keys in bin d0 (at most CAND_CAP):
+//      every CTA compacts its keys of bin d0; cluster barrier; every CTA
+//      gathers all of them and finds tau among them locally (the same
+//      deterministic result in every CTA), and from the gathered keys and
+//      the lower-ranked CTAs' counts above bin d0 where its kept positions
+//      go;
+//   3. otherwise (many keys in one bin: heavy ties) the remaining 21 bits
+//      are resolved digit by digit (11 and 10 bits), each digit's histogram
+//      reduced over the cluster slice by slice, then counted.
+// Each CTA then writes its kept positions in position order, keeping its
+// keys equal to tau after those of lower-ranked CTAs (smaller positions
+// first).  Every wait is a hardware cluster barrier that all CTAs of the
+// cluster reach in the same sequence (the path taken is decided from values
+// every CTA holds identically): no flag, no spin-wait, no global workspace.
 #pragma once
+
+#include <cstddef>
 
 #include "topk_common.cuh"
 
@@ -32,15 +37,30 @@ namespace csel {
 
 constexpr int HBINS = 2048;             // 11-bit digits
 
+constexpr int CAND_CAP = 2 * HBINS;   // keys of bin d0 the compaction path takes (cluster total)
+
 template <int NW>
 struct __align__(16) ClusterSmem {
-    uint32_t hist[HBINS];               // this CTA's histogram of the current digit
-    uint32_t red[HBINS];                // reduced bins owned by this CTA (W / CL of them)
+    // this CTA's histogram of the current digit, then the cluster's reduced
+    // bins; on the compaction path both arrays together hold the gathered
+    // candidates of every CTA (CAND_CAP keys)
+    uint32_t hist[HBINS];
+    uint32_t red[HBINS];
+    uint32_t cand[CAND_CAP];            // this CTA's keys of bin d0 (compaction path)
+    SelectState<NW> st;                 // local radix select over the gathered candidates
     uint32_t warp_cnt[2][NW];
     uint32_t slice_tot;                 // total of the reduced bins owned by this CTA
     uint32_t cnt_gt, cnt_eq;            // keys > tau and == tau in this CTA's segment
     uint32_t prefix, need;              // digits chosen so far; keys still to take at the prefix
+    uint32_t n_cand, gt0;               // this CTA's keys in bin d0, and above bin d0
+    uint32_t d0_total;                  // the cluster's keys in bin d0
+    uint32_t cand_off[17];              // gathered candidates: CTA c's start (c <= CL)
+    uint32_t gt_before;                 // keys above bin d0 in the lower-ranked CTAs
 };
+static_assert(2 * HBINS >= CAND_CAP, "gathered candidates fit in hist + red");
+// the gathered candidates use hist and red as one array
+static_assert(offsetof(ClusterSmem<16>, red) == offsetof(ClusterSmem<16>, hist) + sizeof(uint32_t) * HBINS,
+              "hist and red are adjacent");
 
 __device__ __forceinline__ uint32_t ld_dsmem(uint32_t cluster_addr) {
     uint32_t v;
@@ -121,6 +141,82 @@ __device__ __forceinline__ void warp_find_from_top(const uint32_t* c, int m, uin
 }
 
 
+// One pass of warp-aggregated shared-memory histogramming over this CTA's
+// keys: bin (key >> shift) & (W-1) of every key whose bits above the digit
+// equal `prefix` (all keys when done_bits == 0).  All NT threads.
+template <int NT>
+__device__ __forceinline__ void digit_histogram(uint32_t* hist, const uint32_t* keys, int m,
+                                                int done_bits, int width, uint32_t prefix) {
+    const int lane = threadIdx.x & 31;
+    const int W = 1 << width;
+    const int shift = 32 - done_bits - width;
+    for (int b = threadIdx.x; b < W; b += NT) hist[b] = 0;
+    __syncthreads();
+    const int m_round = (m + 31) & ~31;      // whole warps: the match below takes every lane
+    for (int j = threadIdx.x; j < m_round; j += NT) {
+        bool live = j < m;
+        const uint32_t key = live ? keys[j] : 0u;
+        if (done_bits > 0) live = live && (key >> (32 - done_bits)) == prefix;
+        const uint32_t digit = live ? ((key >> shift) & (uint32_t)(W - 1)) : 0xffffffffu;
+        const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+        if (live && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+    }
+}
+
+// Writes this CTA's kept positions (keys > tau, and the first eq_keep keys
+// equal to tau) in position order from dst[out_off].  All NT threads.
+template <int NT>
+__device__ __forceinline__ void ordered_write(uint32_t (&warp_cnt)[2][NT / 32], const uint32_t* keys,
+                                              int m, int s0, uint32_t tau, uint32_t out_off,
+                                              uint32_t eq_keep, int32_t* __restrict__ dst) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t run_gt = 0, run_eq = 0;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const int m_round = (m + NT - 1) / NT * NT;
+    for (int base = 0; base < m_round; base += NT) {
+        const int j = base + threadIdx.x;
+        const uint32_t key = j < m ? keys[j] : 0u;
+        const bool gt = j < m && key > tau;
+        const bool eq = j < m && key == tau;
+        const uint32_t bg = __ballot_sync(0xffffffffu, gt);
+        const uint32_t be = __ballot_sync(0xffffffffu, eq);
+        const int buf = (base / NT) & 1;
+        if (lane == 0) warp_cnt[buf][warp] = __popc(bg) | ((uint32_t)__popc(be) << 16);
+        __syncthreads();
+        uint32_t pre_gt = 0, pre_eq = 0, tot_gt = 0, tot_eq = 0;
+#pragma unroll
+        for (int w2 = 0; w2 < NW; ++w2) {
+            const uint32_t v = warp_cnt[buf][w2];
+            if (w2 < warp) { pre_gt += v & 0xffffu; pre_eq += v >> 16; }
+            tot_gt += v & 0xffffu;
+            tot_eq += v >> 16;
+        }
+        const uint32_t gt_before = run_gt + pre_gt + __popc(bg & lt_mask);
+        const uint32_t eq_before = run_eq + pre_eq + __popc(be & lt_mask);
+        if (gt || (eq && eq_before < eq_keep))
+            dst[out_off + gt_before + min(eq_before, eq_keep)] = s0 + j;
+        run_gt += tot_gt;
+        run_eq += tot_eq;
+        // warp_cnt is double-buffered, so one barrier per chunk suffices
+    }
+}
+
+// Block-wide sum of one value per thread; the result in every thread.
+template <int NT>
+__device__ __forceinline__ uint32_t block_sum(uint32_t v, uint32_t* scratch /* NT/32 words */) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();                     // scratch may still be read by a previous use
+    if (lane == 0) scratch[warp] = v;
+    __syncthreads();
+    uint32_t t = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) t += scratch[w];
+    return t;
+}
+
 // Exact top-k of one row of n > k candidates, the segment [s0, s0 + m) of
 // which is cached in this CTA's shared memory as order keys `keys`; called
 // by all NT threads of every CTA of the cluster (CL CTAs, this one `rank`),
@@ -129,166 +225,213 @@ __device__ __forceinline__ void warp_find_from_top(const uint32_t* c, int m, uin
 template <int NT>
 __device__ void cluster_select(ClusterSmem<NT / 32>& S, const uint32_t* keys, int m, int s0, int k,
                                int32_t* __restrict__ dst, uint32_t CL, uint32_t rank) {
-    constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (threadIdx.x == 0) {
-        S.prefix = 0;
-        S.need = (uint32_t)k;
+
+    // ------------------------------------------------------ top 11 bits, bin d0
+    digit_histogram<NT>(S.hist, keys, m, 0, 11, 0u);
+    cluster_barrier();   // every CTA's histogram is complete
+    // every CTA sums all CL histograms (the same sums everywhere); the CL
+    // remote loads of a bin are all in flight before they are added
+    for (int b = threadIdx.x; b < HBINS; b += NT) {
+        uint32_t v[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+            if (c < (int)CL) v[c] = ld_dsmem(map_rank(&S.hist[b], (uint32_t)c));
+        uint32_t sum = 0;
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+            if (c < (int)CL) sum += v[c];
+        S.red[b] = sum;
     }
     __syncthreads();
-
-    // ---------------------------------------------------------------- digits
-    int done_bits = 0;
-    for (int pass = 0; pass < 3; ++pass) {
-        const int width = pass < 2 ? 11 : 10;
-        const int W = 1 << width;
-        const int shift = 32 - done_bits - width;
-        for (int b = threadIdx.x; b < W; b += NT) S.hist[b] = 0;
-        __syncthreads();
-        const uint32_t prefix = S.prefix;
-        const int m_round = (m + 31) & ~31;
-        for (int j = threadIdx.x; j < m_round; j += NT) {
-            bool live = j < m;
-            uint32_t key = live ? keys[j] : 0u;
-            if (done_bits > 0) live = live && (key >> (32 - done_bits)) == prefix;
-            const uint32_t digit = live ? ((key >> shift) & (uint32_t)(W - 1)) : 0xffffffffu;
-            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-            if (live && lane == __ffs(peers) - 1) atomicAdd(&S.hist[digit], __popc(peers));
+    if (warp == 0) {
+        uint32_t d0, above;
+        warp_find_from_top(S.red, HBINS, (uint32_t)k, false, 0u, d0, above);
+        if (lane == 0) {
+            S.prefix = d0;
+            S.need = (uint32_t)k - above;          // keys still to take from bin d0
+            S.d0_total = S.red[d0];
         }
-        cluster_barrier();   // every CTA's histogram is complete
-        // reduce my slice of the bins over the cluster
-        const int per = W / (int)CL;
-        uint32_t part = 0;
-        for (int t = threadIdx.x; t < per; t += NT) {
-            const int bin = (int)rank * per + t;
-            uint32_t sum = 0;
-            for (uint32_t c = 0; c < CL; ++c) sum += ld_dsmem(map_rank(&S.hist[bin], c));
-            S.red[t] = sum;
-            part += sum;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        if (lane == 0) S.warp_cnt[0][warp] = part;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            uint32_t tot = 0;
-            for (int w = 0; w < NW; ++w) tot += S.warp_cnt[0][w];
-            S.slice_tot = tot;
-        }
-        cluster_barrier();   // every CTA's reduced slice and total are complete
-        if (warp == 0) {
-            const uint32_t need = S.need;
-            // the slice (owner CTA) holding the need-th largest key, from the top
-            uint32_t owner, above_slices;
-            {
-                uint32_t tot = lane < (int)CL ? ld_dsmem(map_rank(&S.slice_tot, (uint32_t)lane)) : 0u;
-                // top-down: slice CL-1 holds the highest bins
-                const int pos = lane;                       // top-down position
-                const int sl = (int)CL - 1 - pos;
-                // every lane takes part in the shuffle (a full-mask shuffle that
-                // some lanes skip never completes); lanes past CL then drop it
-                const uint32_t from_sl = __shfl_sync(0xffffffffu, tot, sl < 0 ? 0 : sl);
-                const uint32_t mine = pos < (int)CL ? from_sl : 0u;
-                uint32_t incl = mine;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += v;
-                }
-                const uint32_t hit = __ballot_sync(0xffffffffu, incl >= need && pos < (int)CL);
-                const int p = hit ? __ffs(hit) - 1 : 0;
-                owner = (uint32_t)((int)CL - 1 - p);
-                above_slices = __shfl_sync(0xffffffffu, incl - mine, p);
-            }
-            uint32_t bin_in_slice, before;
-            warp_find_from_top(nullptr, per, need - above_slices, true, map_rank(&S.red[0], owner),
-                               bin_in_slice, before);
-            if (lane == 0) {
-                const uint32_t digit = owner * (uint32_t)per + bin_in_slice;
-                S.prefix = (S.prefix << width) | digit;
-                S.need = need - above_slices - before;
-            }
-        }
-        __syncthreads();
-        done_bits += width;
     }
-    const uint32_t tau = S.prefix;
-    const uint32_t need_eq = S.need;      // keys equal to tau to keep (smallest positions first)
+    __syncthreads();
+    const uint32_t d0 = S.prefix;
+    uint32_t tau, need_eq, out_off, eq_keep;
 
-    // ---------------------------------------------------------------- counts
-    {
+    if (S.d0_total <= (uint32_t)CAND_CAP) {
+        // ----------------------------------------------- compaction path
+        // this CTA's keys of bin d0 (any order) and its count above bin d0
+        if (threadIdx.x == 0) S.n_cand = 0;
+        __syncthreads();
+        uint32_t gt0 = 0;
+        const int m_round = (m + 31) & ~31;      // whole warps: ballot and shuffle take every lane
+        for (int j = threadIdx.x; j < m_round; j += NT) {
+            const uint32_t key = j < m ? keys[j] : 0u;
+            const uint32_t dig = key >> 21;
+            const bool cand = j < m && dig == d0;
+            gt0 += (j < m && dig > d0) ? 1u : 0u;
+            const uint32_t bal = __ballot_sync(0xffffffffu, cand);
+            if (bal != 0u) {                     // the same in every lane
+                const int src = __ffs(bal) - 1;
+                uint32_t slot0 = 0;
+                if (lane == src) slot0 = atomicAdd(&S.n_cand, __popc(bal));
+                slot0 = __shfl_sync(0xffffffffu, slot0, src);
+                if (cand) S.cand[slot0 + __popc(bal & ((1u << lane) - 1u))] = key;
+            }
+        }
+        gt0 = block_sum<NT>(gt0, S.warp_cnt[0]);
+        if (threadIdx.x == 0) S.gt0 = gt0;
+        cluster_barrier();   // every CTA's candidates and counts are complete; no CTA
+                             // reads another's histogram any more
+        if (warp == 0) {
+            const uint32_t nc = lane < (int)CL ? ld_dsmem(map_rank(&S.n_cand, (uint32_t)lane)) : 0u;
+            const uint32_t g0 = lane < (int)CL ? ld_dsmem(map_rank(&S.gt0, (uint32_t)lane)) : 0u;
+            uint32_t incl = nc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            uint32_t gb = lane < (int)rank ? g0 : 0u;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) gb += __shfl_xor_sync(0xffffffffu, gb, o);
+            if (lane <= (int)CL) S.cand_off[lane] = incl - nc;   // lane CL: the total
+            if (lane == 0) S.gt_before = gb;
+        }
+        __syncthreads();
+        // every CTA's candidates, in rank order, into this CTA's hist + red
+        uint32_t* gathered = S.hist;
+        const uint32_t total = S.cand_off[CL];
+        for (uint32_t base = 0; base < total; base += 8u * NT) {
+            uint32_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t i = base + (uint32_t)u * NT + threadIdx.x;
+                v[u] = 0u;
+                if (i < total) {
+                    uint32_t c = 0;
+                    while (c + 1 < CL && S.cand_off[c + 1] <= i) ++c;
+                    v[u] = ld_dsmem(map_rank(&S.cand[i - S.cand_off[c]], c));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t i = base + (uint32_t)u * NT + threadIdx.x;
+                if (i < total) gathered[i] = v[u];
+            }
+        }
+        __syncthreads();
+        // tau among the gathered keys of bin d0 (identical in every CTA)
+        select_smem_known<NT>(gathered, (int)total, S.need, d0, 11, S.st);
+        tau = S.st.prefix;
+        need_eq = S.st.need;
+        // keys above and equal to tau in the lower-ranked CTAs' candidates, and
+        // this CTA's keys equal to tau
+        const uint32_t lo = S.cand_off[rank], hi = S.cand_off[rank + 1];
+        uint32_t before = 0, eq_me = 0;
+        for (uint32_t i = threadIdx.x; i < hi; i += NT) {
+            const uint32_t key = gathered[i];
+            if (i < lo) before += (key > tau ? 1u : 0u) | (key == tau ? 0x10000u : 0u);
+            else eq_me += key == tau ? 1u : 0u;
+        }
+        before = block_sum<NT>(before, S.warp_cnt[0]);
+        eq_me = block_sum<NT>(eq_me, S.warp_cnt[0]);
+        const uint32_t gt_p = before & 0xffffu, eq_p = before >> 16;
+        out_off = S.gt_before + gt_p + min(eq_p, need_eq);
+        eq_keep = need_eq > eq_p ? min(eq_me, need_eq - eq_p) : 0u;
+    } else {
+        // ----------------------------------------------- many keys in bin d0
+        cluster_barrier();   // no CTA reads another's histogram any more
+        // the remaining 21 bits, digit by digit (11 then 10 bits), each
+        // digit's histogram reduced over the cluster slice by slice
+        int done_bits = 11;
+        for (int pass = 1; pass < 3; ++pass) {
+            const int width = pass < 2 ? 11 : 10;
+            const int W = 1 << width;
+            digit_histogram<NT>(S.hist, keys, m, done_bits, width, S.prefix);
+            cluster_barrier();   // every CTA's histogram is complete
+            // reduce my slice of the bins over the cluster
+            const int per = W / (int)CL;
+            uint32_t part = 0;
+            for (int t = threadIdx.x; t < per; t += NT) {
+                const int bin = (int)rank * per + t;
+                uint32_t v[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    if (c < (int)CL) v[c] = ld_dsmem(map_rank(&S.hist[bin], (uint32_t)c));
+                uint32_t sum = 0;
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    if (c < (int)CL) sum += v[c];
+                S.red[t] = sum;
+                part += sum;
+            }
+            part = block_sum<NT>(part, S.warp_cnt[0]);
+            if (threadIdx.x == 0) S.slice_tot = part;
+            cluster_barrier();   // every CTA's reduced slice and total are complete
+            if (warp == 0) {
+                const uint32_t need = S.need;
+                // the slice (owner CTA) holding the need-th largest key, from the top
+                uint32_t owner, above_slices;
+                {
+                    const uint32_t tot = lane < (int)CL ? ld_dsmem(map_rank(&S.slice_tot, (uint32_t)lane)) : 0u;
+                    // top-down: slice CL-1 holds the highest bins
+                    const int pos = lane;                       // top-down position
+                    const int sl = (int)CL - 1 - pos;
+                    // every lane takes part in the shuffle (a full-mask shuffle that
+                    // some lanes skip never completes); lanes past CL then drop it
+                    const uint32_t from_sl = __shfl_sync(0xffffffffu, tot, sl < 0 ? 0 : sl);
+                    const uint32_t mine = pos < (int)CL ? from_sl : 0u;
+                    uint32_t incl = mine;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += v;
+                    }
+                    const uint32_t hit = __ballot_sync(0xffffffffu, incl >= need && pos < (int)CL);
+                    const int p = hit ? __ffs(hit) - 1 : 0;
+                    owner = (uint32_t)((int)CL - 1 - p);
+                    above_slices = __shfl_sync(0xffffffffu, incl - mine, p);
+                }
+                uint32_t bin_in_slice, before;
+                warp_find_from_top(nullptr, per, need - above_slices, true, map_rank(&S.red[0], owner),
+                                   bin_in_slice, before);
+                if (lane == 0) {
+                    const uint32_t digit = owner * (uint32_t)per + bin_in_slice;
+                    S.prefix = (S.prefix << width) | digit;
+                    S.need = need - above_slices - before;
+                }
+            }
+            __syncthreads();
+            done_bits += width;
+        }
+        tau = S.prefix;
+        need_eq = S.need;      // keys equal to tau to keep (smallest positions first)
+        // this CTA's keys above and equal to tau
         uint32_t gt = 0, eq = 0;
         for (int j = threadIdx.x; j < m; j += NT) {
             const uint32_t key = keys[j];
             gt += key > tau ? 1u : 0u;
             eq += key == tau ? 1u : 0u;
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            gt += __shfl_xor_sync(0xffffffffu, gt, o);
-            eq += __shfl_xor_sync(0xffffffffu, eq, o);
-        }
-        if (lane == 0) {
-            S.warp_cnt[0][warp] = gt;
-            S.warp_cnt[1][warp] = eq;
-        }
-        __syncthreads();
+        gt = block_sum<NT>(gt, S.warp_cnt[0]);
+        eq = block_sum<NT>(eq, S.warp_cnt[0]);
         if (threadIdx.x == 0) {
-            uint32_t a = 0, b = 0;
-            for (int w = 0; w < NW; ++w) { a += S.warp_cnt[0][w]; b += S.warp_cnt[1][w]; }
-            S.cnt_gt = a;
-            S.cnt_eq = b;
+            S.cnt_gt = gt;
+            S.cnt_eq = eq;
         }
-    }
-    cluster_barrier();   // every CTA's counts are complete
-    uint32_t out_off = 0, eq_keep = 0;
-    {
+        cluster_barrier();   // every CTA's counts are complete
         // lower ranks hold smaller positions: they write first and keep their
         // equal-to-tau keys first
-        uint32_t eq_before = 0;
+        uint32_t off = 0, eq_before = 0;
         for (uint32_t c = 0; c < rank; ++c) {
-            const uint32_t g = ld_dsmem(map_rank(&S.cnt_gt, c));
-            const uint32_t e = ld_dsmem(map_rank(&S.cnt_eq, c));
-            const uint32_t keep = eq_before >= need_eq ? 0u : min(e, need_eq - eq_before);
-            out_off += g + keep;
-            eq_before += e;
+            off += ld_dsmem(map_rank(&S.cnt_gt, c));
+            eq_before += ld_dsmem(map_rank(&S.cnt_eq, c));
         }
-        eq_keep = eq_before >= need_eq ? 0u : min(S.cnt_eq, need_eq - eq_before);
+        out_off = off + min(eq_before, need_eq);
+        eq_keep = need_eq > eq_before ? min(eq, need_eq - eq_before) : 0u;
     }
-    __syncthreads();
-
-    // ---------------------------------------------------------------- ordered write
-    {
-        uint32_t run_gt = 0, run_eq = 0;
-        const uint32_t lt_mask = (1u << lane) - 1u;
-        const int m_round = (m + NT - 1) / NT * NT;
-        for (int base = 0; base < m_round; base += NT) {
-            const int j = base + threadIdx.x;
-            const uint32_t key = j < m ? keys[j] : 0u;
-            const bool gt = j < m && key > tau;
-            const bool eq = j < m && key == tau;
-            const uint32_t bg = __ballot_sync(0xffffffffu, gt);
-            const uint32_t be = __ballot_sync(0xffffffffu, eq);
-            const int buf = (base / NT) & 1;
-            if (lane == 0) S.warp_cnt[buf][warp] = __popc(bg) | ((uint32_t)__popc(be) << 16);
-            __syncthreads();
-            uint32_t pre_gt = 0, pre_eq = 0, tot_gt = 0, tot_eq = 0;
-#pragma unroll
-            for (int w2 = 0; w2 < NW; ++w2) {
-                const uint32_t v = S.warp_cnt[buf][w2];
-                if (w2 < warp) { pre_gt += v & 0xffffu; pre_eq += v >> 16; }
-                tot_gt += v & 0xffffu;
-                tot_eq += v >> 16;
-            }
-            const uint32_t gt_before = run_gt + pre_gt + __popc(bg & lt_mask);
-            const uint32_t eq_before = run_eq + pre_eq + __popc(be & lt_mask);
-            if (gt || (eq && eq_before < eq_keep))
-                dst[out_off + gt_before + min(eq_before, eq_keep)] = s0 + j;
-            run_gt += tot_gt;
-            run_eq += tot_eq;
-        }
-    }
-    cluster_barrier();   // no CTA leaves while another may still read its counts
+    ordered_write<NT>(S.warp_cnt, keys, m, s0, tau, out_off, eq_keep, dst);
+    cluster_barrier();   // no CTA leaves while another may still read its shared memory
 }
 
 }  // namespace csel

@@ -20,7 +20,7 @@ namespace {
 using csel::ClusterSmem;
 
 constexpr int NT = 512;
-constexpr int CL_MAX = 8;               // portable cluster size
+constexpr int CL_MAX = 16;              // non-portable cluster size (B200: up to 16)
 constexpr int SEG_MAX = 40960;          // keys of one CTA cached in shared memory (160 KB)
 
 __global__ void __launch_bounds__(NT, 1)
@@ -48,38 +48,90 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, int Lq, int q_
     const int m = s1 - s0;
     const float* src = scores + row * ld + s0;
     // scores -> order keys in shared memory (16-byte loads: s0 and the row
-    // start are multiples of 4 floats)
-    for (int j = 4 * threadIdx.x; j < m; j += 4 * NT) {
-        if (j + 3 < m) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(src + j));
-            *reinterpret_cast<uint4*>(keys + j) =
-                make_uint4(order_key(v.x), order_key(v.y), order_key(v.z), order_key(v.w));
-        } else {
-            for (int q = j; q < m; ++q) keys[q] = order_key(src[q]);
+    // start are multiples of 4 floats), four loads in flight per thread
+    for (int j0 = 4 * threadIdx.x; j0 < m; j0 += 16 * NT) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + 4 * NT * u;
+            if (j + 3 < m) v[u] = __ldg(reinterpret_cast<const float4*>(src + j));
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + 4 * NT * u;
+            if (j + 3 < m) {
+                *reinterpret_cast<uint4*>(keys + j) =
+                    make_uint4(order_key(v[u].x), order_key(v[u].y), order_key(v[u].z), order_key(v[u].w));
+            } else {
+                for (int q = j; q < m; ++q) keys[q] = order_key(src[q]);
+            }
         }
     }
+    __syncthreads();
     csel::cluster_select<NT>(S, keys, m, s0, k, dst, CL, rank);
+}
+
+
+size_t cluster_smem(int seg) { return sizeof(ClusterSmem<NT / 32>) + (size_t)seg * sizeof(uint32_t); }
+
+int segment(int n_max, int cl) { return ((n_max + cl - 1) / cl + 3) & ~3; }
+
+// Co-resident clusters of size cl with `smem` bytes per CTA (0 if none fits).
+int active_clusters(int cl, size_t smem) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cl, 1, 1);
+    cfg.blockDim = dim3(NT, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
+bool kernel_attributes_set() {
+    static int done = -1;
+    if (done < 0)
+        done = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)cluster_smem(SEG_MAX)) == cudaSuccess &&
+               cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                    1) == cudaSuccess;
+    if (!done) cudaGetLastError();
+    return done;
 }
 
 }  // namespace
 
-// Cluster size for `rows` rows of up to n_max candidates: the most CTAs per
-// row (a power of two, at most CL_MAX) that keeps every row in one wave of
-// the GPU's SMs, and enough CTAs that each segment fits in shared memory.
-// Returns 0 if no cluster size fits.
+// Cluster size for `rows` rows of up to n_max candidates: among the sizes
+// whose segment fits in shared memory, the one that minimises (waves of
+// co-resident clusters) x (keys per CTA), i.e. the most CTAs per row that
+// still keep the rows in as few waves as possible.  0 if none fits.
 int topk_cluster_size(ic_rows r, int k) {
     const int64_t rows = (int64_t)r.B * r.Lq;
     const int n_max = r.q_start + r.Lq;
-    if (rows <= 0 || n_max <= k) return 0;
-    int sms = 148;
-    int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int cl = 1;
-    while (cl < CL_MAX && rows * (cl * 2) <= sms) cl *= 2;
-    while (cl < CL_MAX && (n_max + cl - 1) / cl > SEG_MAX) cl *= 2;
-    if (((n_max + cl - 1) / cl + 3) / 4 * 4 > SEG_MAX) return 0;
-    return cl;
+    if (rows <= 0 || n_max <= k || !kernel_attributes_set()) return 0;
+    int best = 0;
+    double best_cost = 1e300;
+    for (int cl = 1; cl <= CL_MAX; cl *= 2) {
+        const int seg = segment(n_max, cl);
+        if (seg > SEG_MAX) continue;
+        const int act = active_clusters(cl, cluster_smem(seg));
+        if (act <= 0) continue;
+        const double cost = (double)((rows + act - 1) / act) * (double)seg;
+        if (cost < best_cost * 0.999) {
+            best_cost = cost;
+            best = cl;
+        }
+    }
+    return best;
 }
 
 bool topk_cluster_applies(ic_rows r, int k) {
@@ -94,11 +146,7 @@ ic_status launch_topk_cluster(const float* scores, int64_t ld, ic_rows r, int k,
     if (cl == 0) return IC_ERR_UNSUPPORTED;
     const int64_t rows = (int64_t)r.B * r.Lq;
     const int n_max = r.q_start + r.Lq;
-    const int seg = ((n_max + cl - 1) / cl + 3) & ~3;
-    const size_t smem = sizeof(ClusterSmem<NT / 32>) + (size_t)seg * sizeof(uint32_t);
-    if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-        return cuda_error("topk_cluster");
+    const size_t smem = cluster_smem(segment(n_max, cl));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(rows * cl), 1, 1);
     cfg.blockDim = dim3(NT, 1, 1);
