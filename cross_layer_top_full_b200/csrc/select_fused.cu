@@ -18,7 +18,10 @@
 //      the CL cached segments, with cluster barriers only.
 // Dense keys, or paged keys with per-sequence lengths.
 #include <algorithm>
+#include <map>
 #include <mutex>
+#include <tuple>
+#include <utility>
 
 #include "cluster_select.cuh"
 #include "indexer_pipeline.cuh"
@@ -168,7 +171,7 @@ int active_clusters(int cl, size_t smem) {
 // Cluster size: the one that minimises (waves of clusters) x (keys per CTA),
 // among the sizes whose segment fits in shared memory.  0 if none does.
 template <int H, bool FP8>
-int choose_cluster(int64_t rows, int n_max, size_t& smem_out) {
+int choose_cluster_uncached(int64_t rows, int n_max, size_t& smem_out) {
     const size_t cap = seg_capacity<H, FP8>();
     int best = 0;
     double best_cost = 1e300;
@@ -186,6 +189,31 @@ int choose_cluster(int64_t rows, int n_max, size_t& smem_out) {
         }
     }
     return best;
+}
+
+// The same, one answer per (device, rows, n_max): the occupancy queries cost
+// host time on every launch otherwise.
+template <int H, bool FP8>
+int choose_cluster(int64_t rows, int n_max, size_t& smem_out) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::mutex mu;
+    static std::map<std::tuple<int, int64_t, int>, std::pair<int, size_t>> cache;
+    const auto key = std::make_tuple(dev, rows, n_max);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        const auto it = cache.find(key);
+        if (it != cache.end()) {
+            smem_out = it->second.second;
+            return it->second.first;
+        }
+    }
+    size_t smem = 0;
+    const int cl = choose_cluster_uncached<H, FP8>(rows, n_max, smem);
+    std::lock_guard<std::mutex> lock(mu);
+    cache[key] = std::make_pair(cl, smem);
+    smem_out = smem;
+    return cl;
 }
 
 template <int H, bool FP8>

@@ -11,6 +11,9 @@
 // exact top-k with three radix digits reduced over distributed shared memory
 // and cluster barriers only (no flag, no spin-wait, no global workspace).
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include "cluster_select.cuh"
 
@@ -118,6 +121,17 @@ int topk_cluster_size(ic_rows r, int k) {
     const int64_t rows = (int64_t)r.B * r.Lq;
     const int n_max = r.q_start + r.Lq;
     if (rows <= 0 || n_max <= k || !kernel_attributes_set()) return 0;
+    // the occupancy queries cost host time: one answer per (device, rows, n_max)
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::mutex mu;
+    static std::map<std::tuple<int, int64_t, int>, int> cache;
+    const auto key = std::make_tuple(dev, rows, n_max);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        const auto it = cache.find(key);
+        if (it != cache.end()) return it->second;
+    }
     int best = 0;
     double best_cost = 1e300;
     for (int cl = 1; cl <= CL_MAX; cl *= 2) {
@@ -131,6 +145,8 @@ int topk_cluster_size(ic_rows r, int k) {
             best = cl;
         }
     }
+    std::lock_guard<std::mutex> lock(mu);
+    cache[key] = best;
     return best;
 }
 
