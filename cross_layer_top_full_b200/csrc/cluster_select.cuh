@@ -8,8 +8,8 @@
 // position, -0.0 = +0.0; kept positions written ascending.
 //
 // The key of the k-th largest score, tau, is found as follows:
-//   1. every CTA histograms the top 11 bits of its keys (warp-aggregated
-//      shared-memory atomics); cluster barrier; every CTA sums all CL
+//   1. every CTA histograms the top 11 bits of its keys (shared-memory
+//      atomics); cluster barrier; every CTA sums all CL
 //      histograms through distributed shared memory (the same sums in every
 //      CTA) and finds the bin d0 that holds the k-th largest key;
 //   2. if the whole cluster holds few keys in bin d0 (at most CAND_CAP):
@@ -141,25 +141,23 @@ __device__ __forceinline__ void warp_find_from_top(const uint32_t* c, int m, uin
 }
 
 
-// One pass of warp-aggregated shared-memory histogramming over this CTA's
+// One pass of shared-memory histogramming (warp_hist_add) over this CTA's
 // keys: bin (key >> shift) & (W-1) of every key whose bits above the digit
 // equal `prefix` (all keys when done_bits == 0).  All NT threads.
 template <int NT>
 __device__ __forceinline__ void digit_histogram(uint32_t* hist, const uint32_t* keys, int m,
                                                 int done_bits, int width, uint32_t prefix) {
-    const int lane = threadIdx.x & 31;
     const int W = 1 << width;
     const int shift = 32 - done_bits - width;
     for (int b = threadIdx.x; b < W; b += NT) hist[b] = 0;
     __syncthreads();
-    const int m_round = (m + 31) & ~31;      // whole warps: the match below takes every lane
+    const int m_round = (m + 31) & ~31;      // whole warps: every lane takes part in the update
     for (int j = threadIdx.x; j < m_round; j += NT) {
         bool live = j < m;
         const uint32_t key = live ? keys[j] : 0u;
         if (done_bits > 0) live = live && (key >> (32 - done_bits)) == prefix;
         const uint32_t digit = live ? ((key >> shift) & (uint32_t)(W - 1)) : 0xffffffffu;
-        const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-        if (live && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+        warp_hist_add(hist, digit, live);
     }
 }
 

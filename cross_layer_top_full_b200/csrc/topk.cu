@@ -12,8 +12,8 @@
 // of non-negatives; -0.0 is first mapped to +0.0).  The row is read from
 // memory ONCE: while it streams in, every key's top 16 bits are kept in
 // shared memory and its top 11 bits are counted in a 2048-bin histogram
-// (warp-aggregated shared-memory atomics, so clustered digits do not
-// serialise).  The bin d that holds the k-th largest key splits the row into
+// (shared-memory atomics; a warp whose 32 keys share one digit adds 32 at
+// once, so clustered digits do not serialise).  The bin d that holds the k-th largest key splits the row into
 // keys that are surely kept (top 11 bits above d), surely dropped (below d)
 // and the candidates (equal to d).  One pass over the shared-memory keys
 // collects the candidates' positions; only their full scores are fetched
@@ -91,8 +91,7 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int Lq, int q_sta
             const uint32_t key = order_key(f[q]);
             if (live) hi[j + q] = (uint16_t)(key >> 16);
             const uint32_t digit = live ? (key >> 21) : 0xffffffffu;
-            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-            if (live && lane == __ffs(peers) - 1) atomicAdd(&S.hist[digit], __popc(peers));
+            warp_hist_add(S.hist, digit, live);
         }
     }
     __syncthreads();

@@ -22,6 +22,20 @@ __device__ __forceinline__ int row_candidates(int64_t row, int Lq, int q_start,
     return (Tb >= Lq && Tb <= T_max) ? Tb - Lq + i + 1 : 0;
 }
 
+// Histogram update of one warp: +1 at hist[digit] for every live lane.  A
+// warp whose lanes all carry the same digit (clustered scores) adds 32 from
+// one lane; otherwise each live lane adds its own 1 (shared-memory atomics
+// resolve the few collisions of scattered digits).  Every lane of the warp
+// must call it; dead lanes pass a digit no live lane can have.
+__device__ __forceinline__ void warp_hist_add(uint32_t* hist, uint32_t digit, bool live) {
+    const uint32_t d0 = __shfl_sync(0xffffffffu, digit, 0);
+    if (__all_sync(0xffffffffu, digit == d0)) {
+        if ((threadIdx.x & 31) == 0 && live) atomicAdd(&hist[digit], 32u);
+    } else if (live) {
+        atomicAdd(&hist[digit], 1u);
+    }
+}
+
 // Larger score -> larger key; -0.0 and +0.0 give the same key.
 __device__ __forceinline__ uint32_t order_key(float f) {
     uint32_t u = __float_as_uint(f);
@@ -94,7 +108,7 @@ __device__ void select_row(const float* __restrict__ src, int n, int k, int32_t*
         for (int j = threadIdx.x; j < 256; j += NT) st.hist[j] = 0;
         __syncthreads();
         const uint32_t prefix = st.prefix;
-        // round the loop up to whole warps so __match_any_sync sees full warps
+        // round the loop up to whole warps: every lane takes part in the warp update
         const int n_round = (n + 31) & ~31;
         for (int j = threadIdx.x; j < n_round; j += NT) {
             bool live = j < n;
@@ -109,8 +123,7 @@ __device__ void select_row(const float* __restrict__ src, int n, int k, int32_t*
                 live = pass == 0 || (key >> (shift + 8)) == prefix;
             }
             const uint32_t digit = live ? ((key >> shift) & 255u) : 256u;
-            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-            if (live && lane == __ffs(peers) - 1) atomicAdd(&st.hist[digit], __popc(peers));
+            warp_hist_add(st.hist, digit, live);
         }
         __syncthreads();
         if (warp == 0) choose_digit(st);
@@ -198,7 +211,7 @@ __device__ void find_bin11(const uint32_t* hist, uint32_t k, uint32_t& d_out, ui
 // key (tau) and how many keys equal to tau fall inside the top `need`.
 template <int NT>
 __device__ void select_smem(const uint32_t* keys, int m, uint32_t need, SelectState<NT / 32>& st) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) { st.prefix = 0; st.need = need; }
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
@@ -211,8 +224,7 @@ __device__ void select_smem(const uint32_t* keys, int m, uint32_t need, SelectSt
             uint32_t key = live ? keys[j] : 0u;
             live = live && (pass == 0 || (key >> (shift + 8)) == prefix);
             const uint32_t digit = live ? ((key >> shift) & 255u) : 256u;
-            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-            if (live && lane == __ffs(peers) - 1) atomicAdd(&st.hist[digit], __popc(peers));
+            warp_hist_add(st.hist, digit, live);
         }
         __syncthreads();
         if (warp == 0) choose_digit(st);
