@@ -7,25 +7,24 @@
 // summary, es page, section 1): the k largest scores, ties to the smaller
 // position, -0.0 = +0.0; kept positions written ascending.
 //
-// The key of the k-th largest score, tau, is found as follows:
-//   1. every CTA histograms the top 11 bits of its keys (shared-memory
-//      atomics); cluster barrier; every CTA sums all CL
-//      histograms through distributed shared memory (the same sums in every
-//      CTA) and finds the bin d0 that holds the k-th largest key;
-//   2. if the whole cluster holds few keys in bin d0 (at most CAND_CAP):
-//      every CTA compacts its keys of bin d0; cluster barrier; every CTA
-//      gathers all of them and finds tau among them locally (the same
-//      deterministic result in every CTA), and from the gathered keys and
-//      the lower-ranked CTAs' counts above bin d0 where its kept positions
-//      go;
-//   3. otherwise (many keys in one bin: heavy ties) the remaining 21 bits
-//      are resolved digit by digit (11 and 10 bits), each digit's histogram
-//      reduced over the cluster slice by slice, then counted.
-// Each CTA then writes its kept positions in position order, keeping its
-// keys equal to tau after those of lower-ranked CTAs (smaller positions
-// first).  Every wait is a hardware cluster barrier that all CTAs of the
-// cluster reach in the same sequence (the path taken is decided from values
-// every CTA holds identically): no flag, no spin-wait, no global workspace.
+// The key of the k-th largest score, tau, is found digit by digit, most
+// significant first (11, 11 and 10 bits).  Each pass: every CTA histograms
+// the digit of its keys that still match the digits chosen so far (shared-
+// memory atomics); cluster barrier; every CTA sums all CL histograms through
+// distributed shared memory (the same sums in every CTA) and appends the
+// digit holding the need-th largest remaining key.  As soon as the cluster
+// holds at most CAND_CAP keys at the prefix (after 11 or 22 bits), every CTA
+// compacts its keys there; after a cluster barrier every CTA gathers all of
+// them and finds tau among them with a local radix select (the same
+// deterministic result in every CTA), and from the gathered keys and the
+// lower-ranked CTAs' counts above the prefix where its kept positions go.
+// Only when a prefix of 22 bits still holds more (heavy ties) are all 32
+// bits resolved and the per-CTA counts exchanged once more.  Each CTA then
+// writes its kept positions in position order, keeping its keys equal to
+// tau after those of lower-ranked CTAs (smaller positions first).  Every
+// wait is a hardware cluster barrier that all CTAs of the cluster reach in
+// the same sequence (the path taken is decided from values every CTA holds
+// identically): no flag, no spin-wait, no global workspace.
 #pragma once
 
 #include <cstddef>
@@ -41,26 +40,23 @@ constexpr int CAND_CAP = 2 * HBINS;   // keys of bin d0 the compaction path take
 
 template <int NW>
 struct __align__(16) ClusterSmem {
-    // this CTA's histogram of the current digit, then the cluster's reduced
-    // bins; on the compaction path both arrays together hold the gathered
-    // candidates of every CTA (CAND_CAP keys)
-    uint32_t hist[HBINS];
-    uint32_t red[HBINS];
-    uint32_t cand[CAND_CAP];            // this CTA's keys of bin d0 (compaction path)
+    // this CTA's histogram of the current digit, in hist[0] and hist[1] by
+    // turns (another CTA may still be reading the previous one); on the
+    // compaction path the two together hold the gathered candidates of
+    // every CTA (CAND_CAP keys)
+    uint32_t hist[2][HBINS];
+    uint32_t red[HBINS];                // the cluster's sums of the current digit (local)
+    uint32_t cand[CAND_CAP];            // this CTA's keys of the chosen bin (compaction path)
     SelectState<NW> st;                 // local radix select over the gathered candidates
     uint32_t warp_cnt[2][NW];
-    uint32_t slice_tot;                 // total of the reduced bins owned by this CTA
     uint32_t cnt_gt, cnt_eq;            // keys > tau and == tau in this CTA's segment
     uint32_t prefix, need;              // digits chosen so far; keys still to take at the prefix
-    uint32_t n_cand, gt0;               // this CTA's keys in bin d0, and above bin d0
-    uint32_t d0_total;                  // the cluster's keys in bin d0
+    uint32_t bin_total;                 // the cluster's keys at the prefix
+    uint32_t n_cand, gt0;               // this CTA's keys at the prefix, and above it
     uint32_t cand_off[17];              // gathered candidates: CTA c's start (c <= CL)
-    uint32_t gt_before;                 // keys above bin d0 in the lower-ranked CTAs
+    uint32_t gt_before;                 // keys above the prefix in the lower-ranked CTAs
 };
-static_assert(2 * HBINS >= CAND_CAP, "gathered candidates fit in hist + red");
-// the gathered candidates use hist and red as one array
-static_assert(offsetof(ClusterSmem<16>, red) == offsetof(ClusterSmem<16>, hist) + sizeof(uint32_t) * HBINS,
-              "hist and red are adjacent");
+static_assert(2 * HBINS >= CAND_CAP, "gathered candidates fit in the two histograms");
 
 __device__ __forceinline__ uint32_t ld_dsmem(uint32_t cluster_addr) {
     uint32_t v;
@@ -225,48 +221,61 @@ __device__ void cluster_select(ClusterSmem<NT / 32>& S, const uint32_t* keys, in
                                int32_t* __restrict__ dst, uint32_t CL, uint32_t rank) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-    // ------------------------------------------------------ top 11 bits, bin d0
-    digit_histogram<NT>(S.hist, keys, m, 0, 11, 0u);
-    cluster_barrier();   // every CTA's histogram is complete
-    // every CTA sums all CL histograms (the same sums everywhere); the CL
-    // remote loads of a bin are all in flight before they are added
-    for (int b = threadIdx.x; b < HBINS; b += NT) {
-        uint32_t v[16];
+    // ------------------------------------------------ digits, most significant first
+    // Each pass: histogram of the next digit of the keys at the prefix; every
+    // CTA sums all CL histograms (the same sums everywhere) and extends the
+    // prefix by the digit holding the need-th largest key.  As soon as the
+    // cluster holds at most CAND_CAP keys at the prefix, they are compacted.
+    uint32_t prefix = 0, need = (uint32_t)k;
+    int done = 0;
+    for (int pass = 0; pass < 3; ++pass) {
+        const int width = pass < 2 ? 11 : 10;
+        const int W = 1 << width;
+        uint32_t* local = S.hist[pass & 1];
+        digit_histogram<NT>(local, keys, m, done, width, prefix);
+        cluster_barrier();   // every CTA's histogram is complete
+        // the CL remote loads of a bin are all in flight before they are added
+        for (int b = threadIdx.x; b < W; b += NT) {
+            uint32_t v[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-            if (c < (int)CL) v[c] = ld_dsmem(map_rank(&S.hist[b], (uint32_t)c));
-        uint32_t sum = 0;
+            for (int c = 0; c < 16; ++c)
+                if (c < (int)CL) v[c] = ld_dsmem(map_rank(&local[b], (uint32_t)c));
+            uint32_t sum = 0;
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-            if (c < (int)CL) sum += v[c];
-        S.red[b] = sum;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        uint32_t d0, above;
-        warp_find_from_top(S.red, HBINS, (uint32_t)k, false, 0u, d0, above);
-        if (lane == 0) {
-            S.prefix = d0;
-            S.need = (uint32_t)k - above;          // keys still to take from bin d0
-            S.d0_total = S.red[d0];
+            for (int c = 0; c < 16; ++c)
+                if (c < (int)CL) sum += v[c];
+            S.red[b] = sum;
         }
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t d, above;
+            warp_find_from_top(S.red, W, need, false, 0u, d, above);
+            if (lane == 0) {
+                S.prefix = (prefix << width) | d;
+                S.need = need - above;           // keys still to take at the new prefix
+                S.bin_total = S.red[d];
+            }
+        }
+        __syncthreads();
+        prefix = S.prefix;
+        need = S.need;
+        done += width;
+        if (done < 32 && S.bin_total <= (uint32_t)CAND_CAP) break;   // the same in every CTA
     }
-    __syncthreads();
-    const uint32_t d0 = S.prefix;
     uint32_t tau, need_eq, out_off, eq_keep;
-
-    if (S.d0_total <= (uint32_t)CAND_CAP) {
+    if (done < 32) {
         // ----------------------------------------------- compaction path
-        // this CTA's keys of bin d0 (any order) and its count above bin d0
+        // this CTA's keys at the prefix (any order) and its count above it
+        const int sh = 32 - done;
         if (threadIdx.x == 0) S.n_cand = 0;
         __syncthreads();
         uint32_t gt0 = 0;
         const int m_round = (m + 31) & ~31;      // whole warps: ballot and shuffle take every lane
         for (int j = threadIdx.x; j < m_round; j += NT) {
             const uint32_t key = j < m ? keys[j] : 0u;
-            const uint32_t dig = key >> 21;
-            const bool cand = j < m && dig == d0;
-            gt0 += (j < m && dig > d0) ? 1u : 0u;
+            const uint32_t top = key >> sh;
+            const bool cand = j < m && top == prefix;
+            gt0 += (j < m && top > prefix) ? 1u : 0u;
             const uint32_t bal = __ballot_sync(0xffffffffu, cand);
             if (bal != 0u) {                     // the same in every lane
                 const int src = __ffs(bal) - 1;
@@ -279,7 +288,7 @@ __device__ void cluster_select(ClusterSmem<NT / 32>& S, const uint32_t* keys, in
         gt0 = block_sum<NT>(gt0, S.warp_cnt[0]);
         if (threadIdx.x == 0) S.gt0 = gt0;
         cluster_barrier();   // every CTA's candidates and counts are complete; no CTA
-                             // reads another's histogram any more
+                             // reads another's histograms any more
         if (warp == 0) {
             const uint32_t nc = lane < (int)CL ? ld_dsmem(map_rank(&S.n_cand, (uint32_t)lane)) : 0u;
             const uint32_t g0 = lane < (int)CL ? ld_dsmem(map_rank(&S.gt0, (uint32_t)lane)) : 0u;
@@ -296,8 +305,8 @@ __device__ void cluster_select(ClusterSmem<NT / 32>& S, const uint32_t* keys, in
             if (lane == 0) S.gt_before = gb;
         }
         __syncthreads();
-        // every CTA's candidates, in rank order, into this CTA's hist + red
-        uint32_t* gathered = S.hist;
+        // every CTA's candidates, in rank order, into this CTA's two histograms
+        uint32_t* gathered = &S.hist[0][0];
         const uint32_t total = S.cand_off[CL];
         for (uint32_t base = 0; base < total; base += 8u * NT) {
             uint32_t v[8];
@@ -318,8 +327,8 @@ __device__ void cluster_select(ClusterSmem<NT / 32>& S, const uint32_t* keys, in
             }
         }
         __syncthreads();
-        // tau among the gathered keys of bin d0 (identical in every CTA)
-        select_smem_known<NT>(gathered, (int)total, S.need, d0, 11, S.st);
+        // tau among the gathered keys at the prefix (identical in every CTA)
+        select_smem_known<NT>(gathered, (int)total, need, prefix, done, S.st);
         tau = S.st.prefix;
         need_eq = S.st.need;
         // keys above and equal to tau in the lower-ranked CTAs' candidates, and
@@ -337,74 +346,9 @@ __device__ void cluster_select(ClusterSmem<NT / 32>& S, const uint32_t* keys, in
         out_off = S.gt_before + gt_p + min(eq_p, need_eq);
         eq_keep = need_eq > eq_p ? min(eq_me, need_eq - eq_p) : 0u;
     } else {
-        // ----------------------------------------------- many keys in bin d0
-        cluster_barrier();   // no CTA reads another's histogram any more
-        // the remaining 21 bits, digit by digit (11 then 10 bits), each
-        // digit's histogram reduced over the cluster slice by slice
-        int done_bits = 11;
-        for (int pass = 1; pass < 3; ++pass) {
-            const int width = pass < 2 ? 11 : 10;
-            const int W = 1 << width;
-            digit_histogram<NT>(S.hist, keys, m, done_bits, width, S.prefix);
-            cluster_barrier();   // every CTA's histogram is complete
-            // reduce my slice of the bins over the cluster
-            const int per = W / (int)CL;
-            uint32_t part = 0;
-            for (int t = threadIdx.x; t < per; t += NT) {
-                const int bin = (int)rank * per + t;
-                uint32_t v[16];
-#pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    if (c < (int)CL) v[c] = ld_dsmem(map_rank(&S.hist[bin], (uint32_t)c));
-                uint32_t sum = 0;
-#pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    if (c < (int)CL) sum += v[c];
-                S.red[t] = sum;
-                part += sum;
-            }
-            part = block_sum<NT>(part, S.warp_cnt[0]);
-            if (threadIdx.x == 0) S.slice_tot = part;
-            cluster_barrier();   // every CTA's reduced slice and total are complete
-            if (warp == 0) {
-                const uint32_t need = S.need;
-                // the slice (owner CTA) holding the need-th largest key, from the top
-                uint32_t owner, above_slices;
-                {
-                    const uint32_t tot = lane < (int)CL ? ld_dsmem(map_rank(&S.slice_tot, (uint32_t)lane)) : 0u;
-                    // top-down: slice CL-1 holds the highest bins
-                    const int pos = lane;                       // top-down position
-                    const int sl = (int)CL - 1 - pos;
-                    // every lane takes part in the shuffle (a full-mask shuffle that
-                    // some lanes skip never completes); lanes past CL then drop it
-                    const uint32_t from_sl = __shfl_sync(0xffffffffu, tot, sl < 0 ? 0 : sl);
-                    const uint32_t mine = pos < (int)CL ? from_sl : 0u;
-                    uint32_t incl = mine;
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-                        if (lane >= o) incl += v;
-                    }
-                    const uint32_t hit = __ballot_sync(0xffffffffu, incl >= need && pos < (int)CL);
-                    const int p = hit ? __ffs(hit) - 1 : 0;
-                    owner = (uint32_t)((int)CL - 1 - p);
-                    above_slices = __shfl_sync(0xffffffffu, incl - mine, p);
-                }
-                uint32_t bin_in_slice, before;
-                warp_find_from_top(nullptr, per, need - above_slices, true, map_rank(&S.red[0], owner),
-                                   bin_in_slice, before);
-                if (lane == 0) {
-                    const uint32_t digit = owner * (uint32_t)per + bin_in_slice;
-                    S.prefix = (S.prefix << width) | digit;
-                    S.need = need - above_slices - before;
-                }
-            }
-            __syncthreads();
-            done_bits += width;
-        }
-        tau = S.prefix;
-        need_eq = S.need;      // keys equal to tau to keep (smallest positions first)
-        // this CTA's keys above and equal to tau
+        // ----------------------------------------------- every bit resolved (heavy ties)
+        tau = prefix;
+        need_eq = need;        // keys equal to tau to keep (smallest positions first)
         uint32_t gt = 0, eq = 0;
         for (int j = threadIdx.x; j < m; j += NT) {
             const uint32_t key = keys[j];
