@@ -158,41 +158,50 @@ __device__ __forceinline__ void digit_histogram(uint32_t* hist, const uint32_t* 
 }
 
 // Writes this CTA's kept positions (keys > tau, and the first eq_keep keys
-// equal to tau) in position order from dst[out_off].  All NT threads.
+// equal to tau) in position order from dst[out_off].  Every warp takes a
+// contiguous range of the segment: it counts its kept keys, one block-wide
+// scan of the counts gives it its offset, and it writes its keys in order
+// with warp ballots (no block barrier per chunk).  All NT threads.
 template <int NT>
 __device__ __forceinline__ void ordered_write(uint32_t (&warp_cnt)[2][NT / 32], const uint32_t* keys,
                                               int m, int s0, uint32_t tau, uint32_t out_off,
                                               uint32_t eq_keep, int32_t* __restrict__ dst) {
     constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t run_gt = 0, run_eq = 0;
+    const int per = ((m + NW - 1) / NW + 31) & ~31;          // keys per warp, whole 32-key steps
+    const int b0 = min(m, warp * per), b1 = min(m, b0 + per);
+    uint32_t ngt = 0, neq = 0;
+    for (int j0 = b0; j0 < b1; j0 += 32) {                   // the same trip count in every lane
+        const int j = j0 + lane;
+        const uint32_t key = j < b1 ? keys[j] : 0u;
+        ngt += __popc(__ballot_sync(0xffffffffu, j < b1 && key > tau));
+        neq += __popc(__ballot_sync(0xffffffffu, j < b1 && key == tau));
+    }
+    __syncthreads();                                         // warp_cnt may still be read
+    if (lane == 0) {
+        warp_cnt[0][warp] = ngt;
+        warp_cnt[1][warp] = neq;
+    }
+    __syncthreads();
+    uint32_t run_gt = 0, run_eq = 0;                         // kept keys of the lower warps
+    for (int w = 0; w < warp; ++w) {
+        run_gt += warp_cnt[0][w];
+        run_eq += warp_cnt[1][w];
+    }
     const uint32_t lt_mask = (1u << lane) - 1u;
-    const int m_round = (m + NT - 1) / NT * NT;
-    for (int base = 0; base < m_round; base += NT) {
-        const int j = base + threadIdx.x;
-        const uint32_t key = j < m ? keys[j] : 0u;
-        const bool gt = j < m && key > tau;
-        const bool eq = j < m && key == tau;
+    for (int j0 = b0; j0 < b1; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t key = j < b1 ? keys[j] : 0u;
+        const bool gt = j < b1 && key > tau;
+        const bool eq = j < b1 && key == tau;
         const uint32_t bg = __ballot_sync(0xffffffffu, gt);
         const uint32_t be = __ballot_sync(0xffffffffu, eq);
-        const int buf = (base / NT) & 1;
-        if (lane == 0) warp_cnt[buf][warp] = __popc(bg) | ((uint32_t)__popc(be) << 16);
-        __syncthreads();
-        uint32_t pre_gt = 0, pre_eq = 0, tot_gt = 0, tot_eq = 0;
-#pragma unroll
-        for (int w2 = 0; w2 < NW; ++w2) {
-            const uint32_t v = warp_cnt[buf][w2];
-            if (w2 < warp) { pre_gt += v & 0xffffu; pre_eq += v >> 16; }
-            tot_gt += v & 0xffffu;
-            tot_eq += v >> 16;
-        }
-        const uint32_t gt_before = run_gt + pre_gt + __popc(bg & lt_mask);
-        const uint32_t eq_before = run_eq + pre_eq + __popc(be & lt_mask);
+        const uint32_t gt_before = run_gt + __popc(bg & lt_mask);
+        const uint32_t eq_before = run_eq + __popc(be & lt_mask);
         if (gt || (eq && eq_before < eq_keep))
             dst[out_off + gt_before + min(eq_before, eq_keep)] = s0 + j;
-        run_gt += tot_gt;
-        run_eq += tot_eq;
-        // warp_cnt is double-buffered, so one barrier per chunk suffices
+        run_gt += __popc(bg);
+        run_eq += __popc(be);
     }
 }
 
