@@ -110,25 +110,19 @@ constexpr int OFF_X = OFF_KV + NSTAGE * KV_STAGE;   // partner's fixed-point par
 constexpr int OFF_XOFF = OFF_X + 2 * X_TILE;        // partner's per-head offset/step words
 constexpr int OFF_MASK = OFF_XOFF + 2 * X_OFF;
 constexpr int OFF_BARS = OFF_MASK + 2 * MAX_UNIT_BLOCKS * 8;
-constexpr int GW = 2;                               // gather warps
+constexpr int GW = 4;                               // gather warps
 constexpr int KPW = NB / GW;                        // key rows of a block per gather warp
-constexpr int W_Y = GW + 8, W_S = GW + 16, W_PV = GW + 17;  // first warp of each role (exchange: GW)
-constexpr int N_THREADS = 32 * (GW + 18);           // gather, 8 exchange, 8 softmax, 2 MMA warps
+constexpr int W_Y = GW + 4, W_S = GW + 8, W_PV = GW + 9;   // first warp of each role (exchange: GW)
+constexpr int N_THREADS = 32 * (GW + 10);           // gather, 4 exchange, 4 softmax, 2 MMA warps
 constexpr int KV_FULL_ARRIVALS = GW;                // one expect-tx arrival per gather warp
 static_assert(W_PV + 1 == N_THREADS / 32, "warp roles");
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t TM_O = 0;
 constexpr uint32_t TM_S = 256;                      // S/P buffer b at TM_S + 64 b
 constexpr uint32_t TM_QT = TM_S + 64 * NSBUF;       // Q_r slice 3 (32 cols) + rope (16 cols), bf16 pairs
-// per-head values the two warps of a role pair share through TMEM: block
-// extremes of the partial logits (exchange pairs, by block parity), block
-// max of the full logits (softmax pairs, by block parity), the unit's sum
-constexpr uint32_t TM_XE = TM_QT + 48;              // [parity][half][max, min]
-constexpr uint32_t TM_XM = TM_XE + 8;               // [parity][half]
-constexpr uint32_t TM_XL = TM_XM + 4;               // [half]
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_THRESHOLD = 8.f;            // log2 units
-static_assert(TM_XL + 2 <= TMEM_COLS, "tensor memory budget");
+static_assert(TM_QT + 48 <= TMEM_COLS, "tensor memory budget");
 
 struct __align__(8) AttnBars {
     uint64_t q_full, q_empty, q_tmem_full;
@@ -229,79 +223,55 @@ __device__ __forceinline__ float add_bf16x2(uint32_t p, float acc) {
     return r;
 }
 
-// largest / smallest of 32 values; smallest of those above -inf (+inf if none)
-__device__ __forceinline__ float max32(const float (&v)[32]) {
-    float mx[10];
-#pragma unroll
-    for (int x = 0; x < 10; ++x) mx[x] = max3(v[3 * x], v[3 * x + 1], v[3 * x + 2]);
-    float m = max3(v[30], v[31], mx[0]);
-#pragma unroll
-    for (int x = 1; x + 1 < 10; x += 2) m = max3(m, mx[x], mx[x + 1]);
-    return fmaxf(m, mx[9]);
-}
-__device__ __forceinline__ float min32(const float (&v)[32]) {
-    float mn[10];
-#pragma unroll
-    for (int x = 0; x < 10; ++x) mn[x] = min3(v[3 * x], v[3 * x + 1], v[3 * x + 2]);
-    float m = min3(v[30], v[31], mn[0]);
-#pragma unroll
-    for (int x = 1; x + 1 < 10; x += 2) m = min3(m, mn[x], mn[x + 1]);
-    return fminf(m, mn[9]);
-}
-__device__ __forceinline__ float min32_finite(const float (&v)[32]) {
-    float m = INFINITY;
-#pragma unroll
-    for (int c = 0; c < 32; ++c) m = fminf(m, v[c] > -INFINITY ? v[c] : INFINITY);
-    return m;
-}
-
-// This thread's (head's) own partial logits of 32 keys of an S buffer in
-// base-2 units, the keys of invalid indices (mask bits 0) set to -inf.
-__device__ __forceinline__ void own_half(uint32_t taddr, float sl2, uint32_t mask, float (&x)[32]) {
-    uint32_t r[32];
-    tmem_ld32(taddr, r);
+// This thread's (head's) own partial logits of a 64-key S buffer in base-2
+// units, the keys of invalid indices (mask bits 0) set to -inf.
+__device__ __forceinline__ void own_logits(uint32_t taddr, float sl2, const uint32_t* mask2,
+                                           float (&x)[NB]) {
+    uint32_t r0[32], r1[32];
+    tmem_ld32(taddr, r0);
+    tmem_ld32(taddr + 32, r1);
+    const uint32_t m_lo = mask2[0], m_hi = mask2[1];
     tmem_ld_wait();
 #pragma unroll
-    for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(r[c]) * sl2;
-    if (mask != 0xffffffffu) {
+    for (int c = 0; c < 32; ++c) {
+        x[c] = __uint_as_float(r0[c]) * sl2;
+        x[32 + c] = __uint_as_float(r1[c]) * sl2;
+    }
+    if ((m_lo & m_hi) != 0xffffffffu) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-            if (!((mask >> c) & 1u)) x[c] = -INFINITY;
+        for (int c = 0; c < NB; ++c)
+            if (!(((c < 32 ? m_lo : m_hi) >> (c & 31)) & 1u)) x[c] = -INFINITY;
     }
 }
 
-// One or two TMEM columns of this warp's lanes, load and wait in one step
-__device__ __forceinline__ float tmem_ld1_now(uint32_t taddr) {
-    uint32_t v;
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
-                 "tcgen05.wait::ld.sync.aligned;" : "=r"(v) : "r"(taddr) : "memory");
-    return __uint_as_float(v);
-}
-__device__ __forceinline__ float2 tmem_ld2_now(uint32_t taddr) {
-    uint32_t a, b;
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];\n\t"
-                 "tcgen05.wait::ld.sync.aligned;" : "=r"(a), "=r"(b) : "r"(taddr) : "memory");
-    return make_float2(__uint_as_float(a), __uint_as_float(b));
-}
-__device__ __forceinline__ void tmem_st2(uint32_t taddr, float a, float b) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};"
-                 ::"r"(taddr), "r"(__float_as_uint(a)), "r"(__float_as_uint(b)) : "memory");
+// largest of 64 values
+__device__ __forceinline__ float max64(const float (&v)[NB]) {
+    float mx[21];
+#pragma unroll
+    for (int x = 0; x < 21; ++x) mx[x] = max3(v[3 * x], v[3 * x + 1], v[3 * x + 2]);
+    float m = max3(mx[0], mx[1], v[63]);
+#pragma unroll
+    for (int x = 2; x + 1 < 21; x += 2) m = max3(m, mx[x], mx[x + 1]);
+    return fmaxf(m, mx[20]);
 }
 
-// The two warps of a role pair in one TMEM lane quadrant (named barrier
-// `id`, 64 threads): both arrive with their `ok`, both leave with the AND of
-// the two.  Every
-// pass through the block loop takes the same sequence of these, whatever
-// the outcome of the bounded waits in between, so neither warp can be left
-// waiting for the other.
-__device__ __forceinline__ bool pair_and(uint32_t id, bool ok) {
-    uint32_t r;
-    asm volatile("{\n\t.reg .pred p, q;\n\t"
-                 "setp.ne.u32 p, %1, 0;\n\t"
-                 "bar.red.and.pred q, %2, 64, p;\n\t"
-                 "selp.u32 %0, 1, 0, q;\n\t}"
-                 : "=r"(r) : "r"((uint32_t)ok), "r"(id) : "memory");
-    return r != 0;
+// smallest of 64 values
+__device__ __forceinline__ float min64(const float (&v)[NB]) {
+    float mn[21];
+#pragma unroll
+    for (int x = 0; x < 21; ++x) mn[x] = min3(v[3 * x], v[3 * x + 1], v[3 * x + 2]);
+    float m = min3(mn[0], mn[1], v[63]);
+#pragma unroll
+    for (int x = 2; x + 1 < 21; x += 2) m = min3(m, mn[x], mn[x + 1]);
+    return fminf(m, mn[20]);
+}
+
+// smallest of the values above -inf (+inf if there is none)
+__device__ __forceinline__ float min64_finite(const float (&v)[NB]) {
+    float m = INFINITY;
+#pragma unroll
+    for (int c = 0; c < NB; ++c) m = fminf(m, v[c] > -INFINITY ? v[c] : INFINITY);
+    return m;
 }
 
 struct AttnArgs {
@@ -381,7 +351,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
         mbar_init(&bars->q_empty, 1);
-        mbar_init(&bars->q_tmem_full, 8);
+        mbar_init(&bars->q_tmem_full, 4);
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(&bars->kv_full[s], KV_FULL_ARRIVALS);
             mbar_init(&bars->kv_empty[s], 1);
@@ -389,21 +359,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         for (int s = 0; s < NSBUF; ++s) {
             mbar_init(&bars->s_full[s], 1);
             mbar_init(&bars->s_free[s], 1);
-            mbar_init(&bars->p_full[s], 8);
-            for (int q = 0; q < 4; ++q) mbar_init(&bars->own_full[s][q], 2);
+            mbar_init(&bars->p_full[s], 4);
+            for (int q = 0; q < 4; ++q) mbar_init(&bars->own_full[s][q], 1);
         }
         for (int s = 0; s < 2; ++s) {
             for (int q = 0; q < 4; ++q) {
                 mbar_init(&bars->x_full[s][q], 1);
-                mbar_init(&bars->peer_free[s][q], 2);
+                mbar_init(&bars->peer_free[s][q], 1);
             }
             mbar_init(&bars->o_done[s], 1);
             mbar_init(&bars->info_full[s], 1);
-            mbar_init(&bars->info_empty[s], 18);
+            mbar_init(&bars->info_empty[s], 10);
             mbar_init(&bars->scan_done[s], GW);
         }
         mbar_init(&bars->o_final, 1);
-        mbar_init(&bars->o_free, 8);
+        mbar_init(&bars->o_free, 4);
         mbar_init(&bars->drain[0], 1);
         mbar_init(&bars->drain[1], 1);
         bars->abort = 0;
@@ -522,127 +492,99 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 mbar_wait_drain(&bars->kv_full[j % NSTAGE], (j / NSTAGE) & 1, 50000000ull);
         __syncwarp();
     } else if (warp < W_Y) {
-        // ------------------------------------------------------------ exchange halves
-        // Warps GW..GW+7, thread = head = TMEM lane: the two warps of a lane
-        // quadrant (w, w+4) send keys 0-31 and 32-63 of every block.
-        const int quad = warp & 3;                    // TMEM lanes 32*quad .. +31
-        const int half = (warp - GW) >> 2;            // keys 32*half .. +31 of a block
-        const int h = quad * 32 + lane;               // head of this thread
+        // ------------------------------------------------------------ exchange
+        const int quad = warp & 3;                // TMEM lanes 32*quad .. +31
+        const int h = quad * 32 + lane;           // head of this thread
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t x_remote = map_to_rank(smem_base + OFF_X + h * 128, peer);
         const uint32_t xoff_remote = map_to_rank(smem_base + OFF_XOFF + h * 4, peer);
-        const uint32_t pair_id = 1 + quad;            // named barrier of the pair
         const float sl2 = args.scale_log2;
         uint32_t g = 0;
         int n = 0;
         bool ok = true;
         for (int seq = pair; seq < args.n_units && ok; seq += n_pairs, ++n) {
-            const Unit u = decode_unit(args, seq);
             const int ip = n & 1;
-            ok = pair_and(pair_id, warp_wait(&bars->info_full[ip], (n >> 1) & 1, status, abort, 4));
-            if (!ok) break;
+            if (!warp_wait(&bars->info_full[ip], (n >> 1) & 1, status, abort, 4)) break;
             const int nb = bars->n_blocks[ip];
+            __syncwarp();
             if (nb > 0) {
-                // Q_r columns the S MMA reads from TMEM: half 0 value slice 3,
-                // half 1 the rope columns, row h, as bf16 pairs.  Every S MMA of
-                // the previous unit has finished: these warps have seen the S
-                // of its last block.
+                // Q_r columns the S MMA reads from TMEM (value slice 3 and the rope
+                // columns), row h, packed as bf16 pairs.  Every S MMA of the previous
+                // unit has finished: this warp has seen the S of its last block.
+                const Unit u = decode_unit(args, seq);
                 const __nv_bfloat16* qrow = args.q + ((int64_t)u.row * HQ + h) * KVW;
-                if (half == 0) {
-                    uint32_t qa[32];
+                uint32_t qa[32], qb[16];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint4 v = *reinterpret_cast<const uint4*>(qrow + (int)r * 256 + 192 + 8 * i);
-                        qa[4 * i] = v.x; qa[4 * i + 1] = v.y; qa[4 * i + 2] = v.z; qa[4 * i + 3] = v.w;
-                    }
-                    tmem_st32(t_lane + TM_QT, qa);
-                } else {
-                    uint32_t qb[16];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint4 v = *reinterpret_cast<const uint4*>(qrow + 512 + (int)r * 32 + 8 * i);
-                        qb[4 * i] = v.x; qb[4 * i + 1] = v.y; qb[4 * i + 2] = v.z; qb[4 * i + 3] = v.w;
-                    }
-                    tmem_st16(t_lane + TM_QT + 32, qb);
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(qrow + (int)r * 256 + 192 + 8 * i);
+                    qa[4 * i] = v.x; qa[4 * i + 1] = v.y; qa[4 * i + 2] = v.z; qa[4 * i + 3] = v.w;
                 }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(qrow + 512 + (int)r * 32 + 8 * i);
+                    qb[4 * i] = v.x; qb[4 * i + 1] = v.y; qb[4 * i + 2] = v.z; qb[4 * i + 3] = v.w;
+                }
+                tmem_st32(t_lane + TM_QT, qa);
+                tmem_st16(t_lane + TM_QT + 32, qb);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->q_tmem_full);
             }
+            // Per block: this CTA's half of the logits to the partner.  The
+            // softmax warp of the quadrant combines the two halves; this warp
+            // runs ahead of it by up to the two inbox slots.
             for (int j = 0; j < nb; ++j) {
                 const uint32_t gs = g + j;
                 const int sb = gs % NSBUF;
                 const int slot = gs & 1;
-                const uint32_t mask = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j + half];
-                // ---- this half of S(gs), its extremes shared with the other warp
-                float x[32];
-                float mb = -INFINITY, mn = INFINITY;
-                if (ok) ok = warp_wait(&bars->s_full[sb], (gs / NSBUF) & 1, status, abort, 5);
-                if (ok) {
-                    tc_fence_after();
-                    own_half(t_lane + TM_S + 64 * sb + 32 * half, sl2, mask, x);
-                    // this half of S(gs) has been read: once both halves have, the
-                    // softmax warps may overwrite it with P
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
-                    mb = max32(x);
-                    mn = min32(x);
-                    if (mn == -INFINITY) mn = min32_finite(x);      // a block with invalid keys
-                    tmem_st2(t_lane + TM_XE + 4 * slot + 2 * half, mb, mn);
-                    tmem_st_wait();
-                }
-                tc_fence_before();
-                ok = pair_and(pair_id, ok);
-                if (!ok) break;
+                if (!warp_wait(&bars->s_full[sb], (gs / NSBUF) & 1, status, abort, 5)) { ok = false; break; }
                 tc_fence_after();
-                {
-                    const float2 o = tmem_ld2_now(t_lane + TM_XE + 4 * slot + 2 * (half ^ 1));
-                    mb = fmaxf(mb, o.x);
-                    mn = fminf(mn, o.y);
-                }
+                float x[NB];
+                own_logits(t_lane + TM_S + 64 * sb, sl2, masks + ip * 2 * MAX_UNIT_BLOCKS + 2 * j, x);
+                // S(gs) has been read: the softmax warp may read it too and then
+                // overwrite it with P
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->own_full[sb][quad]);
+                // the encoding's offset and step come from the block's largest and
+                // smallest VALID partial logits (invalid keys are -inf from here on)
+                const float mb = max64(x);
+                float mn = min64(x);
+                if (mn == -INFINITY) mn = min64_finite(x);      // a block with invalid keys
                 const XCode xc = x_encoder(mb, mn);
-                // the partner's softmax warps of quadrant q must have released this
-                // inbox slot (block gs-2)
-                ok = warp_wait_cluster(&bars->peer_free[slot][quad], ((gs >> 1) & 1) ^ 1, status, abort, 6);
-                if (ok) {
-                    // row h of the partner's inbox, 16 bytes (8 keys) at a time, and
-                    // (half 0) the head's offset/step word; each st.async counts its
-                    // bytes on the partner's x_full (no fence or arrive on this side)
-                    const uint32_t xr = x_remote + slot * X_TILE;
-                    const uint32_t br = map_to_rank(smem_u32(&bars->x_full[slot][quad]), peer);
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        const int c = 4 * half + cc;
-                        st_async_v4(xr + ((c ^ (h & 7)) << 4),
-                                    x_encode2(xc, x[8 * cc + 0], x[8 * cc + 1]),
-                                    x_encode2(xc, x[8 * cc + 2], x[8 * cc + 3]),
-                                    x_encode2(xc, x[8 * cc + 4], x[8 * cc + 5]),
-                                    x_encode2(xc, x[8 * cc + 6], x[8 * cc + 7]), br);
-                    }
-                    if (half == 0) st_async_b32(xoff_remote + slot * X_OFF, xc.word, br);
+                // the partner's softmax warp q must have finished this inbox slot
+                // (block gs-2)
+                if (!warp_wait_cluster(&bars->peer_free[slot][quad], ((gs >> 1) & 1) ^ 1, status, abort, 6)) {
+                    ok = false;
+                    break;
                 }
-                // (a failed wait here ends the loop at the next pair barrier)
+                // row h of the partner's inbox, 16 bytes (8 keys) at a time, and
+                // the head's offset/step word; each st.async counts its bytes on the
+                // partner's x_full (no fence or arrive on this side)
+                const uint32_t xr = x_remote + slot * X_TILE;
+                const uint32_t br = map_to_rank(smem_u32(&bars->x_full[slot][quad]), peer);
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_async_v4(xr + ((c ^ (h & 7)) << 4),
+                                x_encode2(xc, x[8 * c + 0], x[8 * c + 1]),
+                                x_encode2(xc, x[8 * c + 2], x[8 * c + 3]),
+                                x_encode2(xc, x[8 * c + 4], x[8 * c + 5]),
+                                x_encode2(xc, x[8 * c + 6], x[8 * c + 7]), br);
+                st_async_b32(xoff_remote + slot * X_OFF, xc.word, br);
             }
             g += nb;
-            // both warps of the pair leave the unit with the same outcome
-            ok = pair_and(pair_id, ok);
+            // the unit's masks have been read: the gather warps may refill them
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->info_empty[ip]);
         }
     } else if (warp < W_S) {
-        // ------------------------------------------------------------ softmax halves
-        // Warps W_Y..W_Y+7: the two warps of a lane quadrant combine and
-        // exponentiate keys 0-31 and 32-63 of every block.
+        // ------------------------------------------------------------ softmax
         const int quad = warp & 3;
-        const int half = (warp - W_Y) >> 2;
         const int h = quad * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t free_remote0 = map_to_rank(smem_u32(&bars->peer_free[0][quad]), peer);
         const uint32_t free_remote1 = map_to_rank(smem_u32(&bars->peer_free[1][quad]), peer);
-        const uint32_t pair_id = 5 + quad;            // named barrier of the pair
-        const uint32_t t_l_mine = t_lane + TM_XL + half, t_l_other = t_lane + TM_XL + (half ^ 1);
         const float sl2 = args.scale_log2;
         uint32_t g = 0, o_use = 0;
         int n = 0;
@@ -650,69 +592,68 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         for (int seq = pair; seq < args.n_units && ok; seq += n_pairs, ++n) {
             const Unit u = decode_unit(args, seq);
             const int ip = n & 1;
-            ok = pair_and(pair_id, warp_wait(&bars->info_full[ip], (n >> 1) & 1, status, abort, 7));
-            if (!ok) break;
+            if (!warp_wait(&bars->info_full[ip], (n >> 1) & 1, status, abort, 7)) { ok = false; break; }
             const int nb = bars->n_blocks[ip];
             float m_use = 0.f;      // running max (log2 units); meaningful once m_set
             bool m_set = false;
-            float l = 0.f;          // this half's running sum of the bf16-rounded P
+            float l = 0.f;          // running sum of the bf16-rounded P
             for (int j = 0; j < nb; ++j, ++g) {
                 const int sb = g % NSBUF;
                 const int slot = g & 1;
-                const uint32_t mask = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j + half];
                 // arm this CTA's inbox slot for the partner's half of block g
-                if (half == 0 && lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD + X_OFF_QUAD);
-                float sv[32];
-                float ml = -INFINITY;
-                // S(g) is final in TMEM and both exchange warps have read it
-                if (ok) ok = warp_wait(&bars->own_full[sb][quad], (g / NSBUF) & 1, status, abort, 8);
-                if (ok) {
-                    tc_fence_after();
-                    uint32_t s0[32];
-                    tmem_ld32(t_lane + TM_S + 64 * sb + 32 * half, s0);
-                    // the partner's half of block g
-                    ok = warp_wait_cluster(&bars->x_full[slot][quad], (g >> 1) & 1, status, abort, 9);
-                    tmem_ld_wait();          // no TMEM load outlives this block
-                    if (ok) {
-                        const uint32_t ow = reinterpret_cast<const uint32_t*>(smem + OFF_XOFF + slot * X_OFF)[h];
-                        const float pm = __uint_as_float(ow << 16);
-                        const float pstep = __uint_as_float(((ow >> 16) & 0xffu) << 23);
-                        // the running max is folded into the rebuild: values relative to m_use
-                        const float cz = fmaf(8388608.f, pstep, pm - m_use);
-                        const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + slot * X_TILE + h * 128);
-                        // full logits of this half's 32 keys in base 2, minus m_use: own
-                        // half (float32) plus the partner's rebuilt half; invalid keys -inf
+                if (lane == 0) mbar_arrive_expect_tx(&bars->x_full[slot][quad], X_QUAD + X_OFF_QUAD);
+                const uint32_t m_lo = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j];
+                const uint32_t m_hi = masks[ip * 2 * MAX_UNIT_BLOCKS + 2 * j + 1];
+                // S(g) is final in TMEM and the exchange warp has read it
+                if (!warp_wait(&bars->own_full[sb][quad], (g / NSBUF) & 1, status, abort, 8)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t s0[32], s1[32];
+                tmem_ld32(t_lane + TM_S + 64 * sb, s0);
+                tmem_ld32(t_lane + TM_S + 64 * sb + 32, s1);
+                // the partner's half of block g
+                if (!warp_wait_cluster(&bars->x_full[slot][quad], (g >> 1) & 1, status, abort, 9)) {
+                    tmem_ld_wait();          // no TMEM load outlives the loop
+                    ok = false;
+                    break;
+                }
+                const uint32_t ow = reinterpret_cast<const uint32_t*>(smem + OFF_XOFF + slot * X_OFF)[h];
+                const float pm = __uint_as_float(ow << 16);
+                const float pstep = __uint_as_float(((ow >> 16) & 0xffu) << 23);
+                // the running max is folded into the rebuild: values relative to m_use
+                const float cz = fmaf(8388608.f, pstep, pm - m_use);
+                const uint4* xp = reinterpret_cast<const uint4*>(smem + OFF_X + slot * X_TILE + h * 128);
+                tmem_ld_wait();
+                // full logits of the 64 keys in base 2, minus m_use: own half (float32)
+                // plus the partner's half rebuilt from its codes; invalid keys -inf
+                float sv[NB];
 #pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) {
-                            const uint4 w4 = xp[(4 * half + cc) ^ (h & 7)];
-                            const uint32_t pw4[4] = {w4.x, w4.y, w4.z, w4.w};
+                for (int cc = 0; cc < 8; ++cc) {
+                    const uint4 w4 = xp[cc ^ (h & 7)];                 // keys 8cc .. 8cc+7
+                    const uint32_t pw4[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const float part = (e & 1) ? x_decode_hi(pw4[e >> 1], cz, pstep)
-                                                           : x_decode_lo(pw4[e >> 1], cz, pstep);
-                                sv[8 * cc + e] = fmaf(__uint_as_float(s0[8 * cc + e]), sl2, part);
-                            }
-                        }
-                        if (mask != 0xffffffffu) {
-#pragma unroll
-                            for (int c = 0; c < 32; ++c)
-                                if (!((mask >> c) & 1u)) sv[c] = -INFINITY;
-                        }
-                        // this warp's inbox values are consumed: its share of the slot
-                        // goes back to the partner (two arrivals free it)
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive_remote_relaxed(slot ? free_remote1 : free_remote0);
-                        ml = max32(sv);
-                        tmem_st1(t_lane + TM_XM + 2 * slot + half, __float_as_uint(ml));
-                        tmem_st_wait();
+                    for (int e = 0; e < 8; ++e) {
+                        const int key = 8 * cc + e;
+                        const float raw = __uint_as_float(key < 32 ? s0[key] : s1[key - 32]);
+                        const float part = (e & 1) ? x_decode_hi(pw4[e >> 1], cz, pstep)
+                                                   : x_decode_lo(pw4[e >> 1], cz, pstep);
+                        sv[key] = fmaf(raw, sl2, part);
                     }
                 }
-                tc_fence_before();
-                ok = pair_and(pair_id, ok);
-                if (!ok) break;
-                tc_fence_after();
-                const float mrel = fmaxf(ml, tmem_ld1_now(t_lane + TM_XM + 2 * slot + (half ^ 1)));  // block max - m_use
-                // ---- online softmax in base 2 (the same decisions in both warps)
+                if ((m_lo & m_hi) != 0xffffffffu) {
+#pragma unroll
+                    for (int kk = 0; kk < NB; ++kk) {
+                        const uint32_t mw = kk < 32 ? m_lo : m_hi;
+                        if (!((mw >> (kk & 31)) & 1u)) sv[kk] = -INFINITY;
+                    }
+                }
+                const float mrel = max64(sv);            // block max - m_use
+                // every inbox value of this slot has been consumed (mrel depends on
+                // all of them): hand the slot back to the partner's exchange warp
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote_relaxed(slot ? free_remote1 : free_remote0);
                 bool rescale = false;
                 float alpha = 1.f;
                 if (mrel > -INFINITY && (!m_set || mrel > RESCALE_THRESHOLD)) {
@@ -721,12 +662,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     m_use += mrel;               // the block max
                     m_set = true;
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) sv[c] -= mrel;
+                    for (int c = 0; c < NB; ++c) sv[c] -= mrel;
                 }
-                uint32_t pw[16];
+                uint32_t pw[NB / 2];
                 float ps[2] = {0.f, 0.f};
 #pragma unroll
-                for (int x = 0; x < 16; ++x) {
+                for (int x = 0; x < NB / 2; ++x) {
                     pw[x] = pack_bf16(ex2_approx(sv[2 * x]), ex2_approx(sv[2 * x + 1]));
                     ps[x & 1] = add_bf16x2(pw[x], ps[x & 1]);
                 }
@@ -734,59 +675,46 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 // The decision is per head (lane), but the O rescale below is
                 // warp-collective (the wait shuffles over the whole warp and the
                 // TMEM loads and stores are .aligned): the warp takes it when any
-                // of its heads needs it, and the other heads scale by 1.  Each
-                // warp rescales its 128 of the 256 O columns.
+                // of its heads needs it, and the other heads scale by 1.
                 if (__any_sync(0xffffffffu, rescale)) {
                     const float a = rescale ? alpha : 1.f;
-                    // O must hold P V of block g-1 before it is rescaled
-                    ok = warp_wait(&bars->o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, status, abort, 10);
-                    if (ok) {
-                        tc_fence_after();
+                    // O and l must hold P V of block g-1 before they are rescaled
+                    if (!warp_wait(&bars->o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, status, abort, 10)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
 #pragma unroll 1
-                        for (int c = 0; c < 4; ++c) {
-                            uint32_t o[32];
-                            const uint32_t ta = t_lane + TM_O + 128 * half + 32 * c;
-                            tmem_ld32(ta, o);
-                            tmem_ld_wait();
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(t_lane + TM_O + 32 * c, o);
+                        tmem_ld_wait();
 #pragma unroll
-                            for (int v = 0; v < 32; ++v) o[v] = __float_as_uint(__uint_as_float(o[v]) * a);
-                            tmem_st32(ta, o);
-                        }
+                        for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * a);
+                        tmem_st32(t_lane + TM_O + 32 * c, o);
                     }
                 }
-                if (ok) {
-                    // P of this half's keys over S (the MMA reads it from TMEM)
-                    tmem_st16(t_lane + TM_S + 64 * sb + 16 * half, pw);
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->p_full[sb]);
-                }
-                // (a failed wait here ends the loop at the next pair barrier)
+                tmem_st32(t_lane + TM_S + 64 * sb, pw);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->p_full[sb]);
             }
-            // (a loop that ended early ends the unit loop at the pair barrier
-            // below: both warps of the pair get there)
+            if (!ok) break;
             // ---------------------------------------------------------- unit epilogue
             const bool split = args.splits > 1;
             float l_all = 0.f;
             if (nb > 0) {
-                // this half's sum to the other warp; O complete
-                tmem_st1(t_l_mine, __float_as_uint(l));
-                tmem_st_wait();
-                if (ok) ok = warp_wait(&bars->o_final, o_use & 1, status, abort, 11);
-                tc_fence_before();
-                ok = pair_and(pair_id, ok);
-                if (!ok) break;
+                if (!warp_wait(&bars->o_final, o_use & 1, status, abort, 11)) { ok = false; break; }
                 tc_fence_after();
-                l_all = m_set ? l + tmem_ld1_now(t_l_other) : 0.f;
+                l_all = m_set ? l : 0.f;
                 const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
-                // this warp's 128 of the CTA's 256 output columns
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     uint32_t o[32];
-                    tmem_ld32(t_lane + TM_O + 128 * half + 32 * c, o);
+                    tmem_ld32(t_lane + TM_O + 32 * c, o);
                     tmem_ld_wait();
-                    const int col = (int)r * 256 + 128 * half + 32 * c;     // column of the output row
+                    const int col = (int)r * 256 + 32 * c;     // column of the output row
                     if (!split) {
                         uint4* dst = reinterpret_cast<uint4*>(args.out + ((int64_t)u.row * HQ + h) * DV + col);
 #pragma unroll
@@ -817,13 +745,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 if (lane == 0) mbar_arrive(&bars->o_free);
                 ++o_use;
             } else if (!split) {
-                // no valid key: this warp's 128 columns of the output row are zero
-                uint4* dst = reinterpret_cast<uint4*>(args.out + ((int64_t)u.row * HQ + h) * DV + r * 256 + 128 * half);
-                for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+                // no valid key: the output row is zero
+                uint4* dst = reinterpret_cast<uint4*>(args.out + ((int64_t)u.row * HQ + h) * DV + r * 256);
+                for (int v = 0; v < 32; ++v) dst[v] = make_uint4(0, 0, 0, 0);
             }
             // each CTA half keeps its own (m, l): the two CTAs' logits differ by
             // rounding, so their running maxima and sums may differ slightly
-            if (split && half == 0) args.part_ml[((int64_t)u.unit * 2 + r) * HQ + h] = make_float2(m_use, l_all);
+            if (split) args.part_ml[((int64_t)u.unit * 2 + r) * HQ + h] = make_float2(m_use, l_all);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->info_empty[ip]);
         }

@@ -16,11 +16,13 @@
 #ifndef IC_WAIT_LIMIT_NS
 #define IC_WAIT_LIMIT_NS 1000000000ull  // 1 s
 #endif
-// Suspend-time hint of the waiting try_wait: a waiting warp sleeps until the
-// phase completes (or this many ns pass) instead of re-issuing the poll, so
-// it leaves the issue slots to the warps doing work.  0 = no hint.
+// Suspend-time hint of the waiting try_wait (0 = none: the hardware's own
+// limit).  With a hint of 20 us a waiting warp sleeps until the phase
+// completes or the hint runs out; measured on the prefill attention (512
+// rows) the plain form was 7 % faster (0.560 against 0.599 ms), so the hint
+// is off unless a build sets it.
 #ifndef IC_WAIT_SUSPEND_NS
-#define IC_WAIT_SUSPEND_NS 20000u
+#define IC_WAIT_SUSPEND_NS 0u
 #endif
 
 namespace ic {

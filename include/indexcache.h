@@ -175,10 +175,12 @@ ic_status ic_topk(const float* scores, int64_t ld_scores, ic_rows r, int k, int3
  * with the same inputs, layouts and rules: the same indices, bit for bit
  * (the scores are computed by the same arithmetic in the same order).  For
  * decode-shaped rows (Lq <= 2, at most one row per SM, more than 4096
- * candidates) on the tensor-core shapes the two run as ONE kernel: one
- * thread-block cluster per row keeps the row's scores in shared memory and
- * selects from there, so no score row is written to memory.  Otherwise the
- * scores go through the workspace.  (IndexCache's F layer computes exactly
+ * candidates) on the tensor-core shapes, when the row clusters together
+ * cover most of the SMs, the two run as ONE kernel: one thread-block
+ * cluster per row keeps the row's scores in shared memory and selects from
+ * there, so no score row is written to memory.  Otherwise (fewer rows: the
+ * stand-alone indexer on every SM is faster) the scores go through the
+ * workspace.  (IndexCache's F layer computes exactly
  * this selection and caches it: es page, section 2 "Arquitectura del Método".)
  *   idx  [B, Lq, k] int32 (output), as ic_topk
  * Workspace: ic_indexer_topk_workspace_size.
