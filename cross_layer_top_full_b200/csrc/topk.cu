@@ -159,30 +159,31 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int Lq, int q_sta
     }
     __syncthreads();
 
-    // ---- pass 3: write the kept positions in order
+    // ---- pass 3: write the kept positions in order.  Every warp takes a
+    // contiguous range of the row: it counts its kept keys, one scan of the
+    // counts gives its offset, then it writes them in order with ballots.
+    const int per = ((n + NW - 1) / NW + 31) & ~31;          // keys per warp, whole 32-key steps
+    const int b0 = min(n, warp * per), b1 = min(n, b0 + per);
+    auto kept = [&](int j) -> bool {
+        if (j >= b1) return false;
+        const uint32_t dg = (uint32_t)hi[j] >> 5;
+        return dg > d || (dg == d && ((keep[j >> 5] >> (j & 31)) & 1u));
+    };
+    uint32_t cnt = 0;
+    for (int j0 = b0; j0 < b1; j0 += 32) cnt += __popc(__ballot_sync(0xffffffffu, kept(j0 + lane)));
+    if (lane == 0) S.warp_cnt[0][warp] = cnt;
+    __syncthreads();
     uint32_t run = 0;
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    for (int base = 0; base < n; base += NT) {
-        const int j = base + threadIdx.x;
-        bool kp = false;
-        if (j < n) {
-            const uint32_t dg = (uint32_t)hi[j] >> 5;
-            kp = dg > d || (dg == d && ((keep[j >> 5] >> (j & 31)) & 1u));
-        }
-        const uint32_t b = __ballot_sync(0xffffffffu, kp);
-        const int buf = (base / NT) & 1;
-        if (lane == 0) S.warp_cnt[buf][warp] = __popc(b);
-        __syncthreads();
-        uint32_t pre = 0, tot = 0;
 #pragma unroll
-        for (int w2 = 0; w2 < NW; ++w2) {
-            const uint32_t v = S.warp_cnt[buf][w2];
-            if (w2 < warp) pre += v;
-            tot += v;
-        }
-        if (kp) dst[run + pre + __popc(b & lt_mask)] = j;
-        run += tot;
-        // warp_cnt is double-buffered, so one barrier per chunk suffices
+    for (int w2 = 0; w2 < NW; ++w2)
+        if (w2 < warp) run += S.warp_cnt[0][w2];
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int j0 = b0; j0 < b1; j0 += 32) {
+        const int j = j0 + lane;
+        const bool kp = kept(j);
+        const uint32_t b = __ballot_sync(0xffffffffu, kp);
+        if (kp) dst[run + __popc(b & lt_mask)] = j;
+        run += __popc(b);
     }
 }
 
