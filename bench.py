@@ -265,7 +265,7 @@ def fused_selection(wl):
     library's own rule, restated."""
     T_max = wl.q_start + wl.L
     return (wl.L <= 2 and wl.idx_dtype in ("bf16", "e4m3") and wl.d_I == 128
-            and wl.H_I in (16, 32, 64, 128) and wl.B * wl.L <= 148 and T_max > wl.k
+            and wl.H_I in (16, 32, 64, 128) and 16 <= wl.B * wl.L <= 148 and T_max > wl.k
             and T_max >= 4096)
 
 

@@ -292,10 +292,14 @@ bool select_fused_applies(ic_dtype dt, int H_I, int d_I, ic_rows r, int k) {
     // (the largest head count leaves the least room for keys)
     const size_t cap = dt == IC_FP8_E4M3 ? seg_capacity<128, true>() : seg_capacity<128, false>();
     if ((size_t)((n_max + CL_MAX - 1) / CL_MAX) > cap) return false;
-    // The fused kernel scans the keys with rows x CL CTAs.  When that leaves
-    // many SMs idle (few rows: the co-resident clusters cap CL), the
-    // stand-alone indexer on every SM followed by the one-launch top-k is
-    // faster (8 rows of 200K keys: 177 us fused against 55 + 38 us).
+    // The fused kernel scans the keys with rows x CL CTAs, one row per
+    // cluster.  With few rows the co-resident clusters of the largest sizes
+    // run in more than one wave, and the stand-alone indexer on every SM
+    // followed by the one-launch top-k is faster: measured on a B200, 8 rows
+    // of 200K keys took 175 us fused against 55 + 38 us; 32 rows of 32K keys
+    // 74 us fused against 61 + 26 us.  So: at least 16 rows, and CTAs on at
+    // least 85 % of the SMs.
+    if (rows < 16) return false;
     size_t smem = 0;
     int cl = 0;
     const bool fp8 = dt == IC_FP8_E4M3;
