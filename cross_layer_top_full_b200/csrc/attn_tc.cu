@@ -28,7 +28,7 @@
 // TMEM, normalised by its own softmax sum.  No key byte is gathered twice and no flop is done
 // twice.
 //
-// Per CTA (448 threads), persistent over work units (one unit = one query
+// Per CTA (512 threads), persistent over work units (one unit = one query
 // row, or one split of a row's indices in decode):
 //   warps 0-3  gather: per unit, one batched pass over the unit's indices
 //              computes the per-block validity masks and the block count;
@@ -57,6 +57,9 @@
 //   warp 13    single-thread issue of O += P(j) V_r(j), P read from TMEM
 //              ("TS" form), as soon as P(j) is ready.  Two issuing threads
 //              keep a P V from waiting behind the gather of a later block.
+//   warps 14-15 idle (they complete the MMA warps' warpgroup, so that the
+//              gather and MMA warpgroups can hand registers to the exchange
+//              and softmax warpgroups with setmaxnreg).
 // TMEM: O at columns 0..255, three S/P buffers at 256..447, Q_r slice 3 and
 // rope columns at 448..495.  Keeping that part of Q_r in TMEM frees the
 // shared memory for a fourth KV stage.
@@ -113,9 +116,15 @@ constexpr int OFF_BARS = OFF_MASK + 2 * MAX_UNIT_BLOCKS * 8;
 constexpr int GW = 4;                               // gather warps
 constexpr int KPW = NB / GW;                        // key rows of a block per gather warp
 constexpr int W_Y = GW + 4, W_S = GW + 8, W_PV = GW + 9;   // first warp of each role (exchange: GW)
-constexpr int N_THREADS = 32 * (GW + 10);           // gather, 4 exchange, 4 softmax, 2 MMA warps
+constexpr int N_THREADS = 32 * (GW + 12);           // gather, 4 exchange, 4 softmax, 2 MMA, 2 idle warps
+// Registers per thread after the warpgroups re-balance them (setmaxnreg):
+// the gather and MMA warpgroups give theirs up to the exchange and softmax
+// warpgroups.  Launched at 128 (16 warps x 32 x 128 = 65536), the shares
+// add up to the same total: 4 x 32 x (72 + 184 + 184 + 72) = 65536.
+constexpr int REGS_SMALL = 72, REGS_LARGE = 184;
+static_assert(4 * 32 * (2 * REGS_SMALL + 2 * REGS_LARGE) == N_THREADS * 128, "register shares");
 constexpr int KV_FULL_ARRIVALS = GW;                // one expect-tx arrival per gather warp
-static_assert(W_PV + 1 == N_THREADS / 32, "warp roles");
+static_assert(W_PV + 3 == N_THREADS / 32, "warp roles");
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t TM_O = 0;
 constexpr uint32_t TM_S = 256;                      // S/P buffer b at TM_S + 64 b
@@ -386,6 +395,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
     cluster_sync();  // the partner's barriers are initialised before any remote arrive
     const uint32_t tmem = bars->tmem_base;
 
+    // Warpgroups 0 (gather) and 3 (the two MMA issuers and two idle warps)
+    // shrink to REGS_SMALL, 1 (exchange) and 2 (softmax) grow to REGS_LARGE;
+    // every warp of a warpgroup executes its group's instruction.
+    if (warp < GW) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(REGS_SMALL) : "memory");
+    else if (warp < W_S) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(REGS_LARGE) : "memory");
+    else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(REGS_SMALL) : "memory");
     if (warp < GW) {
         // ------------------------------------------------------------ gather
         const int gt = threadIdx.x;
@@ -846,7 +861,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 mbar_wait(&bars->drain[0], 0, status, abort, 20);
             }
         }
-    } else {
+    } else if (warp == W_PV) {
         // ------------------------------------------------------------ O += P V, l += P 1 issuer
         if (lane == 0) {
             constexpr uint32_t id_pv = idesc_f32acc(1, 1, HQ, 256, 0, 1);    // O += P V (V MN-major)
