@@ -207,21 +207,46 @@ __device__ __forceinline__ XCode x_encoder(float mb, float mn) {
 }
 
 // two values {lo = a, hi = b} as 16-bit codes (m - x) / step, rounded
-__device__ __forceinline__ uint32_t x_encode2(const XCode& c, float a, float b) {
-    const float ua = fmaf(a, -c.scale, c.ms) + 8388608.f;   // 2^23 + u: u in the low 16 bits
-    const float ub = fmaf(b, -c.scale, c.ms) + 8388608.f;
-    return __byte_perm(__float_as_uint(ua), __float_as_uint(ub), 0x5410);
+// Two float32 values in one 64-bit register pair, for the packed (f32x2)
+// FFMA / FADD / FMUL of sm_100: one instruction for two lanes' worth of
+// the same arithmetic, rounded exactly as two scalar operations.
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float2 f2_split(uint64_t v) {
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+    return make_float2(a, b);
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
 }
 
-// The value of the low / high code u of a packed pair, minus a constant z:
+__device__ __forceinline__ uint32_t x_encode2(const XCode& c, float a, float b) {
+    // 2^23 + u for both values (u in the low 16 bits of each)
+    const float2 u = f2_split(fadd2(ffma2(f2(a, b), f2(-c.scale, -c.scale), f2(c.ms, c.ms)),
+                                    f2(8388608.f, 8388608.f)));
+    return __byte_perm(__float_as_uint(u.x), __float_as_uint(u.y), 0x5410);
+}
+
+// The partner's value of a code u, minus a constant z (the running max):
 // m - u*step - z = cz - (2^23 + u)*step with cz = m - z + 2^23*step, the
-// float (2^23 + u) made from the code's bits directly.
-__device__ __forceinline__ float x_decode_lo(uint32_t w, float cz, float step) {
-    return fmaf(-__uint_as_float((w & 0xffffu) | 0x4b000000u), step, cz);
-}
-__device__ __forceinline__ float x_decode_hi(uint32_t w, float cz, float step) {
-    return fmaf(-__uint_as_float(__byte_perm(w, 0x4b000000u, 0x7632)), step, cz);
-}
+// float (2^23 + u) made from the code's bits directly (the softmax warps'
+// rebuild loop does two codes at a time with f32x2 FFMAs).
 
 // acc + the two bf16 values of a packed pair (each added in float32)
 __device__ __forceinline__ float add_bf16x2(uint32_t p, float acc) {
@@ -242,9 +267,13 @@ __device__ __forceinline__ void own_logits(uint32_t taddr, float sl2, const uint
     const uint32_t m_lo = mask2[0], m_hi = mask2[1];
     tmem_ld_wait();
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-        x[c] = __uint_as_float(r0[c]) * sl2;
-        x[32 + c] = __uint_as_float(r1[c]) * sl2;
+    for (int c = 0; c < 32; c += 2) {
+        const float2 a = f2_split(fmul2(f2(__uint_as_float(r0[c]), __uint_as_float(r0[c + 1])), f2(sl2, sl2)));
+        const float2 b = f2_split(fmul2(f2(__uint_as_float(r1[c]), __uint_as_float(r1[c + 1])), f2(sl2, sl2)));
+        x[c] = a.x;
+        x[c + 1] = a.y;
+        x[32 + c] = b.x;
+        x[32 + c + 1] = b.y;
     }
     if ((m_lo & m_hi) != 0xffffffffu) {
 #pragma unroll
@@ -649,12 +678,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     const uint4 w4 = xp[cc ^ (h & 7)];                 // keys 8cc .. 8cc+7
                     const uint32_t pw4[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
+                    for (int e = 0; e < 8; e += 2) {
+                        // two keys at once: the codes' floats (2^23 + u), then
+                        // cz - f*step and raw*sl2 + that, each as one f32x2 FFMA
                         const int key = 8 * cc + e;
-                        const float raw = __uint_as_float(key < 32 ? s0[key] : s1[key - 32]);
-                        const float part = (e & 1) ? x_decode_hi(pw4[e >> 1], cz, pstep)
-                                                   : x_decode_lo(pw4[e >> 1], cz, pstep);
-                        sv[key] = fmaf(raw, sl2, part);
+                        const uint32_t w = pw4[e >> 1];
+                        const uint64_t f = f2(__uint_as_float((w & 0xffffu) | 0x4b000000u),
+                                              __uint_as_float(__byte_perm(w, 0x4b000000u, 0x7632)));
+                        const uint64_t part = ffma2(f, f2(-pstep, -pstep), f2(cz, cz));
+                        const uint64_t raw = key < 32 ? f2(__uint_as_float(s0[key]), __uint_as_float(s0[key + 1]))
+                                                      : f2(__uint_as_float(s1[key - 32]), __uint_as_float(s1[key - 31]));
+                        const float2 v = f2_split(ffma2(raw, f2(sl2, sl2), part));
+                        sv[key] = v.x;
+                        sv[key + 1] = v.y;
                     }
                 }
                 if ((m_lo & m_hi) != 0xffffffffu) {
