@@ -961,42 +961,44 @@ attn_combine_kernel(const __nv_bfloat16* __restrict__ part_o, const float2* __re
     const int half = d / 256;
     // Splits are read CH at a time with every load of a chunk in flight
     // before the first is used (one memory round trip per chunk, not per
-    // split).
+    // split); the running maximum M rescales what earlier chunks added.
     constexpr int CH = 16;
     float M = -INFINITY;
-    for (int c0 = 0; c0 < splits; c0 += CH) {
-        float2 ml[CH];
-#pragma unroll
-        for (int c = 0; c < CH; ++c)
-            ml[c] = c0 + c < splits ? part_ml[((row * splits + c0 + c) * 2 + half) * HQ + h]
-                                    : make_float2(-INFINITY, 0.f);
-#pragma unroll
-        for (int c = 0; c < CH; ++c)
-            if (ml[c].y > 0.f) M = fmaxf(M, ml[c].x);
-    }
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
     float den = 0.f;
-    if (M > -INFINITY) {
-        for (int c0 = 0; c0 < splits; c0 += CH) {
-            float2 ml[CH];
-            uint2 o[CH];
+    for (int c0 = 0; c0 < splits; c0 += CH) {
+        float2 ml[CH];
+        uint2 o[CH];
 #pragma unroll
-            for (int c = 0; c < CH; ++c) {
-                const int64_t u = row * splits + c0 + c;
-                ml[c] = c0 + c < splits ? part_ml[(u * 2 + half) * HQ + h] : make_float2(-INFINITY, 0.f);
-                o[c] = c0 + c < splits ? *reinterpret_cast<const uint2*>(part_o + (u * HQ + h) * DV + d)
-                                       : make_uint2(0u, 0u);
-            }
+        for (int c = 0; c < CH; ++c) {
+            const int64_t u = row * splits + c0 + c;
+            ml[c] = c0 + c < splits ? part_ml[(u * 2 + half) * HQ + h] : make_float2(-INFINITY, 0.f);
+            o[c] = c0 + c < splits ? *reinterpret_cast<const uint2*>(part_o + (u * HQ + h) * DV + d)
+                                   : make_uint2(0u, 0u);
+        }
+        float Mc = M;
 #pragma unroll
-            for (int c = 0; c < CH; ++c) {
-                if (!(ml[c].y > 0.f)) continue;
-                const float wgt = exp2f(ml[c].x - M);
-                den += wgt * ml[c].y;
-                num.x += wgt * __uint_as_float(o[c].x << 16);
-                num.y += wgt * __uint_as_float(o[c].x & 0xffff0000u);
-                num.z += wgt * __uint_as_float(o[c].y << 16);
-                num.w += wgt * __uint_as_float(o[c].y & 0xffff0000u);
-            }
+        for (int c = 0; c < CH; ++c)
+            if (ml[c].y > 0.f) Mc = fmaxf(Mc, ml[c].x);
+        if (Mc == -INFINITY) continue;                   // nothing valid so far
+        if (Mc > M) {
+            const float a = M == -INFINITY ? 0.f : exp2f(M - Mc);
+            num.x *= a;
+            num.y *= a;
+            num.z *= a;
+            num.w *= a;
+            den *= a;
+            M = Mc;
+        }
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            if (!(ml[c].y > 0.f)) continue;
+            const float wgt = exp2f(ml[c].x - M);
+            den += wgt * ml[c].y;
+            num.x += wgt * __uint_as_float(o[c].x << 16);
+            num.y += wgt * __uint_as_float(o[c].x & 0xffff0000u);
+            num.z += wgt * __uint_as_float(o[c].y << 16);
+            num.w += wgt * __uint_as_float(o[c].y & 0xffff0000u);
         }
     }
     const float inv = den > 0.f ? 1.f / den : 0.f;
