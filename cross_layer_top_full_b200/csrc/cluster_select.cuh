@@ -10,9 +10,11 @@
 // The key of the k-th largest score, tau, is found digit by digit, most
 // significant first (11, 11 and 10 bits).  Each pass: every CTA histograms
 // the digit of its keys that still match the digits chosen so far (shared-
-// memory atomics); cluster barrier; every CTA sums all CL histograms through
-// distributed shared memory (the same sums in every CTA) and appends the
-// digit holding the need-th largest remaining key.  As soon as the cluster
+// memory atomics); cluster barrier; every CTA obtains the sums of all CL
+// histograms through distributed shared memory (the same sums in every CTA:
+// for 4 or more CTAs each first sums its own slice of the bins, and after
+// another cluster barrier every CTA reads all slices) and appends the digit
+// holding the need-th largest remaining key.  As soon as the cluster
 // holds at most CAND_CAP keys at the prefix (after 11 or 22 bits), every CTA
 // compacts its keys there; after a cluster barrier every CTA gathers all of
 // them and finds tau among them with a local radix select (the same
@@ -46,6 +48,7 @@ struct __align__(16) ClusterSmem {
     // every CTA (CAND_CAP keys)
     uint32_t hist[2][HBINS];
     uint32_t red[HBINS];                // the cluster's sums of the current digit (local)
+    uint32_t slice[HBINS / 4];          // this CTA's slice of those sums (clusters of 4 or more)
     uint32_t cand[CAND_CAP];            // this CTA's keys of the chosen bin (compaction path)
     SelectState<NW> st;                 // local radix select over the gathered candidates
     uint32_t warp_cnt[2][NW];
@@ -243,17 +246,51 @@ __device__ void cluster_select(ClusterSmem<NT / 32>& S, const uint32_t* keys, in
         uint32_t* local = S.hist[pass & 1];
         digit_histogram<NT>(local, keys, m, done, width, prefix);
         cluster_barrier();   // every CTA's histogram is complete
-        // the CL remote loads of a bin are all in flight before they are added
-        for (int b = threadIdx.x; b < W; b += NT) {
-            uint32_t v[16];
+        if (CL < 4) {
+            // every CTA sums every bin over the CL histograms; the CL remote
+            // loads of a bin are all in flight before they are added
+            for (int b = threadIdx.x; b < W; b += NT) {
+                uint32_t v[4];
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-                if (c < (int)CL) v[c] = ld_dsmem(map_rank(&local[b], (uint32_t)c));
-            uint32_t sum = 0;
+                for (int c = 0; c < 4; ++c)
+                    if (c < (int)CL) v[c] = ld_dsmem(map_rank(&local[b], (uint32_t)c));
+                uint32_t sum = 0;
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-                if (c < (int)CL) sum += v[c];
-            S.red[b] = sum;
+                for (int c = 0; c < 4; ++c)
+                    if (c < (int)CL) sum += v[c];
+                S.red[b] = sum;
+            }
+        } else {
+            // two steps, W (CL + 1) remote loads per CTA instead of W CL: CTA
+            // `rank` sums its slice of the bins over the CL histograms, then
+            // every CTA reads all CL slices
+            const int per = W / (int)CL;
+            for (int t = threadIdx.x; t < per; t += NT) {
+                const int bin = (int)rank * per + t;
+                uint32_t v[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    if (c < (int)CL) v[c] = ld_dsmem(map_rank(&local[bin], (uint32_t)c));
+                uint32_t sum = 0;
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    if (c < (int)CL) sum += v[c];
+                S.slice[t] = sum;
+            }
+            cluster_barrier();   // every CTA's slice is complete
+            for (int b0 = 0; b0 < W; b0 += 4 * NT) {
+                uint32_t v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int b = b0 + u * NT + threadIdx.x;
+                    v[u] = b < W ? ld_dsmem(map_rank(&S.slice[b % per], (uint32_t)(b / per))) : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int b = b0 + u * NT + threadIdx.x;
+                    if (b < W) S.red[b] = v[u];
+                }
+            }
         }
         __syncthreads();
         if (warp == 0) {
