@@ -25,8 +25,8 @@
 // inside the attention tolerance.  Each CTA adds its own half in float32,
 // straight from TMEM, to the partner's rebuilt half; each then runs the
 // online softmax and accumulates its own 256 value columns, O_r += P V_r, in
-// TMEM, normalised by its own softmax sum.  No key byte is gathered twice and no flop is done
-// twice.
+// TMEM, normalised by its own softmax sum.  No key byte is gathered twice
+// and no flop is done twice.
 //
 // Per CTA (512 threads), persistent over work units (one unit = one query
 // row, or one split of a row's indices in decode):
@@ -42,13 +42,15 @@
 //              from TMEM -> base 2 -> (offset, step, 16-bit codes),
 //              sent straight into the partner's inbox with st.async (counted
 //              in bytes on the partner's mbarrier); they run ahead of the
-//              softmax warps by up to the two inbox slots;
+//              softmax warps by up to the two inbox slots.  The encode, the
+//              scaling of S and the softmax warps' rebuild use packed f32x2
+//              arithmetic (two keys per instruction);
 //   warps 8-11 softmax (thread = head): own half (float32, from TMEM) + the
-//              partner's rebuilt half, row max, online softmax in base 2 with
-//              lazy rescaling (O is rescaled
-//              only when the running max grows by more than 2^8), P as bf16
-//              into TMEM over the S columns, the row sum l of the same
-//              rounded P, final normalisation and store;
+//              partner's rebuilt half (relative to the running max, folded
+//              into the rebuild), row max, online softmax in base 2 with lazy
+//              rescaling (O is rescaled only when the running max grows by
+//              more than 2^8), P as bf16 into TMEM over the S columns, the
+//              row sum l of the same rounded P, final normalisation and store;
 //   warp 12    TMEM allocation, TMA load of Q_r's value slices 0-2 (the next
 //              unit's while the current unit finishes), and single-thread
 //              issue of S(j) = Q_r K_r(j)^T (K = 288; A from shared memory for
