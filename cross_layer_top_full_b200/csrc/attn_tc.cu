@@ -425,6 +425,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
     tc_fence_after();
     cluster_sync();  // the partner's barriers are initialised before any remote arrive
     const uint32_t tmem = bars->tmem_base;
+    // everything above is on-chip; the indices, Q and the KV rows may come
+    // from the kernel before this one on the stream
+    pdl_trigger();
+    pdl_wait();
 
     // Warpgroups 0 (gather) and 3 (the two MMA issuers and two idle warps)
     // shrink to REGS_SMALL, 1 (exchange) and 2 (softmax) grow to REGS_LARGE;
@@ -957,6 +961,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
 __global__ void __launch_bounds__(128)
 attn_combine_kernel(const __nv_bfloat16* __restrict__ part_o, const float2* __restrict__ part_ml,
                     int splits, __nv_bfloat16* __restrict__ out) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t row = blockIdx.x;
     const int h = blockIdx.y;
     const int d = threadIdx.x * 4;
@@ -1159,13 +1165,17 @@ ic_status attn_tc_core(const void* q, const void* kv, const int32_t* idx, int k,
                              (int)SMEM_BYTES) != cudaSuccess)
         return cuda_error("attn_tc");
     const int64_t pairs = std::min<int64_t>(units, std::max(1, sm_count() / 2));
-    attn_tc_kernel<<<(unsigned)(2 * pairs), N_THREADS, SMEM_BYTES, s>>>(map_q, map_kv, map_kvr, a);
+    const bool pdl = pdl_rows((int64_t)r.B * r.Lq);
+    if (launch_ex(attn_tc_kernel, dim3((unsigned)(2 * pairs)), dim3(N_THREADS), SMEM_BYTES, s, pdl,
+                  0, map_q, map_kv, map_kvr, a) != cudaSuccess)
+        return cuda_error("attn_tc");
     count_launch(IC_LK_ATTN_TC);
     ic_status st = last_launch_status();
     if (st != IC_OK || a.splits <= 1) return st;
     dim3 grid((unsigned)((int64_t)r.B * r.Lq), HQ);
-    attn_combine_kernel<<<grid, 128, 0, s>>>(a.part_o, a.part_ml, a.splits,
-                                             static_cast<__nv_bfloat16*>(out));
+    if (launch_ex(attn_combine_kernel, grid, dim3(128), 0, s, pdl, 0, a.part_o, a.part_ml, a.splits,
+                  static_cast<__nv_bfloat16*>(out)) != cudaSuccess)
+        return cuda_error("attn_combine");
     count_launch(IC_LK_COMBINE);
     return last_launch_status();
 }

@@ -200,7 +200,7 @@ __host__ __device__ constexpr size_t pipeline_smem_bytes() {
 // that `sched` hands out, each finished score (causal keys only) passed to
 // sink.put.  smem: pipeline_smem_bytes<C, H>() bytes, 1024-byte aligned.
 // Allocates and frees its TMEM; ends with a CTA barrier.
-template <int H, int NTOK, bool FP8, class C, class Sched, class Sink>
+template <int H, int NTOK, bool FP8, class C, bool EARLY_TRIGGER = true, class Sched, class Sink>
 __device__ __forceinline__ void indexer_pipeline(
     const CUtensorMap* map_k_p, const CUtensorMap* map_q_p, uint8_t* smem,
     const float* __restrict__ w, const float* __restrict__ q_scale,
@@ -244,6 +244,9 @@ __device__ __forceinline__ void indexer_pipeline(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = bars->tmem_base;
+    // the keys, queries and weights may come from the stream's previous kernel
+    if (EARLY_TRIGGER) pdl_trigger();
+    pdl_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer

@@ -98,8 +98,10 @@ ic_status launch_cfg(const void* q_idx, const float* q_scale, const float* w, co
         cudaSuccess)
         return cuda_error("indexer_tc");
     const int grid = (int)std::min<int64_t>(items, sms);
-    kern<<<grid, N_THREADS, smem, s>>>(map_k, map_q, w, q_scale, k_scale, scores, ld, r.B, r.Lq,
-                                       r.q_start, r.T, wk, pg, status);
+    if (launch_ex(kern, dim3(grid), dim3(N_THREADS), smem, s, pdl_rows((int64_t)r.B * r.Lq), 0,
+                  map_k, map_q, w, q_scale, k_scale, scores, ld, r.B, r.Lq, r.q_start, r.T, wk, pg,
+                  status) != cudaSuccess)
+        return cuda_error("indexer_tc");
     count_launch(IC_LK_INDEXER_TC);
     return last_launch_status();
 }

@@ -57,6 +57,8 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int Lq, int q_sta
     uint32_t* keep = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowSmem));        // [words]
     uint16_t* hi = reinterpret_cast<uint16_t*>(keep + ((words + 3) & ~3));            // [n_max]
 
+    pdl_trigger();
+    pdl_wait();
     const int64_t row = blockIdx.x;
     const int n = row_candidates(row, Lq, q_start, seq_lens, T_max);
     const float* src = scores + row * ld;
@@ -194,6 +196,8 @@ constexpr int NT_LONG = 512;
 __global__ void __launch_bounds__(NT_LONG)
 topk_radix_kernel(const float* __restrict__ scores, int64_t ld, int Lq, int q_start, int k,
                   int32_t* __restrict__ idx, const int32_t* __restrict__ seq_lens, int T_max) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t row = blockIdx.x;
     const int n = row_candidates(row, Lq, q_start, seq_lens, T_max);
     __shared__ SelectState<NT_LONG / 32> st;
@@ -214,11 +218,13 @@ ic_status launch_topk_rows(const float* scores, int64_t ld, ic_rows r, int k, in
             cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return cuda_error("topk");
-        topk_rows_kernel<<<(unsigned)rows, NT, smem, s>>>(scores, ld, r.Lq, r.q_start, k, idx, n_max,
-                                                          seq_lens, r.T);
+        if (launch_ex(topk_rows_kernel, dim3((unsigned)rows), dim3(NT), smem, s, pdl_rows(rows), 0,
+                      scores, ld, r.Lq, r.q_start, k, idx, n_max, seq_lens, r.T) != cudaSuccess)
+            return cuda_error("topk");
     } else {
-        topk_radix_kernel<<<(unsigned)rows, NT_LONG, 0, s>>>(scores, ld, r.Lq, r.q_start, k, idx,
-                                                             seq_lens, r.T);
+        if (launch_ex(topk_radix_kernel, dim3((unsigned)rows), dim3(NT_LONG), 0, s, pdl_rows(rows),
+                      0, scores, ld, r.Lq, r.q_start, k, idx, seq_lens, r.T) != cudaSuccess)
+            return cuda_error("topk");
     }
     count_launch(IC_LK_TOPK);
     return last_launch_status();

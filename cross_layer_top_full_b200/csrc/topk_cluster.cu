@@ -33,6 +33,8 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, int Lq, int q_
     ClusterSmem<NT / 32>& S = *reinterpret_cast<ClusterSmem<NT / 32>*>(smem_raw);
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(ClusterSmem<NT / 32>));
 
+    pdl_trigger();
+    pdl_wait();
     const uint32_t CL = csel::cluster_ctas();
     const uint32_t rank = csel::cta_rank();
     const int64_t row = blockIdx.x / CL;
@@ -163,20 +165,9 @@ ic_status launch_topk_cluster(const float* scores, int64_t ld, ic_rows r, int k,
     const int64_t rows = (int64_t)r.B * r.Lq;
     const int n_max = r.q_start + r.Lq;
     const size_t smem = cluster_smem(segment(n_max, cl));
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(rows * cl), 1, 1);
-    cfg.blockDim = dim3(NT, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, ld, r.Lq, r.q_start, k, idx, seq_lens,
-                           r.T) != cudaSuccess)
+    if (launch_ex(topk_cluster_kernel, dim3((unsigned)(rows * cl)), dim3(NT), smem, s,
+                  pdl_rows(rows), (unsigned)cl, scores, ld, r.Lq, r.q_start, k, idx, seq_lens,
+                  r.T) != cudaSuccess)
         return cuda_error("topk_cluster");
     count_launch(IC_LK_TOPK);
     return last_launch_status();
