@@ -368,9 +368,32 @@ __device__ __forceinline__ void indexer_pipeline(
                     qs_w[lane] = i < Lq ? q_scale[(int64_t)b * Lq + i] : 0.f;
                 }
                 __syncwarp();
+                // Where a tile's keys live (a block-table load when paged) and this
+                // lane's key scale (FP8) are global loads that do not depend on the
+                // accumulator.  With one token per accumulator (decode) the tile
+                // epilogue is short and that latency would follow each tile's
+                // accumulator: they are issued one of this warp's tiles ahead.
+                struct TileMeta {
+                    int64_t krow0;
+                    float ks;
+                };
+                auto tile_meta = [&](int kt) -> TileMeta {
+                    TileMeta m;
+                    m.krow0 = key_row(pg, b, T, kt * BM);
+                    m.ks = 1.f;
+                    if (FP8 && kt * BM + quad * 32 + lane < Tb && m.krow0 < pg.key_rows)
+                        m.ks = k_scale[m.krow0 + quad * 32 + lane];
+                    return m;
+                };
+                constexpr bool AHEAD = C::ALT_TILES;               // this warp's tiles: every other one
+                const int kt_mine = ((int)(acc_it & 1) != group) ? kt0 + 1 : kt0;
+                TileMeta meta_next{};
+                if (AHEAD) meta_next = tile_meta(kt_mine < kt1 ? kt_mine : kt0);
                 bool ok = true;
                 for (int kt = kt0; kt < kt1; ++kt, ++acc_it) {
                     if (C::ALT_TILES && (int)(acc_it & 1) != group) continue;   // the other warpgroup's tile
+                    TileMeta meta = meta_next;
+                    if (AHEAD && kt + 2 < kt1) meta_next = tile_meta(kt + 2);
                     const int acc = acc_it % C::NACC;
                     if (!warp_wait(&bars->acc_full[acc], (acc_it / C::NACC) & 1, status, abort)) {
                         ok = false;
@@ -402,12 +425,11 @@ __device__ __forceinline__ void indexer_pipeline(
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->acc_empty[acc]);   // TMEM free again
 
+                    if (!AHEAD) meta = tile_meta(kt);
                     const int s = kt * BM + quad * 32 + lane;
-                    const int64_t krow0 = key_row(pg, b, T, kt * BM);
-                    const bool key_ok = krow0 < pg.key_rows;
+                    const bool key_ok = meta.krow0 < pg.key_rows;
                     if (!key_ok && lane == 0 && quad == 0) flag_status(status, IC_DEV_INDEX_RANGE);
-                    float ks = 1.f;
-                    if (FP8 && s < Tb && key_ok) ks = k_scale[krow0 + quad * 32 + lane];
+                    const float ks = meta.ks;
 #pragma unroll
                     for (int jj = 0; jj < C::TOK_PER_GROUP; ++jj) {
                         const int j = tok0 + jj;
