@@ -20,7 +20,12 @@
  *   - Arrays are dense, row-major, with the layouts stated per argument.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream) and never synchronise, except ic_read_status and
- *     ic_check_status.
+ *     ic_check_status.  Calls over at most 256 query rows (decode) launch
+ *     their kernels with programmatic stream serialization: a kernel may be
+ *     scheduled, and run its on-chip setup, while the previous kernel on the
+ *     stream finishes, but it touches no global memory before that kernel
+ *     has completed.  Stream order holds as for plain launches, inside CUDA
+ *     graph capture too.
  *   - Argument errors are returned before anything is launched.  A failed
  *     launch returns IC_ERR_CUDA.  Errors the kernels detect themselves (an
  *     index outside its row's causal range, a wait that ran out of time) are
