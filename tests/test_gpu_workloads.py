@@ -11,6 +11,8 @@ check covers outputs the oracle computes one by one (tests/stack_check.py):
     first and last row), indices and attention of all 12 layers.
   * prefill 8K with the FP8 indexer: indices of 512 seeded rows, attention
     on 128 of them, all 4 layers.
+The decode stack is also replayed from a captured CUDA graph, as the
+benchmark times it, and compared bit for bit with direct launches.
 Per checked row: an F layer's indices obey the top-k band rule against the
 oracle's float64 scores; an S layer's indices are the F layer's bit for bit
 (all rows); attention of EVERY sampled row is within the attention
@@ -94,6 +96,58 @@ def test_decode_b32_t32k_bf16_full_size(dev):
                                 [0], [0], range(wl.n_layers), "decode_b32")
     report("decode_b32", n_cmp, n_same)
     del inputs, outs, copies
+    torch.cuda.empty_cache()
+
+
+def test_decode_graph_replay_matches_plain_launches(dev):
+    """The decode stack as the benchmark runs it: captured once as a CUDA
+    graph (its kernels joined by programmatic launch edges, the few-row
+    calls' early launch) and replayed, against the same stack launched
+    directly: the indices and every layer's output are identical bit for
+    bit, replay after replay, and the status word stays clean."""
+    wl = synth.WORKLOADS["decode_b32_t32k_bf16"]
+    inputs = [synth.layer_inputs(wl, l, dev) for l in range(wl.n_layers)]
+    r = ic.Rows(wl.B, 1, wl.q_start, wl.T)
+    sh = ic.StackShape(r, wl.H_I, wl.d_I, DT[wl.idx_dtype], wl.k, wl.Hq, wl.d_qk, wl.d_v,
+                       DT[wl.attn_dtype], wl.d_qk, wl.d_qk if wl.latent else wl.d_v, wl.scale)
+    ws = torch.empty(ic.workspace_size(sh), dtype=torch.uint8, device=dev)
+    ic.workspace_init(ws)
+    idx_buf = torch.empty(wl.B, 1, wl.k, dtype=torch.int32, device=dev)
+    outs = [torch.empty(wl.B, 1, wl.Hq, wl.d_v, dtype=torch.bfloat16, device=dev)
+            for _ in wl.pattern]
+    layers = [dict(q_idx=x.get("q_I"), q_scale=x.get("q_scale"), w=x.get("w"), k_idx=x.get("k_I"),
+                   k_scale=x.get("k_scale"), q=x["q"], kmat=x["kv"], vmat=x["kv"], out=o)
+              for x, o in zip(inputs, outs)]
+
+    def step(stream=None):
+        ic.layer_stack_forward(wl.pattern, layers, sh, idx_buf, ws, stream=stream)
+
+    step()
+    torch.cuda.synchronize()
+    assert ic.read_status(ws) == 0
+    ref_out = [o.clone() for o in outs]
+    ref_idx = idx_buf.clone()
+
+    g = torch.cuda.CUDAGraph()
+    s_cap = torch.cuda.Stream()
+    s_cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s_cap):
+        step(s_cap)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s_cap):
+            step(s_cap)
+    torch.cuda.current_stream().wait_stream(s_cap)
+    for rep in range(3):
+        for o in outs:
+            o.zero_()
+        idx_buf.fill_(-7)
+        g.replay()
+        torch.cuda.synchronize()
+        assert ic.read_status(ws) == 0
+        assert torch.equal(idx_buf, ref_idx), "replay %d: indices differ" % rep
+        for l, (o, ro) in enumerate(zip(outs, ref_out)):
+            assert torch.equal(o, ro), "replay %d: layer %d output differs" % (rep, l)
+    del g, inputs, outs, ref_out
     torch.cuda.empty_cache()
 
 
