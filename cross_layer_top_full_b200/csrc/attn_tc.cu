@@ -958,31 +958,36 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q,
 // Merge split-k partials: out = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c,
 // with (m_c, l_c) of the CTA half that produced the columns (O_c in bf16:
 // 2^-9 relative, inside the attention tolerance).
-__global__ void __launch_bounds__(128)
+// Each thread merges 8 adjacent columns of one head (one 16-byte load per
+// split), a CTA 4 heads: grid (rows, HQ / 4) x 256 threads.  Splits are read
+// CH at a time with every load of a chunk in flight before the first is used
+// (one memory round trip per chunk, not per split); the running maximum M
+// rescales what earlier chunks added.  CH follows the split count, so that
+// few splits keep few registers and the whole grid fits on the GPU at once.
+constexpr int COMBINE_THREADS = 256;
+constexpr int COMBINE_HEADS = COMBINE_THREADS / (DV / 8);     // 4 heads per CTA
+template <int CH>
+__global__ void __launch_bounds__(COMBINE_THREADS)
 attn_combine_kernel(const __nv_bfloat16* __restrict__ part_o, const float2* __restrict__ part_ml,
                     int splits, __nv_bfloat16* __restrict__ out) {
     pdl_trigger();
     pdl_wait();
     const int64_t row = blockIdx.x;
-    const int h = blockIdx.y;
-    const int d = threadIdx.x * 4;
+    const int h = blockIdx.y * COMBINE_HEADS + (int)(threadIdx.x / (DV / 8));
+    const int d = (int)(threadIdx.x % (DV / 8)) * 8;
     const int half = d / 256;
-    // Splits are read CH at a time with every load of a chunk in flight
-    // before the first is used (one memory round trip per chunk, not per
-    // split); the running maximum M rescales what earlier chunks added.
-    constexpr int CH = 16;
     float M = -INFINITY;
-    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    float num[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     float den = 0.f;
     for (int c0 = 0; c0 < splits; c0 += CH) {
         float2 ml[CH];
-        uint2 o[CH];
+        uint4 o[CH];
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
             const int64_t u = row * splits + c0 + c;
             ml[c] = c0 + c < splits ? part_ml[(u * 2 + half) * HQ + h] : make_float2(-INFINITY, 0.f);
-            o[c] = c0 + c < splits ? *reinterpret_cast<const uint2*>(part_o + (u * HQ + h) * DV + d)
-                                   : make_uint2(0u, 0u);
+            o[c] = c0 + c < splits ? *reinterpret_cast<const uint4*>(part_o + (u * HQ + h) * DV + d)
+                                   : make_uint4(0u, 0u, 0u, 0u);
         }
         float Mc = M;
 #pragma unroll
@@ -991,10 +996,8 @@ attn_combine_kernel(const __nv_bfloat16* __restrict__ part_o, const float2* __re
         if (Mc == -INFINITY) continue;                   // nothing valid so far
         if (Mc > M) {
             const float a = M == -INFINITY ? 0.f : exp2f(M - Mc);
-            num.x *= a;
-            num.y *= a;
-            num.z *= a;
-            num.w *= a;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) num[j] *= a;
             den *= a;
             M = Mc;
         }
@@ -1003,17 +1006,21 @@ attn_combine_kernel(const __nv_bfloat16* __restrict__ part_o, const float2* __re
             if (!(ml[c].y > 0.f)) continue;
             const float wgt = exp2f(ml[c].x - M);
             den += wgt * ml[c].y;
-            num.x += wgt * __uint_as_float(o[c].x << 16);
-            num.y += wgt * __uint_as_float(o[c].x & 0xffff0000u);
-            num.z += wgt * __uint_as_float(o[c].y << 16);
-            num.w += wgt * __uint_as_float(o[c].y & 0xffff0000u);
+            const uint32_t w4[4] = {o[c].x, o[c].y, o[c].z, o[c].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                num[2 * j] += wgt * __uint_as_float(w4[j] << 16);
+                num[2 * j + 1] += wgt * __uint_as_float(w4[j] & 0xffff0000u);
+            }
         }
     }
     const float inv = den > 0.f ? 1.f / den : 0.f;
-    uint2 pk;
-    pk.x = pack_bf16(num.x * inv, num.y * inv);
-    pk.y = pack_bf16(num.z * inv, num.w * inv);
-    *reinterpret_cast<uint2*>(out + (row * HQ + h) * DV + d) = pk;
+    uint4 pk;
+    pk.x = pack_bf16(num[0] * inv, num[1] * inv);
+    pk.y = pack_bf16(num[2] * inv, num[3] * inv);
+    pk.z = pack_bf16(num[4] * inv, num[5] * inv);
+    pk.w = pack_bf16(num[6] * inv, num[7] * inv);
+    *reinterpret_cast<uint4*>(out + (row * HQ + h) * DV + d) = pk;
 }
 
 // ------------------------------------------------------------------ host side
@@ -1172,8 +1179,13 @@ ic_status attn_tc_core(const void* q, const void* kv, const int32_t* idx, int k,
     count_launch(IC_LK_ATTN_TC);
     ic_status st = last_launch_status();
     if (st != IC_OK || a.splits <= 1) return st;
-    dim3 grid((unsigned)((int64_t)r.B * r.Lq), HQ);
-    if (launch_ex(attn_combine_kernel, grid, dim3(128), 0, s, pdl, 0, a.part_o, a.part_ml, a.splits,
+    static_assert(HQ % COMBINE_HEADS == 0, "combine grid");
+    const dim3 grid((unsigned)((int64_t)r.B * r.Lq), HQ / COMBINE_HEADS);
+    auto kern = a.splits <= 2 ? attn_combine_kernel<2>
+              : a.splits <= 4 ? attn_combine_kernel<4>
+              : a.splits <= 8 ? attn_combine_kernel<8>
+                              : attn_combine_kernel<16>;
+    if (launch_ex(kern, grid, dim3(COMBINE_THREADS), 0, s, pdl, 0, a.part_o, a.part_ml, a.splits,
                   static_cast<__nv_bfloat16*>(out)) != cudaSuccess)
         return cuda_error("attn_combine");
     count_launch(IC_LK_COMBINE);
