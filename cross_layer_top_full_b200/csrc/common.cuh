@@ -55,9 +55,10 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // per step, where the early launch removes most of each kernel boundary:
 // measured on B200, 2199 -> 2125 us for the 48-layer decode step of 8
 // sequences of 200K keys.  Many-row calls do not: the same early launch made
-// the 8K prefill step 2% slower (26.28 -> 26.85 ms); the cost follows the
-// attention grid being launched while the previous kernel's CTAs drain,
-// which places its 2-CTA clusters on whichever SMs free up first.
+// the 8K prefill step 2% slower (26.28 -> 26.85 ms).  The cost appears only
+// when the attention grid is launched while the previous kernel's CTAs
+// drain, probably because its 2-CTA clusters are then placed on whichever
+// SMs free up first rather than on neighbouring ones.
 constexpr int64_t kPdlMaxRows = 256;
 inline bool pdl_rows(int64_t rows) { return IC_PDL && rows <= kPdlMaxRows; }
 
